@@ -1,0 +1,420 @@
+/*
+ * s3r_oracle.c -- plain fp64 CPU oracle of the Speed3R dual-branch sparse global attention.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE: it exists to check the CUDA library, and only the tests,
+ * the smoke check and the benchmark's CPU-baseline leg use it. It is deliberately slow and direct:
+ * every quantity is computed from its definition, in double precision, one row at a time, with no
+ * tiling, fusion or reordering beyond what the definition states. Work is spread over threads by
+ * (head, query block) only, which does not change any arithmetic.
+ *
+ * Source of the method: the gist.science summary of "Speed3R: Sparse Feed-forward 3D
+ * Reconstruction Models" (arXiv 2603.08055), "Technische samenvatting" -> "Methodologie":
+ *   §1 "Compressie-tak": spatial downsampling by average pooling; attention over the pooled
+ *      tokens yields a score matrix that identifies the relevant regions;
+ *   §1 "Selectie-tak": fine attention restricted to the top-k selection guided by those scores;
+ *   §2 "Gated Aggregation": a learned gate mixes the two branch outputs per token;
+ *   §4 "Efficient Kernel": top-k and softmax are computed together, so the scores are softmax
+ *      probabilities.
+ * Where the pages leave a step open, the reading taken is the plainest one the rest supports:
+ * 1-D blocks of b consecutive tokens of the flattened sequence, the last block partial; pooled
+ * means divide by the count of valid tokens; scores are per head; probabilities are summed over
+ * the rows of a query block that lie inside the sequence; ties in the top-k go to the lower block
+ * index; two independent sigmoid gates, one per branch.
+ *
+ * Parity status of each function (what pins it, in tests/test_oracle_pins.py):
+ *   s3r_ref_round_bf16  exhaustive comparison with the float -> bf16 definition on all halfway
+ *                       and neighbouring cases; torch's bf16 cast on random values.
+ *   s3r_ref_pool        closed forms (constant blocks, linear ramps, ragged tail).
+ *   s3r_ref_cmp         uniform-key closed form, a hand-derived worked example (tests/golden),
+ *                       row-probability sums, library attention (torch SDPA, fp64).
+ *   s3r_ref_topk        brute force over every k-subset; torch.topk on tie-free rows.
+ *   s3r_ref_sel         dense attention (torch SDPA, fp64) when k = nb; brute force per query.
+ *   s3r_ref_combine     gate limits and the zero-logit midpoint.
+ *   whole pipeline      composition of the pinned steps plus permutation invariances.
+ */
+#include "s3r_oracle.h"
+
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+/* ------------------------------------------------------------------------------------------ */
+/* scalar helpers                                                                              */
+/* ------------------------------------------------------------------------------------------ */
+
+/* bfloat16 bit pattern -> its exact value. A bf16 number is the upper half of an IEEE binary32. */
+static double bf16_value(uint16_t bits) {
+  uint32_t u = (uint32_t)bits << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+double s3r_ref_round_bf16(double x) {
+  /* bfloat16: 8 significant bits, exponent range of binary32 (normal >= 2^-126, subnormal
+   * quantum 2^-133). Round the exact double to the nearest representable value, ties to even. */
+  if (x == 0.0 || !isfinite(x)) return x;
+  int e;
+  (void)frexp(x, &e); /* x = m * 2^e with 0.5 <= |m| < 1, so the leading bit weighs 2^(e-1) */
+  int quantum_exp = (e - 1) - 7;             /* weight of the last of 8 significant bits */
+  if (quantum_exp < -133) quantum_exp = -133; /* subnormal range: fixed quantum */
+  double scaled = ldexp(x, -quantum_exp);     /* exact: only the exponent changes */
+  double r = nearbyint(scaled);               /* default rounding mode = to nearest, ties even */
+  double y = ldexp(r, quantum_exp);
+  if (fabs(y) > 3.3895313892515355e38) y = copysign(INFINITY, x); /* above the largest bf16 */
+  return y;
+}
+
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+/* ------------------------------------------------------------------------------------------ */
+/* a minimal parallel-for over independent tasks                                               */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef void (*task_fn)(void* ctx, int64_t task);
+
+typedef struct {
+  task_fn fn;
+  void* ctx;
+  int64_t ntasks;
+  int64_t next; /* accessed atomically */
+} pool_job;
+
+static void* pool_worker(void* arg) {
+  pool_job* job = (pool_job*)arg;
+  for (;;) {
+    int64_t t = __atomic_fetch_add(&job->next, 1, __ATOMIC_RELAXED);
+    if (t >= job->ntasks) break;
+    job->fn(job->ctx, t);
+  }
+  return NULL;
+}
+
+int s3r_ref_hardware_threads(void) {
+  long n = sysconf(_SC_NPROCESSORS_ONLN);
+  return n > 0 ? (int)n : 1;
+}
+
+static void parallel_for(int64_t ntasks, int threads, task_fn fn, void* ctx) {
+  pool_job job = {fn, ctx, ntasks, 0};
+  if (threads <= 0) threads = s3r_ref_hardware_threads();
+  if (threads > ntasks) threads = (int)(ntasks > 0 ? ntasks : 1);
+  if (threads <= 1) {
+    pool_worker(&job);
+    return;
+  }
+  pthread_t* tid = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)threads);
+  int started = 0;
+  for (int i = 0; i < threads; ++i) {
+    if (pthread_create(&tid[i], NULL, pool_worker, &job) != 0) break;
+    ++started;
+  }
+  if (started == 0) pool_worker(&job); /* could not start threads: run inline */
+  for (int i = 0; i < started; ++i) pthread_join(tid[i], NULL);
+  free(tid);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* argument checks shared by the entry points of this file                                     */
+/* ------------------------------------------------------------------------------------------ */
+
+static int check_params(const s3r_ref_params* p) {
+  if (!p) return -1;
+  if (p->L < 1 || p->H < 1 || p->d < 1 || p->block < 1 || p->qblock < 1) return -1;
+  return 0;
+}
+
+/* Rows of the chosen query blocks: first row and count of each, and their concatenated offset. */
+typedef struct {
+  int64_t nq;
+  int64_t* block;  /* query-block index */
+  int64_t* first;  /* first sequence row of the block */
+  int64_t* count;  /* valid rows of the block */
+  int64_t* offset; /* offset of the block's rows in the concatenated row outputs */
+  int64_t rows;    /* total rows */
+} row_map;
+
+static int row_map_make(const s3r_ref_params* p, const int64_t* qblocks, int64_t nq, row_map* m) {
+  int64_t nqb = ceil_div(p->L, p->qblock);
+  if (!qblocks) nq = nqb;
+  if (nq < 0) return -1;
+  m->nq = nq;
+  m->block = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nq + 1));
+  m->first = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nq + 1));
+  m->count = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nq + 1));
+  m->offset = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nq + 1));
+  int64_t off = 0;
+  for (int64_t i = 0; i < nq; ++i) {
+    int64_t qb = qblocks ? qblocks[i] : i;
+    if (qb < 0 || qb >= nqb) {
+      free(m->block), free(m->first), free(m->count), free(m->offset);
+      return -2;
+    }
+    int64_t first = qb * p->qblock;
+    int64_t last = first + p->qblock < p->L ? first + p->qblock : p->L;
+    m->block[i] = qb;
+    m->first[i] = first;
+    m->count[i] = last - first;
+    m->offset[i] = off;
+    off += last - first;
+  }
+  m->rows = off;
+  return 0;
+}
+
+static void row_map_free(row_map* m) {
+  free(m->block), free(m->first), free(m->count), free(m->offset);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* compression branch, step 1: block mean pooling                                              */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+  const s3r_ref_params* p;
+  const uint16_t* x;
+  double* out;
+} pool_ctx;
+
+static void pool_task(void* vctx, int64_t j) {
+  const pool_ctx* c = (const pool_ctx*)vctx;
+  const s3r_ref_params* p = c->p;
+  const int64_t HD = (int64_t)p->H * p->d;
+  int64_t t0 = j * p->block;
+  int64_t t1 = t0 + p->block < p->L ? t0 + p->block : p->L;
+  double n = (double)(t1 - t0);
+  for (int64_t e = 0; e < HD; ++e) {
+    double sum = 0.0;
+    for (int64_t t = t0; t < t1; ++t) sum += bf16_value(c->x[t * HD + e]);
+    double mean = sum / n;
+    c->out[j * HD + e] = p->exact_pool ? mean : s3r_ref_round_bf16(mean);
+  }
+}
+
+int s3r_ref_pool(const s3r_ref_params* p, const uint16_t* x, double* out) {
+  if (check_params(p) || !x || !out) return -1;
+  pool_ctx c = {p, x, out};
+  parallel_for(ceil_div(p->L, p->block), p->threads, pool_task, &c);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* compression branch, step 2: attention over block summaries and the block score matrix       */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+  const s3r_ref_params* p;
+  const uint16_t* q;
+  const double* kc;
+  const double* vc;
+  const row_map* rm;
+  double* lse;
+  double* o_cmp;
+  double* scores;
+} cmp_ctx;
+
+static void cmp_task(void* vctx, int64_t task) {
+  const cmp_ctx* c = (const cmp_ctx*)vctx;
+  const s3r_ref_params* p = c->p;
+  const row_map* rm = c->rm;
+  const int64_t nb = ceil_div(p->L, p->block);
+  const int64_t H = p->H, d = p->d, HD = H * d;
+  const int64_t h = task / rm->nq, i = task % rm->nq;
+  double* s = (double*)malloc(sizeof(double) * (size_t)nb);
+  double* score_row = c->scores ? c->scores + (h * rm->nq + i) * nb : NULL;
+  if (score_row)
+    for (int64_t j = 0; j < nb; ++j) score_row[j] = 0.0;
+
+  for (int64_t r = 0; r < rm->count[i]; ++r) {
+    const int64_t t = rm->first[i] + r;   /* sequence row */
+    const int64_t out_r = rm->offset[i] + r;
+    const uint16_t* qrow = c->q + t * HD + h * d;
+    /* logits s_j = scale * <q, K~_j> for every block summary j */
+    double m = -INFINITY;
+    for (int64_t j = 0; j < nb; ++j) {
+      const double* krow = c->kc + j * HD + h * d;
+      double dot = 0.0;
+      for (int64_t e = 0; e < d; ++e) dot += bf16_value(qrow[e]) * krow[e];
+      s[j] = p->scale * dot;
+      if (s[j] > m) m = s[j];
+    }
+    /* log-sum-exp over all nb summaries (no mask: the partial tail block is a normal summary) */
+    double l = 0.0;
+    for (int64_t j = 0; j < nb; ++j) l += exp(s[j] - m);
+    const double lse = m + log(l);
+    if (c->lse) c->lse[h * rm->rows + out_r] = lse;
+    /* probabilities, the compressed output, and the per-query-block column sums (scores) */
+    double* orow = c->o_cmp ? c->o_cmp + out_r * HD + h * d : NULL;
+    if (orow)
+      for (int64_t e = 0; e < d; ++e) orow[e] = 0.0;
+    for (int64_t j = 0; j < nb; ++j) {
+      const double pj = exp(s[j] - lse);
+      if (orow) {
+        const double* vrow = c->vc + j * HD + h * d;
+        for (int64_t e = 0; e < d; ++e) orow[e] += pj * vrow[e];
+      }
+      if (score_row) score_row[j] += pj;
+    }
+  }
+  free(s);
+}
+
+int s3r_ref_cmp(const s3r_ref_params* p, const uint16_t* q, const double* kc, const double* vc,
+                const int64_t* qblocks, int64_t nq, double* lse, double* o_cmp, double* scores) {
+  if (check_params(p) || !q || !kc || !vc) return -1;
+  row_map rm;
+  int rc = row_map_make(p, qblocks, nq, &rm);
+  if (rc) return rc;
+  cmp_ctx c = {p, q, kc, vc, &rm, lse, o_cmp, scores};
+  parallel_for((int64_t)p->H * rm.nq, p->threads, cmp_task, &c);
+  row_map_free(&rm);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* per-row top-k                                                                               */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+  double score;
+  int64_t index;
+} scored;
+
+/* order: larger score first; equal scores -> lower index first */
+static int scored_cmp(const void* a, const void* b) {
+  const scored* x = (const scored*)a;
+  const scored* y = (const scored*)b;
+  if (x->score > y->score) return -1;
+  if (x->score < y->score) return 1;
+  return (x->index > y->index) - (x->index < y->index);
+}
+
+typedef struct {
+  int64_t n;
+  int32_t k;
+  const double* scores;
+  int32_t* idx;
+  double* gap;
+} topk_ctx;
+
+static void topk_task(void* vctx, int64_t r) {
+  const topk_ctx* c = (const topk_ctx*)vctx;
+  scored* a = (scored*)malloc(sizeof(scored) * (size_t)c->n);
+  for (int64_t j = 0; j < c->n; ++j) {
+    a[j].score = c->scores[r * c->n + j];
+    a[j].index = j;
+  }
+  qsort(a, (size_t)c->n, sizeof(scored), scored_cmp);
+  for (int32_t t = 0; t < c->k; ++t) c->idx[r * c->k + t] = (int32_t)a[t].index;
+  if (c->gap) c->gap[r] = c->k < c->n ? a[c->k - 1].score - a[c->k].score : INFINITY;
+  free(a);
+}
+
+int s3r_ref_topk(int64_t rows, int64_t n, int32_t k, const double* scores, int32_t* idx,
+                 double* gap) {
+  if (rows < 0 || n < 1 || k < 1 || k > n || !scores || !idx) return -1;
+  topk_ctx c = {n, k, scores, idx, gap};
+  parallel_for(rows, 0, topk_task, &c);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* selection branch: exact attention over the union of the selected key blocks                 */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+  const s3r_ref_params* p;
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const row_map* rm;
+  const int32_t* idx;
+  double* o_sel;
+  int bad_index; /* set when an index is out of range */
+} sel_ctx;
+
+static void sel_task(void* vctx, int64_t task) {
+  sel_ctx* c = (sel_ctx*)vctx;
+  const s3r_ref_params* p = c->p;
+  const row_map* rm = c->rm;
+  const int64_t nb = ceil_div(p->L, p->block);
+  const int64_t H = p->H, d = p->d, HD = H * d;
+  const int64_t h = task / rm->nq, i = task % rm->nq;
+  const int32_t* sel = c->idx + (h * rm->nq + i) * p->topk;
+
+  /* the token set T: every token of every selected block, each block once, tokens < L */
+  char* chosen = (char*)calloc((size_t)nb, 1);
+  int64_t* tokens = (int64_t*)malloc(sizeof(int64_t) * (size_t)p->topk * (size_t)p->block);
+  int64_t nt = 0;
+  for (int32_t s = 0; s < p->topk; ++s) {
+    int64_t j = sel[s];
+    if (j < 0 || j >= nb) {
+      c->bad_index = 1;
+      continue;
+    }
+    if (chosen[j]) continue;
+    chosen[j] = 1;
+    for (int64_t t = j * p->block; t < (j + 1) * p->block && t < p->L; ++t) tokens[nt++] = t;
+  }
+  double* s = (double*)malloc(sizeof(double) * (size_t)(nt > 0 ? nt : 1));
+
+  for (int64_t r = 0; r < rm->count[i]; ++r) {
+    const int64_t t_q = rm->first[i] + r;
+    const uint16_t* qrow = c->q + t_q * HD + h * d;
+    double* orow = c->o_sel + (rm->offset[i] + r) * HD + h * d;
+    double m = -INFINITY;
+    for (int64_t a = 0; a < nt; ++a) {
+      const uint16_t* krow = c->k + tokens[a] * HD + h * d;
+      double dot = 0.0;
+      for (int64_t e = 0; e < d; ++e) dot += bf16_value(qrow[e]) * bf16_value(krow[e]);
+      s[a] = p->scale * dot;
+      if (s[a] > m) m = s[a];
+    }
+    double l = 0.0;
+    for (int64_t a = 0; a < nt; ++a) l += exp(s[a] - m);
+    for (int64_t e = 0; e < d; ++e) orow[e] = 0.0;
+    for (int64_t a = 0; a < nt; ++a) {
+      const double w = exp(s[a] - m) / l;
+      const uint16_t* vrow = c->v + tokens[a] * HD + h * d;
+      for (int64_t e = 0; e < d; ++e) orow[e] += w * bf16_value(vrow[e]);
+    }
+  }
+  free(s);
+  free(tokens);
+  free(chosen);
+}
+
+int s3r_ref_sel(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                const int64_t* qblocks, int64_t nq, const int32_t* idx, double* o_sel) {
+  if (check_params(p) || !q || !k || !v || !idx || !o_sel || p->topk < 1) return -1;
+  row_map rm;
+  int rc = row_map_make(p, qblocks, nq, &rm);
+  if (rc) return rc;
+  sel_ctx c = {p, q, k, v, &rm, idx, o_sel, 0};
+  parallel_for((int64_t)p->H * rm.nq, p->threads, sel_task, &c);
+  row_map_free(&rm);
+  return c.bad_index ? -3 : 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* gated aggregation                                                                           */
+/* ------------------------------------------------------------------------------------------ */
+
+int s3r_ref_combine(int64_t n, int32_t H, int32_t d, const double* o_cmp, const double* o_sel,
+                    const float* gates, double* out) {
+  if (n < 0 || H < 1 || d < 1 || !o_cmp || !o_sel || !gates || !out) return -1;
+  for (int64_t r = 0; r < n; ++r)
+    for (int64_t h = 0; h < H; ++h) {
+      const double g_cmp = sigmoid((double)gates[(r * H + h) * 2 + 0]);
+      const double g_sel = sigmoid((double)gates[(r * H + h) * 2 + 1]);
+      for (int64_t e = 0; e < d; ++e) {
+        const int64_t at = (r * H + h) * d + e;
+        out[at] = g_cmp * o_cmp[at] + g_sel * o_sel[at];
+      }
+    }
+  return 0;
+}

@@ -1,0 +1,85 @@
+/*
+ * s3r_oracle.h -- plain fp64 CPU oracle of the Speed3R dual-branch sparse global attention.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE. Only the test-suite, the smoke check and the benchmark's
+ * CPU-baseline leg load this library. It shares no code, header, table or helper with the CUDA
+ * library under sparse_global_attention_s3r_b200/csrc.
+ *
+ * Method (Speed3R, "Technische samenvatting" -> "Methodologie" of the gist.science summary of
+ * arXiv 2603.08055, §1 "Compressie-tak" / "Selectie-tak" and §2 "Gated Aggregation"):
+ *   compression branch: K and V are mean-pooled over blocks of b tokens; every query attends to the
+ *     block summaries; the softmax probabilities form the score matrix that ranks key blocks;
+ *   selection branch: per query block, exact attention over the tokens of the top-k key blocks;
+ *   gated aggregation: the two branch outputs are mixed by per-token, per-head sigmoid gates.
+ *
+ * Conventions (all arrays dense, row-major):
+ *   Q, K, V      [L, H, d]   bf16, passed as their raw 16-bit patterns (uint16_t)
+ *   pooled K/V   [nb, H, d]  double          nb  = ceil(L / block)
+ *   gates        [L, H, 2]   float           [...,0] compression gate logit, [...,1] selection
+ *   lse          [H, R]      double          R = rows of the chosen query blocks (see below)
+ *   o_cmp, o_sel [R, H, d]   double
+ *   scores       [H, nq, nb] double          nq = number of chosen query blocks
+ *   idx          [H, nq, k]  int32
+ * A call may restrict the query side to a list of query-block indices ("sampled mode"); its row
+ * outputs are then the rows of those blocks, concatenated in list order. A NULL list means every
+ * query block 0 .. ceil(L / qblock) - 1.
+ *
+ * Every function returns 0 on success and a negative value on a bad argument; nothing is printed.
+ */
+#ifndef S3R_ORACLE_H
+#define S3R_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct {
+  int64_t L;        /* tokens in the flattened sequence (N views x P tokens per view), >= 1 */
+  int32_t H;        /* heads */
+  int32_t d;        /* head dimension */
+  int32_t block;    /* b: key-block size of the pooling and of the selection unit */
+  int32_t qblock;   /* rows per query block over which probabilities are summed */
+  int32_t topk;     /* k: key blocks selected per query block, 1 <= k <= nb */
+  double scale;     /* softmax scale applied to q.k in both branches */
+  int32_t exact_pool; /* 0: pooled K/V are rounded to bf16 (RNE) like a tensor-core operand;
+                         1: keep the exact fp64 mean (used by the closed-form checks) */
+  int32_t threads;  /* worker threads, 0 = all online cores */
+} s3r_ref_params;
+
+/* Number of cores the oracle uses when params.threads == 0. */
+int s3r_ref_hardware_threads(void);
+
+/* Round a double to the nearest bfloat16 value (ties to even), returned as a double. */
+double s3r_ref_round_bf16(double x);
+
+/* Compression branch, step 1: block means of x over the valid tokens of each block.
+ * out[j,h,c] = (1/n_j) sum_{t in block j, t < L} x[t,h,c], n_j = number of valid tokens. */
+int s3r_ref_pool(const s3r_ref_params* p, const uint16_t* x, double* out);
+
+/* Compression branch, step 2: attention of each chosen query row to all nb block summaries,
+ * and the block score matrix (sum of the row probabilities over each query block).
+ * Any of lse, o_cmp, scores may be NULL. */
+int s3r_ref_cmp(const s3r_ref_params* p, const uint16_t* q, const double* kc, const double* vc,
+                const int64_t* qblocks, int64_t nq, double* lse, double* o_cmp, double* scores);
+
+/* Per-row top-k of a [rows, n] score matrix: the k largest, in descending score order, equal
+ * scores by lower index. gap[r] = k-th largest minus (k+1)-th largest (+inf when k == n).
+ * gap may be NULL. */
+int s3r_ref_topk(int64_t rows, int64_t n, int32_t k, const double* scores, int32_t* idx,
+                 double* gap);
+
+/* Selection branch: exact softmax attention of each chosen query row over the tokens of the k
+ * key blocks idx[h, i, :] of its query block (tokens >= L excluded). */
+int s3r_ref_sel(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                const int64_t* qblocks, int64_t nq, const int32_t* idx, double* o_sel);
+
+/* Gated aggregation over n rows: out = sigmoid(g[...,0]) * o_cmp + sigmoid(g[...,1]) * o_sel. */
+int s3r_ref_combine(int64_t n, int32_t H, int32_t d, const double* o_cmp, const double* o_sel,
+                    const float* gates, double* out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,473 @@
+"""Pins of the fp64 CPU oracle to facts that do not come from the oracle itself.
+
+Each test checks one oracle function against a closed form, an invariant, brute force over every
+candidate, or a library routine (torch SDPA / topk / bf16 cast, all on CPU in fp64), chosen so that
+a plausible slip in the oracle (a dropped term, a wrong index, a swapped operand, a tail divided by
+the wrong count) fails at least one of them. tests/test_oracle_mutants.py plants such slips and
+checks that they are caught.
+
+Method: gist.science summary of "Speed3R: Sparse Feed-forward 3D Reconstruction Models",
+"Technische samenvatting" -> "Methodologie" §1 (compression branch: average pooling and a score
+matrix; selection branch: fine attention on the top-k) and §2 (gated aggregation).
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import oracle as O
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+# --------------------------------------------------------------------------------------------
+# helpers (value <-> bf16 bits; none of them implements a step of the method)
+# --------------------------------------------------------------------------------------------
+
+def bits_of(x) -> np.ndarray:
+    """bf16 bit patterns of values that are exactly representable in bf16 (asserted)."""
+    a = torch.as_tensor(np.asarray(x, dtype=np.float32))
+    b = a.to(torch.bfloat16)
+    assert torch.equal(b.float(), a), "test value not representable in bf16"
+    return O.bf16_bits(b)
+
+
+def values_of(bits: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+
+
+def rand_bits(shape, seed, scale=None):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(shape, generator=g, dtype=torch.float32)
+    if scale is not None:
+        x = x * scale
+    return O.bf16_bits(x.to(torch.bfloat16))
+
+
+def sdpa64(q, k, v, scale, mask=None):
+    """torch SDPA in fp64 on [L, H, d] arrays -> [L, H, dv]."""
+    tq = torch.from_numpy(np.ascontiguousarray(q)).double().permute(1, 0, 2)[None]
+    tk = torch.from_numpy(np.ascontiguousarray(k)).double().permute(1, 0, 2)[None]
+    tv = torch.from_numpy(np.ascontiguousarray(v)).double().permute(1, 0, 2)[None]
+    m = None if mask is None else torch.from_numpy(mask)
+    o = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=m, scale=scale)
+    return o[0].permute(1, 0, 2).numpy()
+
+
+# --------------------------------------------------------------------------------------------
+# bf16 rounding
+# --------------------------------------------------------------------------------------------
+
+def test_round_bf16_matches_library_cast_on_floats():
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(4000, generator=g) * torch.exp2(torch.randint(-40, 40, (4000,), generator=g))
+    # constructed halfway and near-halfway float32 patterns
+    hi = torch.randint(0, 1 << 15, (3000,), generator=g, dtype=torch.int64) << 16
+    lows = torch.tensor([0x8000, 0x7FFF, 0x8001, 0x0000, 0xFFFF], dtype=torch.int64)
+    pats = (hi[:, None] | lows[None, :]).reshape(-1)
+    pats = pats[(pats >> 23) & 0xFF != 0xFF]  # finite only
+    y = pats.to(torch.int32).view(torch.float32)
+    allx = torch.cat([x, y])
+    want = allx.to(torch.bfloat16).double().numpy()
+    got = np.array([O.round_bf16(float(v)) for v in allx.tolist()])
+    np.testing.assert_array_equal(got, want)
+
+
+def test_round_bf16_rounds_the_exact_double_once():
+    # just above / below the halfway point between 1 and 1 + 2^-7: a float32 round trip would
+    # land exactly on the tie and round to even (1.0) in both cases
+    assert O.round_bf16(1 + 2**-8 + 2**-40) == 1 + 2**-7
+    assert O.round_bf16(1 + 2**-8 - 2**-40) == 1.0
+    assert O.round_bf16(1 + 2**-8) == 1.0  # tie -> even
+    assert O.round_bf16(1 + 3 * 2**-8) == 1 + 2**-6  # tie -> even
+    assert O.round_bf16(-(1 + 3 * 2**-8)) == -(1 + 2**-6)
+    # subnormal range: quantum 2^-133
+    assert O.round_bf16(2.0**-134) == 0.0
+    assert O.round_bf16(3 * 2.0**-134) == 2.0**-132
+    assert O.round_bf16(5 * 2.0**-135) == 2.0**-133
+
+
+# --------------------------------------------------------------------------------------------
+# pooling (compression branch, average pooling)
+# --------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("L,b", [(200, 64), (256, 64), (97, 32), (300, 128), (1, 64)])
+def test_pool_constant_blocks(L, b):
+    H, d = 2, 8
+    nb = -(-L // b)
+    rng = np.random.default_rng(L + b)
+    const = rng.integers(-64, 64, size=(nb, H, d)) / 8.0  # bf16-exact
+    x = np.repeat(const, b, axis=0)[:L]
+    pb = O.Problem(L, H, d, b, 1)
+    for exact in (True, False):
+        np.testing.assert_array_equal(O.pool(pb, bits_of(x), exact=exact), const)
+
+
+@pytest.mark.parametrize("L,b", [(200, 64), (97, 32), (300, 128), (129, 128)])
+def test_pool_linear_ramp_gives_midpoint_of_valid_tokens(L, b):
+    H, d = 3, 4
+    t = np.arange(L)
+    # value = position inside the block + 10*e + 100*h: integers, exact in bf16 up to 256
+    x = (t % b)[:, None, None] + 10.0 * np.arange(d)[None, None, :] + 0.0 * np.arange(H)[None, :, None]
+    x = x + 40.0 * np.arange(H)[None, :, None]
+    pb = O.Problem(L, H, d, b, 1)
+    got = O.pool(pb, bits_of(x), exact=True)
+    nb = -(-L // b)
+    for j in range(nb):
+        n = min(b, L - j * b)
+        want = (n - 1) / 2.0 + 10.0 * np.arange(d)[None, :] + 40.0 * np.arange(H)[:, None]
+        np.testing.assert_array_equal(got[j], want)
+    # rounded mode: the exact mean rounded once to bf16 (a library cast of the exact float32 value)
+    got_r = O.pool(pb, bits_of(x), exact=False)
+    want_r = torch.from_numpy(got.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(got_r, want_r)
+
+
+def test_pool_rounded_is_within_half_ulp_of_exact():
+    L, H, d, b = 333, 2, 16, 64
+    x = rand_bits((L, H, d), 5, scale=0.125)
+    pb = O.Problem(L, H, d, b, 1)
+    ex = O.pool(pb, x, exact=True)
+    rd = O.pool(pb, x, exact=False)
+    # bf16 representable
+    np.testing.assert_array_equal(
+        torch.from_numpy(rd).float().to(torch.bfloat16).double().numpy(), rd)
+    ulp = np.exp2(np.floor(np.log2(np.abs(ex) + 1e-300)) - 7)
+    assert np.all(np.abs(rd - ex) <= 0.5 * ulp * (1 + 1e-12))
+
+
+# --------------------------------------------------------------------------------------------
+# compression branch: attention to block summaries and the score matrix
+# --------------------------------------------------------------------------------------------
+
+def _setup(L, H, d, b, k, seed, qscale=None):
+    pb = O.Problem(L, H, d, b, k)
+    s = 1 / math.sqrt(d) if qscale is None else qscale
+    q = rand_bits((L, H, d), seed, s)
+    kk = rand_bits((L, H, d), seed + 1, 1 / math.sqrt(d))
+    v = rand_bits((L, H, d), seed + 2, 1 / math.sqrt(d))
+    return pb, q, kk, v
+
+
+@pytest.mark.parametrize("L,b,k", [(1000, 64, 4), (1024, 64, 4), (500, 32, 3)])
+def test_cmp_uniform_keys_closed_form(L, b, k):
+    """All keys equal: every summary equals that key, so p = 1/nb, lse = s + log nb,
+    o_cmp = mean of the pooled V, scores tie at rows/nb and the top-k is 0..k-1."""
+    H, d = 2, 16
+    pb = O.Problem(L, H, d, b, k)
+    kappa = values_of(rand_bits((H, d), 3, 0.5))
+    kk = bits_of(np.broadcast_to(kappa, (L, H, d)))
+    q = rand_bits((L, H, d), 4, 0.5)
+    v = rand_bits((L, H, d), 5, 0.5)
+    kc = O.pool(pb, kk)
+    vc = O.pool(pb, v)
+    lse, o_cmp, scores = O.cmp_attn(pb, q, kc, vc)
+    qv = values_of(q)
+    s = pb.softmax_scale * np.einsum("lhd,hd->hl", qv, kappa)
+    np.testing.assert_allclose(lse, s + math.log(pb.nb), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o_cmp, np.broadcast_to(vc.mean(axis=0), o_cmp.shape), atol=1e-14)
+    rows = np.array([min(64, L - 64 * i) for i in range(pb.nqb)], np.float64)
+    np.testing.assert_allclose(scores, np.broadcast_to((rows / pb.nb)[None, :, None], scores.shape),
+                               rtol=1e-13)
+    idx, gap = O.topk(scores, k)
+    np.testing.assert_array_equal(idx, np.broadcast_to(np.arange(k), idx.shape))
+
+
+def test_cmp_two_level_keys_closed_form():
+    """Summaries are kappa on a set A of blocks and 0 elsewhere: p_A = e^s / (|A| e^s + nb - |A|)."""
+    L, H, d, b, k = 700, 2, 8, 64, 3
+    pb = O.Problem(L, H, d, b, k)
+    nb = pb.nb
+    A = [1, 4, 5, 10]  # includes the ragged last block (10)
+    kappa = values_of(rand_bits((H, d), 7, 1.0))
+    x = np.zeros((L, H, d))
+    for j in A:
+        x[j * b:(j + 1) * b] = kappa
+    q = rand_bits((L, H, d), 8, 0.7)
+    v = rand_bits((L, H, d), 9, 0.5)
+    kc = O.pool(pb, bits_of(x))
+    vc = O.pool(pb, v)
+    lse, o_cmp, scores = O.cmp_attn(pb, q, kc, vc)
+    s = pb.softmax_scale * np.einsum("lhd,hd->hl", values_of(q), kappa)  # [H, L]
+    Z = len(A) * np.exp(s) + (nb - len(A))
+    pA, p0 = np.exp(s) / Z, 1.0 / Z
+    np.testing.assert_allclose(lse, np.log(Z), atol=1e-12)
+    inA = np.zeros(nb, bool)
+    inA[A] = True
+    want_o = (pA.T[:, :, None] * vc[inA].sum(0)[None] + p0.T[:, :, None] * vc[~inA].sum(0)[None])
+    np.testing.assert_allclose(o_cmp, want_o, atol=1e-14)
+    want_s = np.zeros((H, pb.nqb, nb))
+    for i in range(pb.nqb):
+        r = slice(64 * i, min(L, 64 * i + 64))
+        want_s[:, i, :] = np.where(inA[None, :], pA[:, r].sum(1)[:, None], p0[:, r].sum(1)[:, None])
+    np.testing.assert_allclose(scores, want_s, rtol=1e-13)
+
+
+def test_cmp_scores_sum_to_rows_of_each_query_block():
+    L, H, d, b = 1000, 2, 64, 64
+    pb, q, kk, v = _setup(L, H, d, b, 4, 21)
+    _, _, scores = O.cmp_attn(pb, q, O.pool(pb, kk), O.pool(pb, v))
+    rows = np.array([min(64, L - 64 * i) for i in range(pb.nqb)], np.float64)
+    np.testing.assert_allclose(scores.sum(-1), np.broadcast_to(rows, (H, pb.nqb)), rtol=1e-13)
+
+
+@pytest.mark.parametrize("L,b", [(1000, 64), (777, 32), (900, 128)])
+def test_cmp_matches_library_attention_fp64(L, b):
+    """o_cmp = SDPA(q, K~, V~); SDPA(q, K~, I) returns the probability matrix itself, whose
+    query-block sums are the scores and whose first column fixes lse = s_q0 - log p_q0."""
+    H, d = 2, 64
+    pb, q, kk, v = _setup(L, H, d, b, 4, 31, qscale=1.0)  # larger logits than the workload
+    kc, vc = O.pool(pb, kk), O.pool(pb, v)
+    lse, o_cmp, scores = O.cmp_attn(pb, q, kc, vc)
+    qv = values_of(q)
+    np.testing.assert_allclose(o_cmp, sdpa64(qv, kc, vc, pb.softmax_scale), rtol=0, atol=1e-13)
+    eye = np.broadcast_to(np.eye(pb.nb)[:, None, :], (pb.nb, H, pb.nb))
+    P = sdpa64(qv, kc, eye, pb.softmax_scale)  # [L, H, nb]
+    for i in range(pb.nqb):
+        np.testing.assert_allclose(scores[:, i, :], P[64 * i:64 * i + 64].sum(0), rtol=1e-11,
+                                   atol=1e-15)
+    s0 = pb.softmax_scale * np.einsum("lhd,hd->hl", qv, kc[0])
+    np.testing.assert_allclose(lse, s0 - np.log(P[:, :, 0].T), atol=1e-11)
+
+
+def test_cmp_sampled_blocks_equal_full_run():
+    L, H, d, b = 1000, 2, 32, 64
+    pb, q, kk, v = _setup(L, H, d, b, 4, 41)
+    kc, vc = O.pool(pb, kk), O.pool(pb, v)
+    lse, o, sc = O.cmp_attn(pb, q, kc, vc)
+    pick = [15, 3, 0]  # includes the ragged last query block
+    lse2, o2, sc2 = O.cmp_attn(pb, q, kc, vc, qblocks=pick)
+    rows = pb.rows_of(pick)
+    np.testing.assert_array_equal(lse2, lse[:, rows])
+    np.testing.assert_array_equal(o2, o[rows])
+    np.testing.assert_array_equal(sc2, sc[:, pick])
+
+
+# --------------------------------------------------------------------------------------------
+# per-query-block top-k
+# --------------------------------------------------------------------------------------------
+
+def test_topk_equals_best_subset_by_brute_force():
+    """The top-k set maximises the score sum over all k-subsets; among equal sums the
+    lexicographically smallest index tuple (= lower index first on ties). Integer-valued scores
+    make every sum exact and ties frequent."""
+    rng = np.random.default_rng(0)
+    n = 9
+    for trial in range(60):
+        row = rng.integers(0, 4, size=n).astype(np.float64)
+        for k in range(1, n + 1):
+            best = max(itertools.combinations(range(n), k),
+                       key=lambda c: (sum(row[list(c)]), tuple(-x for x in c)))
+            idx, gap = O.topk(row[None], k)
+            assert sorted(idx[0].tolist()) == list(best), (row, k)
+            # order: descending score, ties by lower index
+            order = sorted(best, key=lambda j: (-row[j], j))
+            assert idx[0].tolist() == order
+            srt = np.sort(row)[::-1]
+            want_gap = math.inf if k == n else srt[k - 1] - srt[k]
+            assert gap[0] == want_gap
+
+
+def test_topk_matches_library_topk_without_ties():
+    g = torch.Generator().manual_seed(3)
+    s = torch.rand(40, 300, generator=g, dtype=torch.float64)
+    for k in (1, 7, 32, 300):
+        idx, _ = O.topk(s.numpy(), k)
+        want = torch.topk(s, k, dim=-1, sorted=True).indices.numpy()
+        np.testing.assert_array_equal(idx, want)
+
+
+# --------------------------------------------------------------------------------------------
+# selection branch
+# --------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("L,b", [(1000, 64), (777, 32), (900, 128)])
+def test_sel_with_every_block_equals_dense_library_attention(L, b):
+    H, d = 2, 64
+    pb0, q, kk, v = _setup(L, H, d, b, 1, 51, qscale=1.0)
+    pb = O.Problem(L, H, d, b, pb0.nb)
+    idx = np.broadcast_to(np.arange(pb.nb, dtype=np.int32), (H, pb.nqb, pb.nb))
+    o = O.sel_attn(pb, q, kk, v, idx)
+    want = sdpa64(values_of(q), values_of(kk), values_of(v), pb.softmax_scale)
+    np.testing.assert_allclose(o, want, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("L,b,k", [(1000, 64, 4), (777, 32, 5), (900, 128, 2)])
+def test_sel_matches_library_attention_under_block_mask(L, b, k):
+    """Arbitrary distinct selections, the ragged last block included: SDPA with a boolean mask
+    that admits exactly the tokens of the selected blocks of each query's block."""
+    H, d = 2, 64
+    pb, q, kk, v = _setup(L, H, d, b, k, 61, qscale=1.0)
+    rng = np.random.default_rng(k)
+    idx = np.stack([np.stack([rng.permutation(pb.nb)[:k] for _ in range(pb.nqb)])
+                    for _ in range(H)]).astype(np.int32)
+    idx[:, -1, 0] = pb.nb - 1 if (pb.nb - 1) not in idx[:, -1, 1:] else idx[:, -1, 0]
+    o = O.sel_attn(pb, q, kk, v, idx)
+    qv, kv, vv = values_of(q), values_of(kk), values_of(v)
+    for h in range(H):
+        mask = np.zeros((L, L), bool)
+        for i in range(pb.nqb):
+            for j in idx[h, i]:
+                mask[64 * i:64 * i + 64, j * b:min(L, j * b + b)] = True
+        want = sdpa64(qv[:, h:h + 1], kv[:, h:h + 1], vv[:, h:h + 1], pb.softmax_scale, mask[None, None])
+        np.testing.assert_allclose(o[:, h:h + 1], want, rtol=0, atol=1e-13)
+
+
+def test_sel_block_order_and_duplicates_do_not_matter():
+    L, H, d, b, k = 640, 1, 32, 64, 3
+    pb, q, kk, v = _setup(L, H, d, b, k, 71)
+    idx = np.array([[[2, 5, 7]] * pb.nqb], np.int32)
+    a = O.sel_attn(pb, q, kk, v, idx)
+    b_ = O.sel_attn(pb, q, kk, v, idx[:, :, ::-1].copy())
+    np.testing.assert_allclose(a, b_, atol=1e-15)
+    dup = np.array([[[2, 5, 5]] * pb.nqb], np.int32)
+    two = O.Problem(L, H, d, b, 2)
+    c = O.sel_attn(pb, q, kk, v, dup)
+    e = O.sel_attn(two, q, kk, v, np.array([[[2, 5]] * pb.nqb], np.int32))
+    np.testing.assert_allclose(c, e, atol=1e-15)
+
+
+# --------------------------------------------------------------------------------------------
+# gated aggregation
+# --------------------------------------------------------------------------------------------
+
+def test_combine_gate_limits_and_midpoint():
+    rng = np.random.default_rng(1)
+    a = rng.standard_normal((50, 3, 8))
+    b = rng.standard_normal((50, 3, 8))
+    z = np.zeros((50, 3, 2), np.float32)
+    np.testing.assert_allclose(O.combine(a, b, z), 0.5 * (a + b), rtol=1e-15)
+    lim = np.zeros_like(z)
+    lim[..., 0], lim[..., 1] = -60, 60
+    np.testing.assert_allclose(O.combine(a, b, lim), b, rtol=1e-15, atol=1e-25)
+    lim[..., 0], lim[..., 1] = 60, -60
+    np.testing.assert_allclose(O.combine(a, b, lim), a, rtol=1e-15, atol=1e-25)
+    # the two gates are independent: both open -> the plain sum
+    lim[..., 0], lim[..., 1] = 60, 60
+    np.testing.assert_allclose(O.combine(a, b, lim), a + b, rtol=1e-15)
+
+
+# --------------------------------------------------------------------------------------------
+# the worked example (tests/golden/worked_example.json)
+# --------------------------------------------------------------------------------------------
+
+def test_worked_example():
+    with open(os.path.join(HERE, "golden", "worked_example.json")) as f:
+        ex = json.load(f)
+    p = ex["problem"]
+    pb = O.Problem(p["L"], p["H"], p["d"], p["block"], p["topk"], qblock=p["qblock"], scale=p["scale"])
+    inp = ex["inputs"]
+    q = bits_of(np.array(inp["q"], np.float64)[:, None, :])
+    k = bits_of(np.array(inp["k"], np.float64)[:, None, :])
+    v = bits_of(np.array(inp["v"], np.float64)[:, None, :])
+    gates = np.array(inp["gates"], np.float32)[:, None, :]
+    r = O.sparse_attn(pb, q, k, v, gates)
+    e = ex["expected"]
+    np.testing.assert_array_equal(r.kc[:, 0], e["pooled_k"])
+    np.testing.assert_array_equal(r.vc[:, 0], e["pooled_v"])
+    s = np.array(e["logits"], np.float64)
+    P = np.exp(s) / np.exp(s).sum(1, keepdims=True)
+    np.testing.assert_allclose(r.lse[0], np.log(np.exp(s).sum(1)), atol=1e-15)
+    np.testing.assert_allclose(r.o_cmp[:, 0], P @ np.array(e["pooled_v"], np.float64), atol=1e-15)
+    want_scores = np.stack([P[0] + P[1], P[2] + P[3], P[4]])
+    np.testing.assert_allclose(r.scores[0], want_scores, atol=1e-15)
+    np.testing.assert_array_equal(r.idx[0], e["idx"])
+    np.testing.assert_allclose(r.o_sel[:, 0], e["o_sel"], atol=1e-15)
+    np.testing.assert_allclose(r.out[:, 0], 0.5 * (r.o_cmp[:, 0] + np.array(e["o_sel"])), atol=1e-15)
+
+
+# --------------------------------------------------------------------------------------------
+# invariances of the whole path
+# --------------------------------------------------------------------------------------------
+
+def _pipeline(pb, q, k, v, gates):
+    return O.sparse_attn(pb, q, k, v, gates)
+
+
+def _gates(L, H, seed):
+    return torch.randn((L, H, 2), generator=torch.Generator().manual_seed(seed)).numpy()
+
+
+def test_invariance_tokens_permuted_within_key_blocks():
+    """Re-ordering tokens inside every key block (K and V together; on the multi-view layout,
+    the order of the views' patches inside a block) changes nothing but summation order."""
+    L, H, d, b, k = 1000, 2, 64, 64, 4
+    pb, q, kk, v = _setup(L, H, d, b, k, 81, qscale=0.6)
+    gates = _gates(L, H, 1)
+    rng = np.random.default_rng(2)
+    perm = np.concatenate([j * b + rng.permutation(min(b, L - j * b)) for j in range(pb.nb)])
+    r0 = _pipeline(pb, q, kk, v, gates)
+    r1 = _pipeline(pb, q, kk[perm].copy(), v[perm].copy(), gates)
+    np.testing.assert_array_equal(r0.kc, r1.kc)
+    np.testing.assert_array_equal(r0.vc, r1.vc)
+    np.testing.assert_allclose(r0.scores, r1.scores, rtol=1e-13)
+    sep = r0.gap > 1e-9
+    np.testing.assert_array_equal(np.sort(r0.idx, -1)[sep], np.sort(r1.idx, -1)[sep])
+    np.testing.assert_allclose(r0.out, r1.out, atol=1e-13)
+
+
+def test_invariance_queries_permuted_within_query_blocks():
+    L, H, d, b, k = 1000, 2, 64, 64, 4
+    pb, q, kk, v = _setup(L, H, d, b, k, 91, qscale=0.6)
+    gates = _gates(L, H, 2)
+    rng = np.random.default_rng(3)
+    perm = np.concatenate([i * 64 + rng.permutation(min(64, L - i * 64)) for i in range(pb.nqb)])
+    r0 = _pipeline(pb, q, kk, v, gates)
+    r1 = _pipeline(pb, q[perm].copy(), kk, v, gates[perm].copy())
+    np.testing.assert_allclose(r1.scores, r0.scores, rtol=1e-13)
+    sep = r0.gap > 1e-9
+    np.testing.assert_array_equal(np.sort(r0.idx, -1)[sep], np.sort(r1.idx, -1)[sep])
+    np.testing.assert_allclose(r1.out, r0.out[perm], atol=1e-13)
+    np.testing.assert_allclose(r1.lse, r0.lse[:, perm], atol=1e-13)
+
+
+def test_invariance_key_blocks_permuted():
+    """Moving whole key blocks permutes the score columns and relabels the selection; the
+    outputs do not change."""
+    L, H, d, b, k = 1024, 2, 64, 64, 4
+    pb, q, kk, v = _setup(L, H, d, b, k, 101, qscale=0.6)
+    gates = _gates(L, H, 3)
+    rng = np.random.default_rng(4)
+    pi = rng.permutation(pb.nb)  # new block pi[j] holds old block j
+    tok = np.empty(L, np.int64)
+    for j in range(pb.nb):
+        tok[pi[j] * b:(pi[j] + 1) * b] = np.arange(j * b, (j + 1) * b)
+    r0 = _pipeline(pb, q, kk, v, gates)
+    r1 = _pipeline(pb, q, kk[tok].copy(), v[tok].copy(), gates)
+    np.testing.assert_allclose(r1.scores[:, :, pi], r0.scores, rtol=1e-13)
+    sep = r0.gap > 1e-9
+    np.testing.assert_array_equal(np.sort(pi[r0.idx], -1)[sep], np.sort(r1.idx, -1)[sep])
+    np.testing.assert_allclose(r1.out, r0.out, atol=1e-13)
+
+
+def test_heads_are_independent():
+    L, H, d, b, k = 700, 3, 32, 64, 3
+    pb, q, kk, v = _setup(L, H, d, b, k, 111, qscale=0.8)
+    gates = _gates(L, H, 4)
+    full = _pipeline(pb, q, kk, v, gates)
+    one = O.Problem(L, 1, d, b, k)
+    for h in range(H):
+        r = _pipeline(one, q[:, h:h + 1].copy(), kk[:, h:h + 1].copy(), v[:, h:h + 1].copy(),
+                      gates[:, h:h + 1].copy())
+        np.testing.assert_array_equal(r.idx[0], full.idx[h])
+        np.testing.assert_array_equal(r.out[:, 0], full.out[:, h])
+
+
+def test_scale_applies_to_both_branches():
+    """(q, scale) and (2q, scale/2) give the same logits exactly, hence identical outputs."""
+    L, H, d, b, k = 600, 2, 32, 64, 3
+    pb, q, kk, v = _setup(L, H, d, b, k, 121, qscale=0.5)
+    gates = _gates(L, H, 5)
+    q2 = bits_of(2 * values_of(q))
+    a = O.sparse_attn(O.Problem(L, H, d, b, k, scale=0.3), q, kk, v, gates)
+    c = O.sparse_attn(O.Problem(L, H, d, b, k, scale=0.15), q2, kk, v, gates)
+    np.testing.assert_array_equal(a.idx, c.idx)
+    np.testing.assert_array_equal(a.out, c.out)
+    # and the scale matters: a different scale changes the compressed output
+    e = O.sparse_attn(O.Problem(L, H, d, b, k, scale=0.6), q, kk, v, gates)
+    assert np.abs(e.o_cmp - a.o_cmp).max() > 1e-6
