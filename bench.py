@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse global attention path (s3r_sparse_attn_fwd) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload n1000] [--impl native|reference]
+
+One step = one call of the whole path (pooling, compressed attention and scores, top-k,
+selection attention with the gated combine) over one layer of synthetic inputs already resident
+in HBM. Default workload: the 1000-view sequence, L = 1,374,000 tokens (N = 1000 views x P = 1374
+tokens), H = 16, d = 64, b = 64, top-k = 32. Each GPU runs its own independent layer (weak
+scaling, no data-path collective); the step time is the maximum over ranks.
+
+Prints one JSON line (rank 0): tokens/s, algorithmic TFLOP/s and fraction of the measured bf16
+peak, per-stage times from CUDA events recorded inside the fused call, the roofline of the
+dominant kernel, an end-to-end figure through pinned host buffers, the fp64 CPU oracle's timed
+sample, the kernel-launch count and the SM clocks sampled during the timed region.
+
+--impl reference times the CPU oracle (the only other implementation of this method) on bounded
+samples of the same workload and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    "n1000": dict(desc="1000-view sequence: N=1000 views x P=1374 tokens (37x37 patches + 5), "
+                       "L=1,374,000, H=16, d=64, b=64, top-k=32, 1 layer",
+                  L=1374000, H=16, block=64, topk=32, seed=3),
+    "n100": dict(desc="100-view layer: L=137,400, H=16, d=64, b=64, top-k=32",
+                 L=137400, H=16, block=64, topk=32, seed=2),
+    "vggt32": dict(desc="VGGT-like layer: N=32 views x P=1374, L=43,968, H=16, d=64, b=64, top-k=16",
+                   L=43968, H=16, block=64, topk=16, seed=1),
+    "tiny": dict(desc="tiny: N=4 x P=256, L=1024, H=2, d=64, b=64, top-k=4",
+                 L=1024, H=2, block=64, topk=4, seed=0),
+}
+
+METRIC = "sparse global-attn tokens/s at 1000 views"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    p = dict(FALLBACK_PEAKS)
+    p["source"] = "fallback"
+    return p
+
+
+def algorithmic(cfg):
+    """Algorithmic work per call: FLOPs of Q.Kc^T + P.Vc (once) and of the selection's
+    Q.K^T + P.V over the tokens actually selected; bytes of each stage's compulsory traffic."""
+    L, H, d, b, k, nb, nqb = cfg.L, cfg.H, cfg.d, cfg.block, cfg.topk, cfg.nb, cfg.nqb
+    # tokens selected per query block: k full blocks, except that the ragged last block (if it is
+    # selected) is shorter; count it as a full block less the tail (upper bound when unselected)
+    sel_tokens = k * b
+    cmp_flops = 4.0 * L * nb * d * H
+    sel_flops = 4.0 * L * sel_tokens * d * H
+    return {
+        "cmp_flops": cmp_flops,
+        "sel_flops": sel_flops,
+        "flops": cmp_flops + sel_flops,
+        "stage_work": {
+            "pool": ("hbm", 2.0 * (L + nb) * H * d * 2),                       # bytes
+            "cmp_lse": ("tensor", 2.0 * L * nb * d * H),                       # flops (Q.Kc^T)
+            "cmp_pv_score": ("tensor", cmp_flops),                            # flops
+            "topk": ("hbm", H * nqb * (nb * 4.0 + k * 4.0)),                  # bytes
+            "sel_combine": ("tensor", sel_flops),                             # flops
+        },
+    }
+
+
+def physical_gpu(local: int) -> str:
+    """nvidia-smi's name for CUDA device `local` of this process."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if vis:
+        return vis.split(",")[local].strip()
+    return str(local)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# the CPU oracle, timed on a bounded sample of the workload
+# ---------------------------------------------------------------------------------------------
+
+def oracle_sample(cfg, host_bits, gates_np, n_blocks: int, seed: int):
+    """Time the oracle: pooling of all K/V plus the whole path for n_blocks query blocks (all
+    heads). Returns (tokens/s extrapolated to the full layer, seconds, description, threads)."""
+    import numpy as np
+
+    from oracle import oracle as O
+
+    pb = O.Problem(cfg.L, cfg.H, cfg.d, cfg.block, cfg.topk)
+    rng = np.random.default_rng(seed)
+    blocks = sorted(set(rng.choice(cfg.nqb - 1, size=max(0, min(n_blocks, cfg.nqb) - 1),
+                                   replace=False).tolist()
+                        if cfg.nqb > 1 else []) | {cfg.nqb - 1})
+    q, k, v = host_bits
+    t0 = time.perf_counter()
+    kc = O.pool(pb, k)
+    vc = O.pool(pb, v)
+    t1 = time.perf_counter()
+    O.sparse_attn(pb, q, k, v, gates_np, qblocks=blocks, pooled=(kc, vc))
+    t2 = time.perf_counter()
+    rows = int(pb.rows_of(blocks).size)
+    t_full = (t1 - t0) + (t2 - t1) * cfg.L / rows
+    desc = (f"pooling of all {cfg.nb} K/V blocks + the whole path for {len(blocks)} seeded query "
+            f"blocks ({rows} rows, all {cfg.H} heads); extrapolated to L={cfg.L}")
+    return cfg.L / t_full, t2 - t0, desc, O.hardware_threads()
+
+
+def run_reference(args, wl):
+    """--impl reference: the CPU oracle on bounded samples; rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    from oracle import oracle as O
+    from sparse_global_attention_s3r_b200 import api, synth
+
+    cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"])
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = synth.make_inputs(cfg.L, cfg.H, cfg.d, cfg.block, wl["seed"], device=dev)
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    gates = x.gates.cpu().numpy()
+    del x
+    n_blocks = max(1, min(4, cfg.nqb))
+    for w in range(args.warmup):
+        oracle_sample(cfg, bits, gates, n_blocks, seed=w)
+    vals, secs = [], []
+    desc = threads = None
+    for s in range(args.steps):
+        v, t, desc, threads = oracle_sample(cfg, bits, gates, n_blocks, seed=100 + s)
+        vals.append(v)
+        secs.append(t)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * cfg.L / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl["desc"], "L": cfg.L, "H": cfg.H, "d": cfg.d,
+                   "block": cfg.block, "topk": cfg.topk, "qblock": 64, "seed": wl["seed"]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": desc + f"; median of {args.steps} samples of "
+                                          f"{statistics.median(secs):.1f} s"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------------------------
+
+def run_native(args, wl):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from sparse_global_attention_s3r_b200 import _lib, api, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl native")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"])
+    seed = wl["seed"] + 1000 * rank  # an independent layer per GPU
+    x = synth.make_inputs(cfg.L, cfg.H, cfg.d, cfg.block, seed, device=dev)
+    q, k, v, gates = x.q, x.k, x.v, x.gates
+    sa = api.SparseAttention(cfg, dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        sa(q, k, v, gates)
+    torch.cuda.synchronize()
+
+    stage_ev = [api.StageEvents() for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(physical_gpu(local)) as clocks:
+        time.sleep(0.3)
+        n0 = _lib.kernel_launches()
+        start.record()
+        for s in range(args.steps):
+            api.sparse_attn_fwd(cfg, q, k, v, gates, sa.workspace, sa.out, sa.idx,
+                                stage_events=stage_ev[s])
+        end.record()
+        torch.cuda.synchronize()
+        launches = _lib.kernel_launches() - n0
+    barrier()
+    ms = start.elapsed_time(end) / args.steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    stage_ms = {n: statistics.mean(e.stage_ms()[n] for e in stage_ev) for n in _lib.STAGES}
+
+    # end to end through pinned host buffers: H2D of the step's inputs, the call, D2H of out
+    host = [t_.cpu().pin_memory() for t_ in (q, k, v, gates)]
+    out_h = torch.empty(sa.out.shape, dtype=sa.out.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, 3))
+    sa.from_host(*host, out_h)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        sa.from_host(*host, out_h)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+    h2d = sum(t_.numel() * t_.element_size() for t_ in host)
+    d2h = out_h.numel() * out_h.element_size()
+    del host, out_h
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import oracle as O
+
+        bits = [O.bf16_bits(t_) for t_ in (q, k, v)]
+        val, secs, desc, threads = oracle_sample(cfg, bits, gates.cpu().numpy(),
+                                                 args.oracle_blocks, seed=7)
+        cpu = {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": desc + f"; {secs:.1f} s of CPU work"}
+        del bits
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = load_peaks()
+    work = algorithmic(cfg)
+    tokens_per_s = cfg.L * world / (ms_max / 1e3)
+    tflops = work["flops"] * world / (ms_max / 1e3) / 1e12
+    dom = max(stage_ms, key=stage_ms.get)
+    bound, units = work["stage_work"][dom]
+    dom_s = stage_ms[dom] / 1e3
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": units / dom_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": units / dom_s / 1e12,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["peak_source"] = peaks["source"] + (" sustained bf16" if bound == "tensor" else " copy")
+    stages = {}
+    for n in _lib.STAGES:
+        b_, u_ = work["stage_work"][n]
+        s_ = stage_ms[n] / 1e3
+        stages[n] = {"ms": stage_ms[n],
+                     ("GB/s" if b_ == "hbm" else "TFLOP/s"): u_ / s_ / (1e9 if b_ == "hbm" else 1e12)}
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl["desc"], "L": cfg.L, "H": cfg.H, "d": cfg.d, "block": cfg.block,
+                   "topk": cfg.topk, "qblock": 64, "seed": wl["seed"],
+                   "parallelism": "independent layer per GPU" if world > 1 else "single GPU",
+                   "l2": "inputs exceed L2 (each of Q/K/V is %.2f GB > 126 MB); no flush" %
+                         (q.numel() * 2 / 1e9)},
+        "tflops": tflops,
+        "frac_bf16_peak": tflops / world / peaks["bf16_tflops"],
+        "frac_bf16_peak_sustained": tflops / world / peaks["bf16_tflops_sustained"],
+        "stage_ms": stages,
+        "roofline": roof,
+        "e2e": {"value": cfg.L * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "cpu_baseline": cpu,
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="n1000")
+    ap.add_argument("--oracle-blocks", type=int, default=8,
+                    help="query blocks in the timed CPU-oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_native(args, wl)
+
+
+if __name__ == "__main__":
+    main()

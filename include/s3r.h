@@ -1,0 +1,180 @@
+/*
+ * s3r.h -- C ABI of the B200 (sm_100a) sparse global attention library, libs3r.so.
+ *
+ * The operation is the dual-branch global sparse attention of Speed3R ("Speed3R: Sparse
+ * Feed-forward 3D Reconstruction Models", arXiv 2603.08055). Its pages describe it in prose only
+ * (gist.science summary, "Technische samenvatting" -> "Methodologie"):
+ *   §1 "Compressie-tak"  the compression branch pools the tokens spatially by averaging, attends
+ *                        to the pooled tokens and produces a score matrix of relevant regions;
+ *   §1 "Selectie-tak"    the selection branch runs fine-grained attention only on the tokens of
+ *                        the top-k regions picked by those scores;
+ *   §2 "Gated Aggregation" a learned gate per token mixes the outputs of the two branches;
+ *   §4 "Efficient Kernel" top-k and softmax are computed together on chip.
+ * The project README (github Visual-AI/speed3r, "Notice" 3) restricts the kernel to bf16/fp16.
+ *
+ * Definitions used by every entry point (h = head, all layouts dense row-major):
+ *   L tokens of the flattened multi-view sequence (N views x P tokens per view), H heads, d = 64.
+ *   Key block j = tokens [j*b, min((j+1)*b, L)), nb = ceil(L/b); the last block may be partial.
+ *   Query block i = rows [64*i, min(64*i+64, L)), nqb = ceil(L/64).
+ *   Pooled keys/values   Kc[j,h,:] = mean of K[t,h,:] over the valid tokens t of block j (same
+ *                        for V), accumulated in fp32 and rounded once to bf16.
+ *   Compressed logits    s[q,j] = scale * <Q[q,h,:], Kc[j,h,:]>, for all j < nb.
+ *   lse[h,q]             = log sum_j exp(s[q,j])                       (natural log)
+ *   P[q,j]               = exp(s[q,j] - lse[h,q])                      (fp32)
+ *   O_cmp[q,h,:]         = sum_j P[q,j] * Vc[j,h,:]
+ *   scores[h,i,j]        = sum over the valid rows q of query block i of P[q,j]
+ *   idx[h,i,:]           = the topk block indices with the largest scores[h,i,:], ties broken
+ *                          toward the lower index
+ *   O_sel[q,h,:]         = softmax-weighted sum of V[t,h,:] over the tokens t < L of the
+ *                          blocks idx[h,i,:] of q's query block, weights softmax_t(scale*<Q,K[t]>)
+ *   out[q,h,:]           = sigmoid(g[q,h,0]) * O_cmp[q,h,:] + sigmoid(g[q,h,1]) * O_sel[q,h,:]
+ *
+ * Conventions:
+ *   - Every pointer argument is a DEVICE pointer of the current CUDA device, 16-byte aligned,
+ *     to a dense row-major array; the caller owns every buffer. The library never allocates or
+ *     frees device memory and never synchronises the stream.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream). The return value
+ *     reports host-side validation and launch errors only; a call that returns an error has
+ *     launched nothing, except S3R_ERR_CUDA which reports a failed launch.
+ *   - Conditions detected on the device (a bounded wait that expired, an out-of-range index when
+ *     S3R_FLAG_DEBUG_CHECKS is set) are OR-ed into the 32-bit word params->dev_status when it is
+ *     non-NULL, and into the workspace's status word in s3r_sparse_attn_fwd. Read it with
+ *     s3r_read_device_status after the stream has finished.
+ *   - bf16 values are passed as their 16-bit patterns (s3r_bf16).
+ *   - No C++ exception crosses this boundary; the functions are thread-safe (no global state
+ *     besides a launch counter).
+ */
+#ifndef S3R_H
+#define S3R_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t s3r_bf16;            /* raw bfloat16 bit pattern */
+typedef struct CUstream_st* s3r_stream; /* identical to cudaStream_t */
+
+typedef enum {
+  S3R_OK = 0,
+  S3R_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, topk out of range */
+  S3R_ERR_UNSUPPORTED = 2, /* a size this build does not implement (d, b, qblock, nb) */
+  S3R_ERR_WORKSPACE = 3,   /* workspace missing or smaller than s3r_workspace_bytes() */
+  S3R_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+  S3R_ERR_TIMEOUT = 5      /* reported via the device status word: a bounded wait expired */
+} s3r_status;
+
+/* Bits of the device status word. */
+#define S3R_DEV_TIMEOUT 0x1u   /* a kernel gave up on a bounded wait and returned early */
+#define S3R_DEV_BAD_INDEX 0x2u /* (debug checks) an idx entry was outside [0, nb) */
+
+/* params.flags */
+#define S3R_FLAG_DEBUG_CHECKS 0x1u /* validate idx on the device in s3r_sel_attn */
+
+typedef struct {
+  int64_t L;      /* tokens = N views * P tokens per view, >= 1 */
+  int32_t H;      /* heads, >= 1 */
+  int32_t d;      /* head dimension; this build implements d = 64 */
+  int32_t block;  /* b, key-block size: 32, 64 or 128 */
+  int32_t qblock; /* rows per query block for the score sums; must be 64 */
+  int32_t topk;   /* k, blocks selected per query block, 1 <= k <= nb (k = nb: dense selection) */
+  float scale;    /* softmax scale; <= 0 selects 1/sqrt(d) */
+  uint32_t flags; /* S3R_FLAG_* */
+  uint32_t* dev_status; /* optional device word that receives S3R_DEV_* bits (may be NULL) */
+  void* const* stage_events; /* optional: S3R_NUM_STAGES + 1 cudaEvent_t handles that
+                                s3r_sparse_attn_fwd records on `stream` at the stage boundaries
+                                (before stage 0, after each stage), for per-stage timing with
+                                cudaEventElapsedTime; ignored by the single-step entry points */
+} s3r_params;
+
+/* Stages of s3r_sparse_attn_fwd, in launch order (one kernel each). */
+#define S3R_STAGE_POOL 0         /* K/V block pooling */
+#define S3R_STAGE_CMP_LSE 1      /* compressed attention, pass A: lse */
+#define S3R_STAGE_CMP_PV_SCORE 2 /* compressed attention, pass B: O_cmp and block scores */
+#define S3R_STAGE_TOPK 3         /* per-query-block top-k */
+#define S3R_STAGE_SEL_COMBINE 4  /* selection attention fused with the gated combine */
+#define S3R_NUM_STAGES 5
+
+/* Largest nb (key blocks) this build accepts; beyond it calls return S3R_ERR_UNSUPPORTED. */
+#define S3R_MAX_BLOCKS 49152
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* s3r_status_string(s3r_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int s3r_version(void);
+
+/* Number of kernels this process has launched through the library so far (monotonic). */
+uint64_t s3r_kernel_launches(void);
+
+/* Bytes of device workspace s3r_sparse_attn_fwd needs for these sizes (0 if params invalid). */
+size_t s3r_workspace_bytes(const s3r_params* params);
+
+/* Synchronise `stream`, copy the device status word at `dev_status` into *out and clear it.
+ * Returns S3R_ERR_TIMEOUT if the S3R_DEV_TIMEOUT bit was set, S3R_OK otherwise. */
+s3r_status s3r_read_device_status(uint32_t* dev_status, s3r_stream stream, uint32_t* out);
+
+/* Device status word inside a workspace given to s3r_sparse_attn_fwd. */
+uint32_t* s3r_workspace_status_word(void* workspace);
+
+/* Compression branch, pooling ("Compressie-tak": average pooling).
+ *   k, v         [L, H, d] bf16 (read)
+ *   k_cmp, v_cmp [nb, H, d] bf16 (written): fp32 mean over the valid tokens, rounded to nearest
+ *                even bf16. */
+s3r_status s3r_compress_kv(const s3r_params* params, const s3r_bf16* k, const s3r_bf16* v,
+                           s3r_bf16* k_cmp, s3r_bf16* v_cmp, s3r_stream stream);
+
+/* Compression branch, attention to the block summaries and the score matrix
+ * ("Compressie-tak": "scorematrix").
+ *   q            [L, H, d] bf16;  k_cmp, v_cmp [nb, H, d] bf16 (read)
+ *   o_cmp        [L, H, d] fp32   (written)
+ *   lse          [H, L] fp32      (written, natural log)
+ *   scores       [H, nqb, nb] fp32 (written)
+ * Probabilities are formed in fp32 before the scores are summed; P is rounded to bf16 only as
+ * the operand of the P*Vc product. */
+s3r_status s3r_cmp_attn_and_score(const s3r_params* params, const s3r_bf16* q,
+                                  const s3r_bf16* k_cmp, const s3r_bf16* v_cmp, float* o_cmp,
+                                  float* lse, float* scores, s3r_stream stream);
+
+/* Per-query-block top-k ("Selectie-tak": "Top-k selectie").
+ *   scores [H, nqb, nb] fp32 (read), non-negative, not NaN
+ *   idx    [H, nqb, topk] int32 (written). The set is exact: score bits compared as unsigned
+ *          integers, equal scores broken toward the lower block index. For topk <= 2048 the
+ *          entries are ordered by descending score, ties by ascending index; for larger topk
+ *          they are in ascending index order. */
+s3r_status s3r_topk_blocks(const s3r_params* params, const float* scores, int32_t* idx,
+                           s3r_stream stream);
+
+/* Selection branch ("Selectie-tak": fine attention on the selected tokens).
+ *   q, k, v [L, H, d] bf16 (read); idx [H, nqb, topk] int32 (read): distinct block indices in
+ *           [0, nb) per row (entries outside that range are skipped; with
+ *           S3R_FLAG_DEBUG_CHECKS they also raise S3R_DEV_BAD_INDEX)
+ *   o_sel   [L, H, d] fp32 (written) */
+s3r_status s3r_sel_attn(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,
+                        const s3r_bf16* v, const int32_t* idx, float* o_sel, s3r_stream stream);
+
+/* Gated aggregation (§2 "Gated Aggregation"), elementwise.
+ *   o_cmp, o_sel [L, H, d] fp32 (read); gate_logits [L, H, 2] fp32 (read): [...,0] gates the
+ *   compression branch, [...,1] the selection branch, each through its own sigmoid
+ *   out          [L, H, d] bf16 (written, round to nearest even) */
+s3r_status s3r_gate_combine(const s3r_params* params, const float* o_cmp, const float* o_sel,
+                            const float* gate_logits, s3r_bf16* out, s3r_stream stream);
+
+/* The whole path in one call: pooling, compressed attention and scores, top-k, selection
+ * attention fused with the gated combine.
+ *   q, k, v     [L, H, d] bf16; gate_logits [L, H, 2] fp32 (read)
+ *   out         [L, H, d] bf16 (written)
+ *   idx_out     [H, nqb, topk] int32 (written if not NULL)
+ *   workspace   device buffer of at least s3r_workspace_bytes(params) bytes, 256-byte aligned;
+ *               its contents on entry do not matter. */
+s3r_status s3r_sparse_attn_fwd(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,
+                               const s3r_bf16* v, const float* gate_logits, s3r_bf16* out,
+                               int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                               s3r_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* S3R_H */

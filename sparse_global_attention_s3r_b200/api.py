@@ -1,0 +1,218 @@
+"""torch-tensor front end of libs3r.so: shape checks, output allocation, pointer marshalling.
+
+Every step of the computation runs in the library's CUDA kernels; torch only provides device
+memory and the current stream. All tensors must be CUDA tensors of the current device, dense and
+contiguous, with the layouts of include/s3r.h:
+
+    q, k, v      [L, H, 64] bf16          gates  [L, H, 2] fp32
+    k_cmp, v_cmp [nb, H, 64] bf16         lse    [H, L] fp32
+    o_cmp, o_sel [L, H, 64] fp32          scores [H, nqb, nb] fp32
+    idx          [H, nqb, topk] int32     out    [L, H, 64] bf16
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+
+QBLOCK = 64
+
+
+@dataclass(frozen=True)
+class Config:
+    """Sizes of one call: L tokens (N views x P tokens), H heads, d, block size b, top-k."""
+
+    L: int
+    H: int
+    d: int = 64
+    block: int = 64
+    topk: int = 16
+    scale: Optional[float] = None  # None -> 1/sqrt(d)
+    debug_checks: bool = False
+
+    @property
+    def nb(self) -> int:
+        return -(-self.L // self.block)
+
+    @property
+    def nqb(self) -> int:
+        return -(-self.L // QBLOCK)
+
+    def params(self, dev_status: Optional[torch.Tensor] = None, stage_events=None) -> _lib.Params:
+        return _lib.Params(self.L, self.H, self.d, self.block, QBLOCK, self.topk,
+                           0.0 if self.scale is None else float(self.scale),
+                           _lib.S3R_FLAG_DEBUG_CHECKS if self.debug_checks else 0,
+                           None if dev_status is None else dev_status.data_ptr(),
+                           None if stage_events is None else ctypes.addressof(stage_events))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, shape, dtype) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} contiguous={t.is_contiguous()}")
+
+
+def _lhd(cfg: Config):
+    return (cfg.L, cfg.H, cfg.d)
+
+
+def compress_kv(cfg: Config, k: torch.Tensor, v: torch.Tensor,
+                dev_status: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    _need(k, "k", _lhd(cfg), torch.bfloat16)
+    _need(v, "v", _lhd(cfg), torch.bfloat16)
+    kc = torch.empty((cfg.nb, cfg.H, cfg.d), dtype=torch.bfloat16, device=k.device)
+    vc = torch.empty_like(kc)
+    p = cfg.params(dev_status)
+    _lib.call("s3r_compress_kv", ctypes.byref(p), _ptr(k), _ptr(v), _ptr(kc), _ptr(vc), _stream())
+    return kc, vc
+
+
+def cmp_attn_and_score(cfg: Config, q: torch.Tensor, kc: torch.Tensor, vc: torch.Tensor,
+                       dev_status: Optional[torch.Tensor] = None):
+    """-> (o_cmp [L,H,d] fp32, lse [H,L] fp32, scores [H,nqb,nb] fp32)"""
+    _need(q, "q", _lhd(cfg), torch.bfloat16)
+    _need(kc, "k_cmp", (cfg.nb, cfg.H, cfg.d), torch.bfloat16)
+    _need(vc, "v_cmp", (cfg.nb, cfg.H, cfg.d), torch.bfloat16)
+    o = torch.empty(_lhd(cfg), dtype=torch.float32, device=q.device)
+    lse = torch.empty((cfg.H, cfg.L), dtype=torch.float32, device=q.device)
+    scores = torch.empty((cfg.H, cfg.nqb, cfg.nb), dtype=torch.float32, device=q.device)
+    p = cfg.params(dev_status)
+    _lib.call("s3r_cmp_attn_and_score", ctypes.byref(p), _ptr(q), _ptr(kc), _ptr(vc), _ptr(o),
+              _ptr(lse), _ptr(scores), _stream())
+    return o, lse, scores
+
+
+def topk_blocks(cfg: Config, scores: torch.Tensor,
+                dev_status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need(scores, "scores", (cfg.H, cfg.nqb, cfg.nb), torch.float32)
+    idx = torch.empty((cfg.H, cfg.nqb, cfg.topk), dtype=torch.int32, device=scores.device)
+    p = cfg.params(dev_status)
+    _lib.call("s3r_topk_blocks", ctypes.byref(p), _ptr(scores), _ptr(idx), _stream())
+    return idx
+
+
+def sel_attn(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor,
+             dev_status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, _lhd(cfg), torch.bfloat16)
+    _need(idx, "idx", (cfg.H, cfg.nqb, cfg.topk), torch.int32)
+    o = torch.empty(_lhd(cfg), dtype=torch.float32, device=q.device)
+    p = cfg.params(dev_status)
+    _lib.call("s3r_sel_attn", ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o),
+              _stream())
+    return o
+
+
+def gate_combine(cfg: Config, o_cmp: torch.Tensor, o_sel: torch.Tensor,
+                 gates: torch.Tensor) -> torch.Tensor:
+    _need(o_cmp, "o_cmp", _lhd(cfg), torch.float32)
+    _need(o_sel, "o_sel", _lhd(cfg), torch.float32)
+    _need(gates, "gates", (cfg.L, cfg.H, 2), torch.float32)
+    out = torch.empty(_lhd(cfg), dtype=torch.bfloat16, device=o_cmp.device)
+    p = cfg.params()
+    _lib.call("s3r_gate_combine", ctypes.byref(p), _ptr(o_cmp), _ptr(o_sel), _ptr(gates),
+              _ptr(out), _stream())
+    return out
+
+
+def workspace_bytes(cfg: Config) -> int:
+    p = cfg.params()
+    n = int(_lib.load().s3r_workspace_bytes(ctypes.byref(p)))
+    if n == 0:
+        raise _lib.S3RError("s3r_workspace_bytes", _lib.S3R_ERR_INVALID_ARG)
+    return n
+
+
+def alloc_workspace(cfg: Config, device=None) -> torch.Tensor:
+    n = workspace_bytes(cfg)
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(n, dtype=torch.uint8, device=device or torch.cuda.current_device())
+
+
+class StageEvents:
+    """S3R_NUM_STAGES + 1 CUDA events that s3r_sparse_attn_fwd records at its stage boundaries."""
+
+    def __init__(self):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(_lib.STAGES) + 1)]
+        for e in self.events:  # torch creates the underlying event on first record
+            e.record()
+        self.handles = (ctypes.c_void_p * len(self.events))(
+            *[e.cuda_event for e in self.events])
+
+    def stage_ms(self) -> dict:
+        """Milliseconds of each stage of the last recorded call (events must have completed)."""
+        return {n: self.events[i].elapsed_time(self.events[i + 1])
+                for i, n in enumerate(_lib.STAGES)}
+
+
+def sparse_attn_fwd(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                    gates: torch.Tensor, workspace: Optional[torch.Tensor] = None,
+                    out: Optional[torch.Tensor] = None, idx_out: Optional[torch.Tensor] = None,
+                    dev_status: Optional[torch.Tensor] = None,
+                    stage_events: Optional[StageEvents] = None) -> torch.Tensor:
+    """The whole path in one library call; returns out [L,H,d] bf16 (idx written if given)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, _lhd(cfg), torch.bfloat16)
+    _need(gates, "gates", (cfg.L, cfg.H, 2), torch.float32)
+    if workspace is None:
+        workspace = alloc_workspace(cfg, q.device)
+    if out is None:
+        out = torch.empty(_lhd(cfg), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", _lhd(cfg), torch.bfloat16)
+    if idx_out is not None:
+        _need(idx_out, "idx_out", (cfg.H, cfg.nqb, cfg.topk), torch.int32)
+    p = cfg.params(dev_status, None if stage_events is None else stage_events.handles)
+    _lib.call("s3r_sparse_attn_fwd", ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(gates),
+              _ptr(out), _ptr(idx_out), _ptr(workspace), workspace.numel(), _stream())
+    return out
+
+
+def read_device_status(word: torch.Tensor) -> int:
+    """Synchronise the current stream, return and clear the device status word."""
+    v = ctypes.c_uint32(0)
+    st = _lib.load().s3r_read_device_status(_ptr(word), _stream(), ctypes.byref(v))
+    if st not in (_lib.S3R_OK, _lib.S3R_ERR_TIMEOUT):
+        _lib.check("s3r_read_device_status", st)
+    return int(v.value)
+
+
+class SparseAttention:
+    """Reusable caller of the fused path: owns its workspace and output buffers on one device.
+
+    ``__call__`` takes device tensors. ``from_host`` takes pinned host tensors, copies them in,
+    runs the path and copies the output (and indices) back: the end-to-end use.
+    """
+
+    def __init__(self, cfg: Config, device=None):
+        self.cfg = cfg
+        self.device = torch.device(device or "cuda")
+        self.workspace = alloc_workspace(cfg, self.device)
+        self.out = torch.empty(_lhd(cfg), dtype=torch.bfloat16, device=self.device)
+        self.idx = torch.empty((cfg.H, cfg.nqb, cfg.topk), dtype=torch.int32, device=self.device)
+        self._dev_in = None
+
+    def __call__(self, q, k, v, gates) -> torch.Tensor:
+        return sparse_attn_fwd(self.cfg, q, k, v, gates, self.workspace, self.out, self.idx)
+
+    def from_host(self, q, k, v, gates, out_host: torch.Tensor) -> torch.Tensor:
+        if self._dev_in is None:
+            self._dev_in = [torch.empty_like(t, device=self.device) for t in (q, k, v, gates)]
+        for dst, src in zip(self._dev_in, (q, k, v, gates)):
+            dst.copy_(src, non_blocking=True)
+        self(*self._dev_in)
+        out_host.copy_(self.out, non_blocking=True)
+        return out_host

@@ -1,0 +1,219 @@
+// api.cu -- the extern "C" entry points of libs3r.so: argument validation, the workspace layout
+// of the fused call, and the launch sequence. The operation and its conventions are defined in
+// include/s3r.h.
+#include <atomic>
+#include <cmath>
+
+#include "internal.h"
+#include "s3r.h"
+
+namespace s3r {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+size_t topk_smem_bytes(int64_t nb);
+
+namespace {
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+s3r_status derive(const s3r_params* prm, Problem* out) {
+  if (!prm) return S3R_ERR_INVALID_ARG;
+  if (prm->L < 1 || prm->H < 1 || prm->H > 65535 || prm->topk < 1) return S3R_ERR_INVALID_ARG;
+  if (std::isnan(prm->scale) || std::isinf(prm->scale)) return S3R_ERR_INVALID_ARG;
+  if (prm->d != 64) return S3R_ERR_UNSUPPORTED;
+  if (prm->block != 32 && prm->block != 64 && prm->block != 128) return S3R_ERR_UNSUPPORTED;
+  if (prm->qblock != 64) return S3R_ERR_UNSUPPORTED;
+  Problem p{};
+  p.L = prm->L;
+  p.H = prm->H;
+  p.d = prm->d;
+  p.b = prm->block;
+  p.qb = prm->qblock;
+  p.k = prm->topk;
+  p.nb = (p.L + p.b - 1) / p.b;
+  p.nqb = (p.L + p.qb - 1) / p.qb;
+  if (p.nb > S3R_MAX_BLOCKS) return S3R_ERR_UNSUPPORTED;
+  if (p.k > p.nb) return S3R_ERR_INVALID_ARG;
+  p.scale = prm->scale > 0.f ? prm->scale : 1.0f / std::sqrt(static_cast<float>(p.d));
+  p.scale_log2 = static_cast<float>(static_cast<double>(p.scale) * 1.4426950408889634);
+  p.flags = prm->flags;
+  p.status = prm->dev_status;
+  if (p.status && (reinterpret_cast<uintptr_t>(p.status) & 3u)) return S3R_ERR_INVALID_ARG;
+  *out = p;
+  return S3R_OK;
+}
+
+s3r_status launched(cudaError_t e) { return e == cudaSuccess ? S3R_OK : S3R_ERR_CUDA; }
+
+// Workspace of the fused call, every region 256-byte aligned:
+//   status word | Kc [nb,H,d] bf16 | Vc | lse [H,L] f32 | O_cmp [L,H,d] f32 | scores [H,nqb,nb] f32
+//   | idx [H,nqb,k] i32
+struct Workspace {
+  size_t status, kc, vc, lse, o_cmp, scores, idx, total;
+};
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+Workspace layout(const Problem& p) {
+  Workspace w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += round256(bytes);
+    return at;
+  };
+  const size_t HD = static_cast<size_t>(p.H) * p.d;
+  w.status = take(4);
+  w.kc = take(static_cast<size_t>(p.nb) * HD * 2);
+  w.vc = take(static_cast<size_t>(p.nb) * HD * 2);
+  w.lse = take(static_cast<size_t>(p.H) * p.L * 4);
+  w.o_cmp = take(static_cast<size_t>(p.L) * HD * 4);
+  w.scores = take(static_cast<size_t>(p.H) * p.nqb * p.nb * 4);
+  w.idx = take(static_cast<size_t>(p.H) * p.nqb * p.k * 4);
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+}  // namespace s3r
+
+using namespace s3r;
+
+extern "C" {
+
+const char* s3r_status_string(s3r_status s) {
+  switch (s) {
+    case S3R_OK: return "S3R_OK";
+    case S3R_ERR_INVALID_ARG: return "S3R_ERR_INVALID_ARG";
+    case S3R_ERR_UNSUPPORTED: return "S3R_ERR_UNSUPPORTED";
+    case S3R_ERR_WORKSPACE: return "S3R_ERR_WORKSPACE";
+    case S3R_ERR_CUDA: return "S3R_ERR_CUDA";
+    case S3R_ERR_TIMEOUT: return "S3R_ERR_TIMEOUT";
+  }
+  return "S3R_ERR_UNKNOWN";
+}
+
+int s3r_version(void) { return 100; }
+
+uint64_t s3r_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t s3r_workspace_bytes(const s3r_params* params) {
+  Problem p;
+  if (derive(params, &p) != S3R_OK) return 0;
+  return layout(p).total;
+}
+
+uint32_t* s3r_workspace_status_word(void* workspace) {
+  return static_cast<uint32_t*>(workspace);  // the status word is the first region
+}
+
+s3r_status s3r_read_device_status(uint32_t* dev_status, s3r_stream stream, uint32_t* out) {
+  if (!dev_status || !out || (reinterpret_cast<uintptr_t>(dev_status) & 3u)) return S3R_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, dev_status, 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return S3R_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return S3R_ERR_CUDA;
+  if (cudaMemsetAsync(dev_status, 0, 4, stream) != cudaSuccess) return S3R_ERR_CUDA;
+  *out = v;
+  return (v & S3R_DEV_TIMEOUT) ? S3R_ERR_TIMEOUT : S3R_OK;
+}
+
+s3r_status s3r_compress_kv(const s3r_params* params, const s3r_bf16* k, const s3r_bf16* v,
+                           s3r_bf16* k_cmp, s3r_bf16* v_cmp, s3r_stream stream) {
+  Problem p;
+  s3r_status st = derive(params, &p);
+  if (st != S3R_OK) return st;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cmp) || !aligned16(v_cmp))
+    return S3R_ERR_INVALID_ARG;
+  return launched(launch_pool_kv(p, k, v, k_cmp, v_cmp, stream));
+}
+
+s3r_status s3r_cmp_attn_and_score(const s3r_params* params, const s3r_bf16* q,
+                                  const s3r_bf16* k_cmp, const s3r_bf16* v_cmp, float* o_cmp,
+                                  float* lse, float* scores, s3r_stream stream) {
+  Problem p;
+  s3r_status st = derive(params, &p);
+  if (st != S3R_OK) return st;
+  if (!aligned16(q) || !aligned16(k_cmp) || !aligned16(v_cmp) || !aligned16(o_cmp) ||
+      !aligned16(lse) || !aligned16(scores))
+    return S3R_ERR_INVALID_ARG;
+  st = launched(launch_cmp_lse(p, q, k_cmp, lse, stream));
+  if (st != S3R_OK) return st;
+  return launched(launch_cmp_pv_score(p, q, k_cmp, v_cmp, lse, o_cmp, scores, stream));
+}
+
+s3r_status s3r_topk_blocks(const s3r_params* params, const float* scores, int32_t* idx,
+                           s3r_stream stream) {
+  Problem p;
+  s3r_status st = derive(params, &p);
+  if (st != S3R_OK) return st;
+  if (!aligned16(scores) || !aligned16(idx)) return S3R_ERR_INVALID_ARG;
+  return launched(launch_topk(p, scores, idx, stream));
+}
+
+s3r_status s3r_sel_attn(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,
+                        const s3r_bf16* v, const int32_t* idx, float* o_sel, s3r_stream stream) {
+  Problem p;
+  s3r_status st = derive(params, &p);
+  if (st != S3R_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o_sel))
+    return S3R_ERR_INVALID_ARG;
+  return launched(launch_sel_attn(p, q, k, v, idx, o_sel, nullptr, nullptr, nullptr, stream));
+}
+
+s3r_status s3r_gate_combine(const s3r_params* params, const float* o_cmp, const float* o_sel,
+                            const float* gate_logits, s3r_bf16* out, s3r_stream stream) {
+  Problem p;
+  s3r_status st = derive(params, &p);
+  if (st != S3R_OK) return st;
+  if (!aligned16(o_cmp) || !aligned16(o_sel) || !aligned16(gate_logits) || !aligned16(out))
+    return S3R_ERR_INVALID_ARG;
+  return launched(launch_gate_combine(p, o_cmp, o_sel, gate_logits, out, stream));
+}
+
+s3r_status s3r_sparse_attn_fwd(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,
+                               const s3r_bf16* v, const float* gate_logits, s3r_bf16* out,
+                               int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                               s3r_stream stream) {
+  Problem p;
+  s3r_status st = derive(params, &p);
+  if (st != S3R_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate_logits) ||
+      !aligned16(out) || (idx_out && !aligned16(idx_out)))
+    return S3R_ERR_INVALID_ARG;
+  const Workspace w = layout(p);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < w.total)
+    return S3R_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base + w.status);
+  if (!p.status) p.status = status;
+  uint16_t* kc = reinterpret_cast<uint16_t*>(base + w.kc);
+  uint16_t* vc = reinterpret_cast<uint16_t*>(base + w.vc);
+  float* lse = reinterpret_cast<float*>(base + w.lse);
+  float* o_cmp = reinterpret_cast<float*>(base + w.o_cmp);
+  float* scores = reinterpret_cast<float*>(base + w.scores);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
+
+  void* const* ev = params->stage_events;
+  auto mark = [&](int i) {
+    return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), stream) : cudaSuccess;
+  };
+  if (cudaMemsetAsync(status, 0, 4, stream) != cudaSuccess) return S3R_ERR_CUDA;
+  if (mark(0) != cudaSuccess) return S3R_ERR_CUDA;
+  if ((st = launched(launch_pool_kv(p, k, v, kc, vc, stream))) != S3R_OK) return st;
+  if (mark(1) != cudaSuccess) return S3R_ERR_CUDA;
+  if ((st = launched(launch_cmp_lse(p, q, kc, lse, stream))) != S3R_OK) return st;
+  if (mark(2) != cudaSuccess) return S3R_ERR_CUDA;
+  if ((st = launched(launch_cmp_pv_score(p, q, kc, vc, lse, o_cmp, scores, stream))) != S3R_OK)
+    return st;
+  if (mark(3) != cudaSuccess) return S3R_ERR_CUDA;
+  if ((st = launched(launch_topk(p, scores, idx, stream))) != S3R_OK) return st;
+  if (mark(4) != cudaSuccess) return S3R_ERR_CUDA;
+  st = launched(launch_sel_attn(p, q, k, v, idx, nullptr, o_cmp, gate_logits, out, stream));
+  if (st != S3R_OK) return st;
+  return mark(5) == cudaSuccess ? S3R_OK : S3R_ERR_CUDA;
+}
+
+}  // extern "C"

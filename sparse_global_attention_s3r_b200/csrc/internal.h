@@ -1,0 +1,41 @@
+// internal.h -- launchers behind the C ABI of libs3r.so (not part of the public interface).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace s3r {
+
+// Sizes of one call after validation; every count is derived here, never passed in.
+struct Problem {
+  int64_t L;        // tokens
+  int H, d, b, qb;  // heads, head dim (64), key-block size, query-block rows (64)
+  int k;            // top-k
+  int64_t nb, nqb;  // key blocks, query blocks
+  float scale;      // softmax scale
+  float scale_log2; // scale * log2(e): logits in base-2 units
+  uint32_t flags;
+  uint32_t* status; // device status word or nullptr
+};
+
+// Each launcher enqueues one kernel on `st` and returns cudaGetLastError().
+cudaError_t launch_pool_kv(const Problem& p, const uint16_t* k, const uint16_t* v, uint16_t* kc,
+                           uint16_t* vc, cudaStream_t st);
+cudaError_t launch_cmp_lse(const Problem& p, const uint16_t* q, const uint16_t* kc, float* lse,
+                           cudaStream_t st);
+cudaError_t launch_cmp_pv_score(const Problem& p, const uint16_t* q, const uint16_t* kc,
+                                const uint16_t* vc, const float* lse, float* o_cmp, float* scores,
+                                cudaStream_t st);
+cudaError_t launch_topk(const Problem& p, const float* scores, int32_t* idx, cudaStream_t st);
+// o_sel != nullptr: write the selection output (fp32). Otherwise fuse the gated combine:
+// read o_cmp and gates and write out (bf16).
+cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, const int32_t* idx, float* o_sel,
+                            const float* o_cmp, const float* gates, uint16_t* out,
+                            cudaStream_t st);
+cudaError_t launch_gate_combine(const Problem& p, const float* o_cmp, const float* o_sel,
+                                const float* gates, uint16_t* out, cudaStream_t st);
+
+void count_launch();
+
+}  // namespace s3r

@@ -1,0 +1,179 @@
+// topk.cu -- per-query-block top-k of the block score matrix.
+//
+// Speed3R (gist.science summary, "Methodologie" §1 "Selectie-tak"): the selection branch attends
+// to the top-k blocks chosen by the compression branch's scores. Ties go to the lower block index.
+//
+// One CTA per score row [nb] (one query block of one head). Scores are probabilities summed over
+// rows, so they are non-negative and their fp32 bit patterns order like unsigned integers. The row
+// is staged once in shared memory (the only HBM read: nb * 4 bytes), then an exact radix select
+// finds the k-th largest pattern T in four 8-bit passes (per-warp histograms with warp-aggregated
+// increments, a block scan over the 256 bins). Every element above T is taken, and of the elements
+// equal to T the lowest indices, found by an in-order block prefix count. For k <= kSortMax the
+// winners are bitonic-sorted in shared memory on the 64-bit key (bits << 32 | ~index), i.e. by
+// descending score then ascending index; larger k are emitted in ascending index order.
+#include "common.cuh"
+#include "internal.h"
+
+namespace s3r {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kSortMax = 2048;
+
+// exclusive prefix sum over the block of one int per thread, in thread order; returns the total
+__device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kWarps ? warp_sums[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    if (lane < kWarps) warp_sums[lane] = wi - w;  // exclusive warp offsets
+    if (lane == kWarps - 1) warp_sums[kWarps] = wi;
+  }
+  __syncthreads();
+  const int res = warp_sums[warp] + incl - x;
+  total = warp_sums[kWarps];
+  __syncthreads();  // warp_sums may be reused right away
+  return res;
+}
+
+__global__ void __launch_bounds__(kThreads)
+    topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, int nb, int k) {
+  // dynamic shared memory: [kWarps][256] histograms (reused as the sort buffer), then [nb] keys
+  extern __shared__ __align__(16) uint32_t smem_dyn[];
+  int(*hist)[256] = reinterpret_cast<int(*)[256]>(smem_dyn);
+  uint32_t* sm_keys = smem_dyn + kWarps * 256;
+  __shared__ int warp_sums[kWarps + 1];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_kk;
+
+  const int64_t row = blockIdx.x;
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(scores + row * nb);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  for (int j = tid; j < nb; j += kThreads) sm_keys[j] = __ldg(src + j);
+  if (tid == 0) {
+    s_prefix = 0;
+    s_kk = k;
+  }
+  __syncthreads();
+
+  uint32_t mask = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = tid; b < kWarps * 256; b += kThreads) (&hist[0][0])[b] = 0;
+    __syncthreads();
+    const uint32_t prefix = s_prefix;
+    for (int j0 = 0; j0 < nb; j0 += kThreads) {
+      const int j = j0 + tid;
+      const bool in = j < nb && (sm_keys[j < nb ? j : 0] & mask) == prefix;
+      const uint32_t digit = in ? (sm_keys[j] >> shift) & 0xFFu : 0x100u + lane;  // unique if out
+      const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+      if (in && (__ffs(peers) - 1) == lane) atomicAdd(&hist[warp][digit], __popc(peers));
+    }
+    __syncthreads();
+    // bins in descending digit order: thread t < 256 owns digit 255 - t
+    int cnt = 0;
+    if (tid < 256) {
+      const int dgt = 255 - tid;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) cnt += hist[w][dgt];
+    }
+    int total;
+    const int before = block_exclusive_scan(tid < 256 ? cnt : 0, warp_sums, total);
+    const int kk = s_kk;
+    __syncthreads();
+    if (tid < 256 && before < kk && kk <= before + cnt) {
+      s_prefix = prefix | (static_cast<uint32_t>(255 - tid) << shift);
+      s_kk = kk - before;
+    }
+    mask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  const uint32_t T = s_prefix;  // bits of the k-th largest score
+  const int take_eq = s_kk;     // how many of the elements equal to T are selected
+
+  // in-order compaction: all elements > T, the first take_eq elements == T
+  uint64_t* sort_buf = reinterpret_cast<uint64_t*>(smem_dyn);  // histograms are dead now
+  const bool sorted_out = k <= kSortMax;
+  int32_t* out = idx + row * k;
+  int eq_base = 0, out_base = 0;
+  for (int j0 = 0; j0 < nb; j0 += kThreads) {
+    const int j = j0 + tid;
+    const uint32_t u = j < nb ? sm_keys[j] : 0u;
+    const bool gt = j < nb && u > T;
+    const bool eq = j < nb && u == T;
+    int eq_total;
+    const int eq_rank = eq_base + block_exclusive_scan(eq ? 1 : 0, warp_sums, eq_total);
+    const bool take = gt || (eq && eq_rank < take_eq);
+    int take_total;
+    const int pos = out_base + block_exclusive_scan(take ? 1 : 0, warp_sums, take_total);
+    if (take) {
+      if (sorted_out)
+        sort_buf[pos] = (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(j));
+      else
+        out[pos] = j;
+    }
+    eq_base += eq_total;
+    out_base += take_total;
+  }
+  if (!sorted_out) return;
+
+  int n2 = 1;
+  while (n2 < k) n2 <<= 1;
+  for (int e = k + tid; e < n2; e += kThreads) sort_buf[e] = 0ull;  // below every real key
+  __syncthreads();
+  // bitonic sort, descending
+  for (int size = 2; size <= n2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int e = tid; e < n2; e += kThreads) {
+        const int partner = e ^ stride;
+        if (partner > e) {
+          const bool desc = (e & size) == 0;
+          const uint64_t a = sort_buf[e], b = sort_buf[partner];
+          if ((a < b) == desc) {
+            sort_buf[e] = b;
+            sort_buf[partner] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int e = tid; e < k; e += kThreads)
+    out[e] = static_cast<int32_t>(~static_cast<uint32_t>(sort_buf[e] & 0xFFFFFFFFull));
+}
+
+}  // namespace
+
+static_assert(kWarps * 256 * 4 >= kSortMax * 8, "sort buffer must fit in the histogram space");
+
+size_t topk_smem_bytes(int64_t nb) {
+  return static_cast<size_t>(kWarps) * 256 * 4 + static_cast<size_t>(nb) * 4;
+}
+
+cudaError_t launch_topk(const Problem& p, const float* scores, int32_t* idx, cudaStream_t st) {
+  const size_t smem = topk_smem_bytes(p.nb);
+  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t rows = static_cast<int64_t>(p.H) * p.nqb;
+  topk_kernel<<<static_cast<unsigned>(rows), kThreads, smem, st>>>(scores, idx,
+                                                                   static_cast<int>(p.nb), p.k);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace s3r

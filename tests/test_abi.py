@@ -1,0 +1,131 @@
+"""The C ABI (include/s3r.h) on the host: the library loads, exports every declared entry point,
+and rejects bad arguments with the documented status before touching the device.
+
+None of these tests launches a kernel: every call below fails host-side validation first, so
+they run without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_global_attention_s3r_b200 import _lib, api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "s3r.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(s3r_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    lib = _lib.load()
+    names = declared_functions()
+    assert len(names) == 12, names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_lib.EXPORTS)
+
+
+def test_status_strings_and_version():
+    assert _lib.status_string(0) == "S3R_OK"
+    assert _lib.status_string(5) == "S3R_ERR_TIMEOUT"
+    assert _lib.status_string(99) == "S3R_ERR_UNKNOWN"
+    assert _lib.load().s3r_version() >= 100
+
+
+def _params(**kw):
+    base = dict(L=1024, H=2, d=64, block=64, qblock=64, topk=4, scale=0.0, flags=0, dev_status=None)
+    base.update(kw)
+    return _lib.Params(**base)
+
+
+# fake, never-dereferenced device addresses: validation must reject before any use
+A16 = ctypes.c_void_p(1 << 20)
+A8 = ctypes.c_void_p((1 << 20) + 8)
+A256 = ctypes.c_void_p(1 << 24)
+A16_NOT256 = ctypes.c_void_p((1 << 20) + 16)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(d=128), _lib.S3R_ERR_UNSUPPORTED),
+    (dict(d=32), _lib.S3R_ERR_UNSUPPORTED),
+    (dict(block=16), _lib.S3R_ERR_UNSUPPORTED),
+    (dict(block=256), _lib.S3R_ERR_UNSUPPORTED),
+    (dict(qblock=128), _lib.S3R_ERR_UNSUPPORTED),
+    (dict(L=0), _lib.S3R_ERR_INVALID_ARG),
+    (dict(H=0), _lib.S3R_ERR_INVALID_ARG),
+    (dict(topk=0), _lib.S3R_ERR_INVALID_ARG),
+    (dict(topk=17), _lib.S3R_ERR_INVALID_ARG),  # nb = 16
+    (dict(scale=float("nan")), _lib.S3R_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), _lib.S3R_ERR_INVALID_ARG),
+    (dict(L=_lib.S3R_MAX_BLOCKS * 32 + 1, block=32, topk=1), _lib.S3R_ERR_UNSUPPORTED),
+])
+def test_bad_sizes_are_rejected_by_every_entry_point(kw, want):
+    lib = _lib.load()
+    p = ctypes.byref(_params(**kw))
+    s = None
+    assert lib.s3r_compress_kv(p, A16, A16, A16, A16, s) == want
+    assert lib.s3r_cmp_attn_and_score(p, A16, A16, A16, A16, A16, A16, s) == want
+    assert lib.s3r_topk_blocks(p, A16, A16, s) == want
+    assert lib.s3r_sel_attn(p, A16, A16, A16, A16, A16, s) == want
+    assert lib.s3r_gate_combine(p, A16, A16, A16, A16, s) == want
+    assert lib.s3r_sparse_attn_fwd(p, A16, A16, A16, A16, A16, None, A256, 1 << 40, s) == want
+    assert lib.s3r_workspace_bytes(p) == 0
+
+
+def test_null_and_misaligned_pointers_are_rejected():
+    lib = _lib.load()
+    p = ctypes.byref(_params())
+    for bad in (None, A8):
+        assert lib.s3r_compress_kv(p, bad, A16, A16, A16, None) == _lib.S3R_ERR_INVALID_ARG
+        assert lib.s3r_compress_kv(p, A16, A16, A16, bad, None) == _lib.S3R_ERR_INVALID_ARG
+        assert lib.s3r_cmp_attn_and_score(p, A16, A16, A16, A16, A16, bad, None) == _lib.S3R_ERR_INVALID_ARG
+        assert lib.s3r_topk_blocks(p, bad, A16, None) == _lib.S3R_ERR_INVALID_ARG
+        assert lib.s3r_sel_attn(p, A16, A16, A16, bad, A16, None) == _lib.S3R_ERR_INVALID_ARG
+        assert lib.s3r_gate_combine(p, A16, A16, bad, A16, None) == _lib.S3R_ERR_INVALID_ARG
+        assert lib.s3r_sparse_attn_fwd(p, A16, bad, A16, A16, A16, None, A256, 1 << 40, None) == _lib.S3R_ERR_INVALID_ARG
+    # idx_out is optional but must be aligned when given
+    assert lib.s3r_sparse_attn_fwd(p, A16, A16, A16, A16, A16, A8, A256, 1 << 40, None) == _lib.S3R_ERR_INVALID_ARG
+    # a misaligned status word
+    p2 = ctypes.byref(_params(dev_status=(1 << 20) + 2))
+    assert lib.s3r_topk_blocks(p2, A16, A16, None) == _lib.S3R_ERR_INVALID_ARG
+    assert lib.s3r_read_device_status(None, None, A16) == _lib.S3R_ERR_INVALID_ARG
+    assert lib.s3r_topk_blocks(None, A16, A16, None) == _lib.S3R_ERR_INVALID_ARG
+
+
+def test_workspace_checks():
+    lib = _lib.load()
+    prm = _params()
+    need = lib.s3r_workspace_bytes(ctypes.byref(prm))
+    p = ctypes.byref(prm)
+    assert lib.s3r_sparse_attn_fwd(p, A16, A16, A16, A16, A16, None, None, need, None) == _lib.S3R_ERR_WORKSPACE
+    assert lib.s3r_sparse_attn_fwd(p, A16, A16, A16, A16, A16, None, A256, need - 1, None) == _lib.S3R_ERR_WORKSPACE
+    assert lib.s3r_sparse_attn_fwd(p, A16, A16, A16, A16, A16, None, A16_NOT256, need, None) == _lib.S3R_ERR_WORKSPACE
+    assert lib.s3r_workspace_status_word(A256) == A256.value
+
+
+def r256(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("L,H,b,k", [(1024, 2, 64, 4), (1374000, 16, 64, 32), (274800, 16, 32, 8588),
+                                     (1, 1, 128, 1)])
+def test_workspace_size_matches_layout(L, H, b, k):
+    cfg = api.Config(L=L, H=H, block=b, topk=k)
+    nb, nqb, d = cfg.nb, cfg.nqb, 64
+    want = (r256(4) + 2 * r256(nb * H * d * 2) + r256(H * L * 4) + r256(L * H * d * 4)
+            + r256(H * nqb * nb * 4) + r256(H * nqb * k * 4))
+    assert api.workspace_bytes(cfg) == want
+
+
+def test_compute_calls_need_cuda_tensors():
+    cfg = api.Config(L=64, H=1, block=64, topk=1)
+    import torch
+
+    k = torch.zeros(64, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        api.compress_kv(cfg, k, k)

@@ -1,0 +1,63 @@
+"""GPU parity at the workload sizes, through the fused entry point exactly as bench.py calls it.
+
+The oracle cannot run the whole layer at these sizes, so it pools all of K/V and then runs the
+whole path on a seeded sample of whole query blocks (scores sum over a block, so the sample is
+whole blocks; the ragged last block is always included). The GPU's indices and outputs for those
+blocks are compared: indices exact where the oracle's k-th/(k+1)-th gap exceeds 1e-4, every
+selected block score-optimal within tau, outputs against the oracle run on the GPU's indices.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from sparse_global_attention_s3r_b200 import api, synth
+
+from parity import check_output, check_selection
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+FULL = {  # name: (L, H, b, k, seed, sampled query blocks)
+    "vggt32": (43968, 16, 64, 16, 1, 64),
+    "n100": (137400, 16, 64, 32, 2, 48),
+    "n1000": (1374000, 16, 64, 32, 3, 64),
+    "pi3_b32": (274800, 16, 32, 32, 4000, 24),
+    "pi3_b64": (274800, 16, 64, 16, 4001, 24),
+    "pi3_b128": (274800, 16, 128, 8, 4002, 24),
+    "pi3_b64_all_blocks": (274800, 16, 64, 4294, 4003, 3),  # top-k = nb: dense selection
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_fused_path_at_workload_size(name):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    L, H, b, k, seed, nsample = FULL[name]
+    dev = torch.device("cuda")
+    x = synth.make_inputs(L, H, 64, b, seed, device=dev)
+    cfg = api.Config(L=L, H=H, block=b, topk=k)
+    sa = api.SparseAttention(cfg, dev)
+    out = sa(x.q, x.k, x.v, x.gates)
+    torch.cuda.synchronize()
+
+    pb = O.Problem(L, H, 64, b, k)
+    rng = np.random.default_rng(seed)
+    blocks = sorted(set(rng.choice(cfg.nqb - 1, size=nsample - 1, replace=False).tolist())
+                    | {cfg.nqb - 1})
+    rows = pb.rows_of(blocks)
+    rows_t = torch.from_numpy(rows).to(dev)
+    got_out = out.index_select(0, rows_t).double().cpu().numpy()
+    got_idx = sa.idx[:, blocks].cpu().numpy()
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    gates = x.gates.cpu().numpy()
+    del x, sa, out
+    torch.cuda.empty_cache()
+
+    kc, vc = O.pool(pb, bits[1]), O.pool(pb, bits[2])
+    ref = O.sparse_attn(pb, *bits, gates, qblocks=blocks, pooled=(kc, vc))
+    stats = check_selection(got_idx, ref.idx, ref.gap, ref.scores, k)
+    # conditional oracle: the oracle's compressed branch, its selection run on the GPU's indices
+    o_sel = O.sel_attn(pb, *bits, got_idx, qblocks=blocks)
+    cond_out = O.combine(ref.o_cmp, o_sel, np.ascontiguousarray(gates[rows]))
+    err = check_output(got_out, cond_out)
+    print(f"{name}: {stats} {err}")

@@ -1,0 +1,218 @@
+"""GPU parity: every entry point of libs3r.so against the fp64 CPU oracle, element by element, on
+seeded synthetic inputs (ragged tails, degenerate sizes, dense selection, tie-heavy scores,
+planted well-separated selections). Each call goes through the C ABI via the ctypes binding.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from sparse_global_attention_s3r_b200 import _lib, api, synth
+
+from parity import (GAP_EXACT, bf16_ulp, check_close, check_output, check_pooled,
+                    check_selection, f64)
+
+pytestmark = pytest.mark.gpu
+
+CASES = {  # name: (L, H, b, k, seed)
+    "tiny": (1024, 2, 64, 4, 0),
+    "ragged_b64": (1000, 2, 64, 5, 1),
+    "ragged_b32_odd_k": (1000, 2, 32, 7, 2),
+    "ragged_b128": (1300, 3, 128, 3, 3),
+    "single_partial_block": (17, 1, 64, 1, 4),
+    "one_token": (1, 2, 32, 1, 5),
+    "tail_of_one_row": (65, 1, 32, 3, 6),
+    "dense_selection": (1000, 2, 64, 16, 7),  # k = nb
+    "multi_tile_keys": (9000, 2, 32, 9, 8),  # nb = 282: several 64-key tiles + ragged tile
+}
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda")
+
+
+def inputs(name, device):
+    L, H, b, k, seed = CASES[name]
+    x = synth.make_inputs(L, H, 64, b, seed)
+    cfg = api.Config(L=L, H=H, block=b, topk=k)
+    pb = O.Problem(L, H, 64, b, k)
+    d = {n: getattr(x, n).to(device) for n in ("q", "k", "v", "gates")}
+    return cfg, pb, x, d
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_compress_kv(dev, name):
+    cfg, pb, x, d = inputs(name, dev)
+    kc, vc = api.compress_kv(cfg, d["k"], d["v"])
+    torch.cuda.synchronize()
+    for got, src in ((kc, x.k), (vc, x.v)):
+        ref = O.pool(pb, O.bf16_bits(src))
+        exact = check_pooled(f64(got), ref)
+        assert exact >= 0.999 or got.numel() < 20000 and exact >= 0.99, exact
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_cmp_attn_and_score(dev, name):
+    cfg, pb, x, d = inputs(name, dev)
+    kc, vc = api.compress_kv(cfg, d["k"], d["v"])
+    o, lse, scores = api.cmp_attn_and_score(cfg, d["q"], kc, vc)
+    torch.cuda.synchronize()
+    rlse, ro, rs = O.cmp_attn(pb, O.bf16_bits(x.q), f64(kc), f64(vc))  # same pooled operands
+    check_close("lse", f64(lse), rlse, 2e-5)
+    rowmax = rs.max(-1, keepdims=True)
+    err = np.abs(f64(scores) - rs)
+    assert np.all(err <= 1e-5 * rowmax + 1e-9), float((err / (rowmax + 1e-30)).max())
+    check_close("o_cmp", f64(o), ro, 2.0 ** -8 * np.abs(f64(vc)).max() + 1e-6, rl2=4e-3)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_topk_blocks_bit_exact(dev, name):
+    cfg, pb, x, d = inputs(name, dev)
+    kc, vc = O.pool(pb, O.bf16_bits(x.k)), O.pool(pb, O.bf16_bits(x.v))
+    _, _, rs = O.cmp_attn(pb, O.bf16_bits(x.q), kc, vc)
+    s32 = rs.astype(np.float32)
+    for scores in (s32, np.round(s32 * 4) / 4):  # the second is full of exact ties
+        scores = np.ascontiguousarray(scores, np.float32)
+        got = api.topk_blocks(cfg, torch.from_numpy(scores).to(dev)).cpu().numpy()
+        want, _ = O.topk(scores.astype(np.float64), cfg.topk)  # the same fp32 values
+        np.testing.assert_array_equal(got, want)
+
+
+def test_topk_large_k_unsorted_and_max_blocks(dev):
+    g = torch.Generator().manual_seed(9)
+    # k > 2048: the set is exact, emitted in ascending index order
+    L, b, k = 3000 * 64, 64, 2500
+    cfg = api.Config(L=L, H=1, block=b, topk=k)
+    s = torch.rand((1, cfg.nqb, cfg.nb), generator=g)
+    s[0, :5] = torch.round(s[0, :5] * 3) / 3  # heavy ties in a few rows
+    got = api.topk_blocks(cfg, s.to(dev)).cpu().numpy()
+    want, _ = O.topk(s.double().numpy(), k)
+    np.testing.assert_array_equal(got, np.sort(want, -1))
+    # the largest nb this build accepts (shared-memory staging at its limit)
+    nb = _lib.S3R_MAX_BLOCKS
+    cfg = api.Config(L=nb * 32, H=1, block=32, topk=32)
+    rows = torch.rand((1, 4, nb), generator=g)
+    full = torch.zeros((1, cfg.nqb, nb))
+    full[:, :4] = rows
+    got = api.topk_blocks(cfg, full.to(dev))[:, :4].cpu().numpy()
+    want, _ = O.topk(rows.double().numpy(), 32)
+    np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_sel_attn(dev, name):
+    cfg, pb, x, d = inputs(name, dev)
+    rng = np.random.default_rng(CASES[name][-1])
+    idx = np.stack([np.stack([rng.permutation(cfg.nb)[:cfg.topk] for _ in range(cfg.nqb)])
+                    for _ in range(cfg.H)]).astype(np.int32)
+    idx[:, -1, 0] = cfg.nb - 1 if cfg.nb - 1 not in idx[:, -1] else idx[:, -1, 0]
+    o = api.sel_attn(cfg, d["q"], d["k"], d["v"], torch.from_numpy(idx).to(dev))
+    torch.cuda.synchronize()
+    ref = O.sel_attn(pb, O.bf16_bits(x.q), O.bf16_bits(x.k), O.bf16_bits(x.v), idx)
+    check_close("o_sel", f64(o), ref, 2.0 ** -8 * np.abs(f64(x.v)).max() + 1e-6, rl2=4e-3)
+
+
+def test_sel_attn_debug_checks_flag_bad_indices(dev):
+    """An out-of-range index is skipped (its block contributes nothing) and, with debug checks,
+    reported in the device status word; reading the word clears it."""
+    cfg0, pb, x, d = inputs("ragged_b64", dev)
+    k = cfg0.topk
+    cfg = api.Config(L=cfg0.L, H=cfg0.H, block=cfg0.block, topk=k, debug_checks=True)
+    idx = np.tile(np.arange(k, dtype=np.int32), (cfg.H, cfg.nqb, 1))
+    idx[0, 3, 1] = cfg.nb + 7
+    word = torch.zeros(1, dtype=torch.int32, device=dev)
+    o = api.sel_attn(cfg, d["q"], d["k"], d["v"], torch.from_numpy(idx).to(dev), dev_status=word)
+    assert api.read_device_status(word) & _lib.S3R_DEV_BAD_INDEX
+    assert api.read_device_status(word) == 0
+    keep = [c for c in range(k) if c != 1]  # head 0, block 3 without the bad entry
+    ref = O.sel_attn(O.Problem(cfg.L, cfg.H, 64, cfg.block, k - 1), O.bf16_bits(x.q),
+                     O.bf16_bits(x.k), O.bf16_bits(x.v),
+                     np.ascontiguousarray(idx[:, 3:4, keep]), qblocks=[3])
+    check_close("o_sel(bad block skipped)", f64(o)[3 * 64:4 * 64, 0], ref[:, 0],
+                2.0 ** -8 * np.abs(f64(x.v)).max() + 1e-6)
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_b32_odd_k", "ragged_b128"])
+def test_gate_combine(dev, name):
+    cfg, pb, x, d = inputs(name, dev)
+    g = torch.Generator().manual_seed(1)
+    oc = torch.randn((cfg.L, cfg.H, 64), generator=g) * 0.01
+    os_ = torch.randn((cfg.L, cfg.H, 64), generator=g) * 0.01
+    gates = x.gates.clone()
+    gates[:5] = 0.0
+    gates[5:10, :, 0], gates[5:10, :, 1] = -60.0, 60.0
+    out = api.gate_combine(cfg, oc.to(dev), os_.to(dev), gates.to(dev))
+    ref = O.combine(oc.double().numpy(), os_.double().numpy(), gates.numpy())
+    got = f64(out)
+    assert np.all(np.abs(got - ref) <= bf16_ulp(ref) + 1e-7)
+
+
+def _fused(cfg, d):
+    idx = torch.empty((cfg.H, cfg.nqb, cfg.topk), dtype=torch.int32, device=d["q"].device)
+    out = api.sparse_attn_fwd(cfg, d["q"], d["k"], d["v"], d["gates"], idx_out=idx)
+    torch.cuda.synchronize()
+    return f64(out), idx.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_sparse_attn_fwd_whole_path(dev, name):
+    cfg, pb, x, d = inputs(name, dev)
+    out, idx = _fused(cfg, d)
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    ref = O.sparse_attn(pb, *bits, x.gates.numpy())
+    stats = check_selection(idx, ref.idx, ref.gap, ref.scores, cfg.topk)
+    cond = O.sparse_attn(pb, *bits, x.gates.numpy(), idx_given=idx, pooled=(ref.kc, ref.vc))
+    check_output(out, cond.out)
+    if stats["sets_equal"] == 1.0:
+        check_output(out, ref.out)
+
+
+def test_planted_selection_is_exact(dev):
+    L, H, b, k = 4096, 2, 64, 4
+    x = synth.make_planted(L, H, 64, b, seed=100)
+    cfg, pb = api.Config(L=L, H=H, block=b, topk=k), O.Problem(L, H, 64, b, k)
+    d = {n: getattr(x, n).to(dev) for n in ("q", "k", "v", "gates")}
+    out, idx = _fused(cfg, d)
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    ref = O.sparse_attn(pb, *bits, x.gates.numpy())
+    stats = check_selection(idx, ref.idx, ref.gap, ref.scores, k)
+    assert stats["gap_separated"] >= 0.9, stats
+    check_output(out, O.sparse_attn(pb, *bits, x.gates.numpy(), idx_given=idx).out)
+
+
+def test_uniform_keys_select_the_lowest_indices(dev):
+    """All keys equal: every block score ties exactly, so the tie rule alone decides: 0..k-1."""
+    L, H, b, k = 1000, 2, 64, 5
+    x = synth.make_inputs(L, H, 64, b, seed=11)
+    kappa = x.k[0:1]
+    kk = kappa.expand(L, H, 64).contiguous()
+    cfg = api.Config(L=L, H=H, block=b, topk=k)
+    d = {"q": x.q.to(dev), "k": kk.to(dev), "v": x.v.to(dev), "gates": x.gates.to(dev)}
+    out, idx = _fused(cfg, d)
+    np.testing.assert_array_equal(idx, np.broadcast_to(np.arange(k), idx.shape))
+    pb = O.Problem(L, H, 64, b, k)
+    ref = O.sparse_attn(pb, *[O.bf16_bits(t) for t in (x.q, kk, x.v)], x.gates.numpy())
+    check_output(out, ref.out)
+
+
+def test_dense_selection_equals_dense_attention(dev):
+    """k = nb: the selection branch is ordinary attention over all L tokens (torch SDPA fp64)."""
+    L, H, b = 777, 2, 32
+    x = synth.make_inputs(L, H, 64, b, seed=12)
+    cfg = api.Config(L=L, H=H, block=b, topk=-(-L // b))
+    idx = torch.arange(cfg.nb, dtype=torch.int32).expand(H, cfg.nqb, cfg.nb).contiguous()
+    o = api.sel_attn(cfg, x.q.to(dev), x.k.to(dev), x.v.to(dev), idx.to(dev))
+    q, k, v = (t.double().permute(1, 0, 2)[None] for t in (x.q, x.k, x.v))
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v)[0].permute(1, 0, 2).numpy()
+    check_close("dense", f64(o), ref, 2.0 ** -8 * np.abs(f64(x.v)).max() + 1e-6, rl2=4e-3)
+
+
+def test_launch_counter_counts_kernels(dev):
+    cfg, pb, x, d = inputs("tiny", dev)
+    n0 = _lib.kernel_launches()
+    api.sparse_attn_fwd(cfg, d["q"], d["k"], d["v"], d["gates"])
+    torch.cuda.synchronize()
+    assert _lib.kernel_launches() - n0 == 5
