@@ -77,8 +77,7 @@ def algorithmic(cfg):
         "flops": cmp_flops + sel_flops,
         "stage_work": {
             "pool": ("hbm", 2.0 * (L + nb) * H * d * 2),                       # bytes
-            "cmp_lse": ("tensor", 2.0 * L * nb * d * H),                       # flops (Q.Kc^T)
-            "cmp_pv_score": ("tensor", cmp_flops),                            # flops
+            "cmp": ("tensor", cmp_flops),                                     # flops
             "topk": ("hbm", H * nqb * (nb * 4.0 + k * 4.0)),                  # bytes
             "sel_combine": ("tensor", sel_flops),                             # flops
         },

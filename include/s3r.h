@@ -72,6 +72,9 @@ typedef enum {
 
 /* params.flags */
 #define S3R_FLAG_DEBUG_CHECKS 0x1u /* validate idx on the device in s3r_sel_attn */
+#define S3R_FLAG_TEST_TIMEOUT 0x2u /* testing only: the compressed-branch kernel waits on a barrier
+                                      that nothing signals, with a 1 ms limit, so the timeout path
+                                      runs: S3R_DEV_TIMEOUT is set and the outputs are invalid */
 
 typedef struct {
   int64_t L;      /* tokens = N views * P tokens per view, >= 1 */
@@ -90,12 +93,11 @@ typedef struct {
 } s3r_params;
 
 /* Stages of s3r_sparse_attn_fwd, in launch order (one kernel each). */
-#define S3R_STAGE_POOL 0         /* K/V block pooling */
-#define S3R_STAGE_CMP_LSE 1      /* compressed attention, pass A: lse */
-#define S3R_STAGE_CMP_PV_SCORE 2 /* compressed attention, pass B: O_cmp and block scores */
-#define S3R_STAGE_TOPK 3         /* per-query-block top-k */
-#define S3R_STAGE_SEL_COMBINE 4  /* selection attention fused with the gated combine */
-#define S3R_NUM_STAGES 5
+#define S3R_STAGE_POOL 0        /* K/V block pooling */
+#define S3R_STAGE_CMP 1         /* compressed attention (lse pass, then O_cmp and block scores) */
+#define S3R_STAGE_TOPK 2        /* per-query-block top-k */
+#define S3R_STAGE_SEL_COMBINE 3 /* selection attention fused with the gated combine */
+#define S3R_NUM_STAGES 4
 
 /* Largest nb (key blocks) this build accepts; beyond it calls return S3R_ERR_UNSUPPORTED. */
 #define S3R_MAX_BLOCKS 49152

@@ -21,8 +21,9 @@ S3R_ERR_TIMEOUT = 5
 S3R_DEV_TIMEOUT = 0x1
 S3R_DEV_BAD_INDEX = 0x2
 S3R_FLAG_DEBUG_CHECKS = 0x1
+S3R_FLAG_TEST_TIMEOUT = 0x2
 S3R_MAX_BLOCKS = 49152
-STAGES = ("pool", "cmp_lse", "cmp_pv_score", "topk", "sel_combine")  # S3R_STAGE_* order
+STAGES = ("pool", "cmp", "topk", "sel_combine")  # S3R_STAGE_* order
 
 # every function the header declares, with its ctypes signature
 _P = ctypes.c_void_p

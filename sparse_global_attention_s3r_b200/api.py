@@ -33,6 +33,7 @@ class Config:
     topk: int = 16
     scale: Optional[float] = None  # None -> 1/sqrt(d)
     debug_checks: bool = False
+    test_timeout: bool = False  # testing only: exercise the bounded-wait timeout path
 
     @property
     def nb(self) -> int:
@@ -45,7 +46,8 @@ class Config:
     def params(self, dev_status: Optional[torch.Tensor] = None, stage_events=None) -> _lib.Params:
         return _lib.Params(self.L, self.H, self.d, self.block, QBLOCK, self.topk,
                            0.0 if self.scale is None else float(self.scale),
-                           _lib.S3R_FLAG_DEBUG_CHECKS if self.debug_checks else 0,
+                           (_lib.S3R_FLAG_DEBUG_CHECKS if self.debug_checks else 0)
+                           | (_lib.S3R_FLAG_TEST_TIMEOUT if self.test_timeout else 0),
                            None if dev_status is None else dev_status.data_ptr(),
                            None if stage_events is None else ctypes.addressof(stage_events))
 

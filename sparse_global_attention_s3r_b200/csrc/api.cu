@@ -48,10 +48,10 @@ s3r_status derive(const s3r_params* prm, Problem* out) {
 s3r_status launched(cudaError_t e) { return e == cudaSuccess ? S3R_OK : S3R_ERR_CUDA; }
 
 // Workspace of the fused call, every region 256-byte aligned:
-//   status word | Kc [nb,H,d] bf16 | Vc | lse [H,L] f32 | O_cmp [L,H,d] f32 | scores [H,nqb,nb] f32
+//   status word | Kc [nb,H,d] bf16 | Vc | O_cmp [L,H,d] f32 | scores [H,nqb,nb] f32
 //   | idx [H,nqb,k] i32
 struct Workspace {
-  size_t status, kc, vc, lse, o_cmp, scores, idx, total;
+  size_t status, kc, vc, o_cmp, scores, idx, total;
 };
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -68,7 +68,6 @@ Workspace layout(const Problem& p) {
   w.status = take(4);
   w.kc = take(static_cast<size_t>(p.nb) * HD * 2);
   w.vc = take(static_cast<size_t>(p.nb) * HD * 2);
-  w.lse = take(static_cast<size_t>(p.H) * p.L * 4);
   w.o_cmp = take(static_cast<size_t>(p.L) * HD * 4);
   w.scores = take(static_cast<size_t>(p.H) * p.nqb * p.nb * 4);
   w.idx = take(static_cast<size_t>(p.H) * p.nqb * p.k * 4);
@@ -139,9 +138,7 @@ s3r_status s3r_cmp_attn_and_score(const s3r_params* params, const s3r_bf16* q,
   if (!aligned16(q) || !aligned16(k_cmp) || !aligned16(v_cmp) || !aligned16(o_cmp) ||
       !aligned16(lse) || !aligned16(scores))
     return S3R_ERR_INVALID_ARG;
-  st = launched(launch_cmp_lse(p, q, k_cmp, lse, stream));
-  if (st != S3R_OK) return st;
-  return launched(launch_cmp_pv_score(p, q, k_cmp, v_cmp, lse, o_cmp, scores, stream));
+  return launched(launch_cmp_attn_tc(p, q, k_cmp, v_cmp, lse, o_cmp, scores, stream));
 }
 
 s3r_status s3r_topk_blocks(const s3r_params* params, const float* scores, int32_t* idx,
@@ -191,7 +188,6 @@ s3r_status s3r_sparse_attn_fwd(const s3r_params* params, const s3r_bf16* q, cons
   if (!p.status) p.status = status;
   uint16_t* kc = reinterpret_cast<uint16_t*>(base + w.kc);
   uint16_t* vc = reinterpret_cast<uint16_t*>(base + w.vc);
-  float* lse = reinterpret_cast<float*>(base + w.lse);
   float* o_cmp = reinterpret_cast<float*>(base + w.o_cmp);
   float* scores = reinterpret_cast<float*>(base + w.scores);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
@@ -204,16 +200,14 @@ s3r_status s3r_sparse_attn_fwd(const s3r_params* params, const s3r_bf16* q, cons
   if (mark(0) != cudaSuccess) return S3R_ERR_CUDA;
   if ((st = launched(launch_pool_kv(p, k, v, kc, vc, stream))) != S3R_OK) return st;
   if (mark(1) != cudaSuccess) return S3R_ERR_CUDA;
-  if ((st = launched(launch_cmp_lse(p, q, kc, lse, stream))) != S3R_OK) return st;
-  if (mark(2) != cudaSuccess) return S3R_ERR_CUDA;
-  if ((st = launched(launch_cmp_pv_score(p, q, kc, vc, lse, o_cmp, scores, stream))) != S3R_OK)
+  if ((st = launched(launch_cmp_attn_tc(p, q, kc, vc, nullptr, o_cmp, scores, stream))) != S3R_OK)
     return st;
-  if (mark(3) != cudaSuccess) return S3R_ERR_CUDA;
+  if (mark(2) != cudaSuccess) return S3R_ERR_CUDA;
   if ((st = launched(launch_topk(p, scores, idx, stream))) != S3R_OK) return st;
-  if (mark(4) != cudaSuccess) return S3R_ERR_CUDA;
+  if (mark(3) != cudaSuccess) return S3R_ERR_CUDA;
   st = launched(launch_sel_attn(p, q, k, v, idx, nullptr, o_cmp, gate_logits, out, stream));
   if (st != S3R_OK) return st;
-  return mark(5) == cudaSuccess ? S3R_OK : S3R_ERR_CUDA;
+  return mark(4) == cudaSuccess ? S3R_OK : S3R_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -1,0 +1,41 @@
+// tma_host.cu -- host-side creation of the TMA tensor maps the tensor-core kernels load through.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "tma_host.h"
+
+namespace s3r {
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap_head_rows(CUtensorMap* map, const void* base, int64_t rows, int H, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  // 2-D view of a [rows, H, 64] bf16 tensor: x = H*64 contiguous elements, y = rows.
+  // A box of 64 x box_rows at x = 64*h is one head's [box_rows, 64] tile; rows past the end read
+  // as zeros. 128-byte swizzle: the shared-memory layout the tcgen05 descriptors describe.
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H) * 64, static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * 64 * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace s3r

@@ -4,13 +4,22 @@
 // to the top-k blocks chosen by the compression branch's scores. Ties go to the lower block index.
 //
 // One CTA per score row [nb] (one query block of one head). Scores are probabilities summed over
-// rows, so they are non-negative and their fp32 bit patterns order like unsigned integers. The row
-// is staged once in shared memory (the only HBM read: nb * 4 bytes), then an exact radix select
-// finds the k-th largest pattern T in four 8-bit passes (per-warp histograms with warp-aggregated
-// increments, a block scan over the 256 bins). Every element above T is taken, and of the elements
-// equal to T the lowest indices, found by an in-order block prefix count. For k <= kSortMax the
-// winners are bitonic-sorted in shared memory on the 64-bit key (bits << 32 | ~index), i.e. by
-// descending score then ascending index; larger k are emitted in ascending index order.
+// rows, so they are non-negative and their fp32 bit patterns order like unsigned integers; the
+// 64-bit key (bits << 32 | ~index) orders by descending score, then ascending index, and is unique.
+// The row is staged once in shared memory (the only HBM read: nb * 4 bytes) while every thread
+// keeps the maximum of the elements it loaded.
+//
+// Fast path (k <= kFilterMax): the k-th largest of the 512 per-thread maxima, T0, is a lower bound
+// of the k-th largest score (k distinct elements reach it), so the exact top-k is contained in the
+// candidates {score >= T0}, which for non-degenerate rows number little more than k. They are
+// compacted with warp-aggregated atomics and bitonic-sorted on the 64-bit key; the first k win.
+//
+// Exact fallback (larger k, or more than kSortMax candidates, e.g. rows of equal scores): a radix
+// select finds the k-th largest pattern T in four 8-bit passes (per-warp histograms with
+// warp-aggregated increments, a block scan over the 256 bins). Every element above T is taken, and
+// of the elements equal to T the lowest indices, found by an in-order block prefix count. For
+// k <= kSortMax the winners are bitonic-sorted as above; larger k are emitted in ascending index
+// order.
 #include "common.cuh"
 #include "internal.h"
 
@@ -19,7 +28,29 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSortMax = 2048;
+constexpr int kSortMax = 2048;   // largest k whose output is sorted; also the candidate cap
+constexpr int kFilterMax = 512;  // largest k for the threshold-filter fast path (= kThreads)
+
+// descending bitonic sort of n keys (n a power of two) in shared memory; all threads call it
+template <typename T>
+__device__ __forceinline__ void bitonic_sort_desc(T* a, int n) {
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int e = threadIdx.x; e < n; e += kThreads) {
+        const int partner = e ^ stride;
+        if (partner > e) {
+          const bool desc = (e & size) == 0;
+          const T x = a[e], y = a[partner];
+          if ((x < y) == desc) {
+            a[e] = y;
+            a[partner] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
 
 // exclusive prefix sum over the block of one int per thread, in thread order; returns the total
 __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int& total) {
@@ -59,17 +90,75 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ int warp_sums[kWarps + 1];
   __shared__ uint32_t s_prefix;
   __shared__ int s_kk;
+  __shared__ uint32_t s_max[kThreads];
+  __shared__ int s_count;
 
   const int64_t row = blockIdx.x;
   const uint32_t* src = reinterpret_cast<const uint32_t*>(scores + row * nb);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int32_t* out = idx + row * k;
+  uint64_t* sort_buf = reinterpret_cast<uint64_t*>(smem_dyn);  // aliases the histograms
 
-  for (int j = tid; j < nb; j += kThreads) sm_keys[j] = __ldg(src + j);
+  uint32_t my_max = 0;
+  {
+    int j = tid;
+    for (; j + 3 * kThreads < nb; j += 4 * kThreads) {  // 4 loads in flight per thread
+      uint32_t x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] = __ldg(src + j + u * kThreads);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        sm_keys[j + u * kThreads] = x[u];
+        my_max = max(my_max, x[u]);
+      }
+    }
+    for (; j < nb; j += kThreads) {
+      const uint32_t x = __ldg(src + j);
+      sm_keys[j] = x;
+      my_max = max(my_max, x);
+    }
+  }
+  s_max[tid] = my_max;  // threads that loaded nothing contribute 0, below every candidate used
   if (tid == 0) {
     s_prefix = 0;
     s_kk = k;
+    s_count = 0;
   }
   __syncthreads();
+
+  if (k <= kFilterMax && k <= nb) {
+    bitonic_sort_desc(s_max, kThreads);
+    const uint32_t t0 = s_max[k - 1];
+    // at least k elements are >= t0 (the k largest per-thread maxima are distinct elements),
+    // unless fewer than k threads loaded anything; then t0 = 0 and every element qualifies
+    for (int j0 = 0; j0 < nb; j0 += kThreads) {
+      const int j = j0 + tid;
+      const bool cand = j < nb && sm_keys[j < nb ? j : 0] >= t0;
+      const uint32_t m = __ballot_sync(0xffffffffu, cand);
+      int base = 0;
+      if (lane == 0 && m) base = atomicAdd(&s_count, __popc(m));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (cand) {
+        const int pos = base + __popc(m & ((1u << lane) - 1u));
+        if (pos < kSortMax)
+          sort_buf[pos] = (static_cast<uint64_t>(sm_keys[j]) << 32) |
+                          static_cast<uint32_t>(~static_cast<uint32_t>(j));
+      }
+    }
+    __syncthreads();
+    const int count = s_count;
+    if (count <= kSortMax) {
+      int n2 = 1;
+      while (n2 < count) n2 <<= 1;
+      for (int e = count + tid; e < n2; e += kThreads) sort_buf[e] = 0ull;
+      __syncthreads();
+      bitonic_sort_desc(sort_buf, n2);
+      for (int e = tid; e < k; e += kThreads)
+        out[e] = static_cast<int32_t>(~static_cast<uint32_t>(sort_buf[e] & 0xFFFFFFFFull));
+      return;
+    }
+    // too many candidates (degenerate row): fall through to the exact radix select
+  }
 
   uint32_t mask = 0;
   for (int shift = 24; shift >= 0; shift -= 8) {
@@ -106,9 +195,7 @@ __global__ void __launch_bounds__(kThreads)
   const int take_eq = s_kk;     // how many of the elements equal to T are selected
 
   // in-order compaction: all elements > T, the first take_eq elements == T
-  uint64_t* sort_buf = reinterpret_cast<uint64_t*>(smem_dyn);  // histograms are dead now
   const bool sorted_out = k <= kSortMax;
-  int32_t* out = idx + row * k;
   int eq_base = 0, out_base = 0;
   for (int j0 = 0; j0 < nb; j0 += kThreads) {
     const int j = j0 + tid;
@@ -135,23 +222,7 @@ __global__ void __launch_bounds__(kThreads)
   while (n2 < k) n2 <<= 1;
   for (int e = k + tid; e < n2; e += kThreads) sort_buf[e] = 0ull;  // below every real key
   __syncthreads();
-  // bitonic sort, descending
-  for (int size = 2; size <= n2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int e = tid; e < n2; e += kThreads) {
-        const int partner = e ^ stride;
-        if (partner > e) {
-          const bool desc = (e & size) == 0;
-          const uint64_t a = sort_buf[e], b = sort_buf[partner];
-          if ((a < b) == desc) {
-            sort_buf[e] = b;
-            sort_buf[partner] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
+  bitonic_sort_desc(sort_buf, n2);
   for (int e = tid; e < k; e += kThreads)
     out[e] = static_cast<int32_t>(~static_cast<uint32_t>(sort_buf[e] & 0xFFFFFFFFull));
 }
