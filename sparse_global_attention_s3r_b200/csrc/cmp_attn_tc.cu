@@ -6,16 +6,19 @@
 //
 // Exact scores need normalised probabilities, so one launch makes two passes over the nb block
 // summaries of its 128-row query tile (two 64-row query blocks) and one head:
-//   pass A: S = Q Kc^T (tcgen05.mma into TMEM), online max / sum  -> lse per row (registers)
+//   pass A: S = Q Kc^T (tcgen05.mma into TMEM), running max / sum -> lse per row
 //   pass B: S again; P = exp2(S*scale*log2e - lse2) in fp32; the column sums of the fp32 P over
 //           each 64-row query block are that block's scores; bf16(P) is stored to TMEM and
 //           O_cmp += P Vc runs on the tensor cores with P as the TMEM operand.
-// Roles (224 threads):
-//   warp 0     TMA producer: Q once, then Kc (pass A) or Kc+Vc (pass B) 64-key tiles into a
-//              4-stage ring of 128-byte-swizzled shared-memory tiles
-//   warp 1     TMEM owner (256 columns) and the single-thread tcgen05.mma issuer
-//   warps 2-5  softmax: one query row per thread (TMEM lane), column sums by shuffle halving
-//   warp 6     sums the two warps' partial column sums of each query block, writes scores
+// Roles (352 threads, 11 warps):
+//   warp 0      TMA producer: Q once, then Kc (pass A) or Kc+Vc (pass B) 64-key tiles into a
+//               4-stage ring of 128-byte-swizzled shared-memory tiles
+//   warp 1      TMEM owner (256 columns) and the single-thread tcgen05.mma issuer
+//   warps 2-9   softmax: warp w reads TMEM lane quadrant w%4 (32 rows) and column half
+//               (w-2)/4 (32 of the tile's 64 columns). With the 16x256b load shape a thread
+//               holds 4 rows x 8 columns, so a column sum is 3 in-thread adds plus 3 shuffle
+//               levels; P goes back with the matching 16x128b store shape.
+//   warp 10     adds the two row-quadrant partial column sums of each query block, writes scores
 // TMEM: S[2] (64 fp32 columns each), P[2] (64 bf16 = 32 columns each), O (64 fp32 columns).
 // Every wait is an mbarrier wait bounded in time that also watches a CTA abort flag; on expiry
 // the kernel records S3R_DEV_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
@@ -30,10 +33,12 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBM = 128;      // query rows per CTA (TMEM lanes)
-constexpr int kBN = 64;       // block summaries per tile
-constexpr int kStages = 4;    // shared-memory ring depth
-constexpr int kThreads = 224; // 7 warps
+constexpr int kBM = 128;       // query rows per CTA (TMEM lanes)
+constexpr int kBN = 64;        // block summaries per tile
+constexpr int kStages = 4;     // shared-memory ring depth
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = (3 + kSoftmaxWarps) * 32;  // producer, MMA, softmax x8, scores
+constexpr int kScoreWarp = 2 + kSoftmaxWarps;
 constexpr uint32_t kQBytes = kBM * 128;   // 16 KB
 constexpr uint32_t kKVBytes = kBN * 128;  // 8 KB
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 192, kTmemCols = 256;
@@ -46,17 +51,19 @@ struct __align__(8) Bars {
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
   uint64_t red_full[2], red_empty[2];
+  uint64_t stat;  // both column halves' row statistics of pass A are in shared memory
   uint64_t o_full, drain;
   uint64_t never;  // never signalled: waited on only under S3R_FLAG_TEST_TIMEOUT
 };
 
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKV = kQBytes;                              // stage s: K at +2s*8K, V +8K
-constexpr uint32_t kOffRed = kOffKV + kStages * 2 * kKVBytes;     // [2][4][64] floats
-constexpr uint32_t kOffBars = kOffRed + 2 * 4 * 64 * 4;
-constexpr uint32_t kOffMisc = kOffBars + sizeof(Bars);            // tmem base, abort flag
+constexpr uint32_t kOffKV = kQBytes;                           // stage s: K at +2s*8K, V +8K
+constexpr uint32_t kOffRed = kOffKV + kStages * 2 * kKVBytes;  // [2 par][4 quadrant][64] f32
+constexpr uint32_t kOffStat = kOffRed + 2 * 4 * 64 * 4;        // [2 halves][128 rows] float2
+constexpr uint32_t kOffBars = kOffStat + 2 * 128 * 8;
+constexpr uint32_t kOffMisc = kOffBars + sizeof(Bars);  // tmem base, abort flag
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
-// Request enough that at most two CTAs share an SM, so two 256-column TMEM allocations always fit.
+// At most two CTAs share an SM (shared memory), so two 256-column TMEM allocations always fit.
 constexpr uint32_t kSmemBytes = (kSmemUsed + 1024 > 80 * 1024 ? kSmemUsed + 1024 : 80 * 1024);
 
 struct CmpArgs {
@@ -76,6 +83,21 @@ __device__ __forceinline__ void raise_abort(volatile int* abort, uint32_t* statu
   set_status(status, S3R_DEV_TIMEOUT);
 }
 
+// Split the 16 registers of a 16x256b.x4 load at row offset 0 and the 16 at row offset 16 into
+// v[i][c]: row i in {tr, tr+8, tr+16, tr+24}, column c in 0..7 = 8*(c/2) + 2*(lane%4) + c%2.
+__device__ __forceinline__ void unpack_rows(const uint32_t (&a)[16], const uint32_t (&b)[16],
+                                            float (&v)[4][8]) {
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      v[0][2 * r + e] = __uint_as_float(a[4 * r + e]);
+      v[1][2 * r + e] = __uint_as_float(a[4 * r + 2 + e]);
+      v[2][2 * r + e] = __uint_as_float(b[4 * r + e]);
+      v[3][2 * r + e] = __uint_as_float(b[4 * r + 2 + e]);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 2)
     cmp_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -88,6 +110,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   float* red = reinterpret_cast<float*>(smem + kOffRed);
+  float2* stat = reinterpret_cast<float2*>(smem + kOffStat);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
@@ -104,12 +127,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_empty[b], 128);
-      mbar_init(&bars->p_full[b], 128);
+      mbar_init(&bars->s_empty[b], kSoftmaxWarps * 32);
+      mbar_init(&bars->p_full[b], kSoftmaxWarps * 32);
       mbar_init(&bars->p_empty[b], 1);
-      mbar_init(&bars->red_full[b], 4);
+      mbar_init(&bars->red_full[b], kSoftmaxWarps);
       mbar_init(&bars->red_empty[b], 1);
     }
+    mbar_init(&bars->stat, kSoftmaxWarps);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->drain, 1);
     mbar_init(&bars->never, 1);
@@ -171,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         const uint64_t dk = desc_sw128(sbase + kOffKV + stage * 2 * kKVBytes);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
+        for (int ks = 0; ks < 4; ++ks)  // 16 of d per step: 32 bytes into the swizzled row
           mma_ss(tbase + kColS + b * kBN, dq + 2 * ks, dk + 2 * ks, kIdescQK, ks > 0);
         return true;
       };
@@ -208,113 +232,180 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_wait(&bars->drain, 0, &dummy, lim);
       }
     }
-  } else if (warp <= 5) {
+  } else if (warp < kScoreWarp) {
     // ------------------------------------------------------------------ softmax warps
-    const int g = warp & 3;  // TMEM lane quadrant this warp may access
-    const int row_local = g * 32 + lane;
-    const int64_t row = q0 + row_local;
-    const bool row_ok = row < a.L;
-    const uint32_t tl = tbase + (static_cast<uint32_t>(g * 32) << 16);
+    const int g = warp & 3;             // TMEM lane quadrant this warp may access
+    const int half = (warp - 2) >> 2;   // which 32 of the tile's 64 columns
+    const int tq = lane & 3, tr = lane >> 2;
+    const uint32_t tl0 = tbase + (static_cast<uint32_t>(g * 32) << 16);
+    const uint32_t tl16 = tbase + (static_cast<uint32_t>(g * 32 + 16) << 16);
     const float sl2 = a.scale_log2;
+    // column (within the tile) of value column c of this thread
+    auto col_of = [&](int c) { return half * 32 + 8 * (c >> 1) + 2 * tq + (c & 1); };
     bool ok = true;
     if (a.flags & S3R_FLAG_TEST_TIMEOUT) ok = mbar_wait(&bars->never, 0, abort, lim);
 
-    // pass A: online max / sum over all nb summaries
-    float m = -INFINITY, l = 0.f;
+    // pass A: per-thread running max (raw logits) and sum over this thread's columns
+    float mr[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mr[i] = -INFINITY, l[i] = 0.f;
     for (int t = 0; ok && t < nt; ++t) {
       const int b = t & 1;
       if (!(ok = mbar_wait(&bars->s_full[b], (t >> 1) & 1, abort, lim))) break;
       tc_fence_after();
-      uint32_t r0[32], r1[32];
-      tmem_ld32(tl + kColS + b * kBN, r0);
-      tmem_ld32(tl + kColS + b * kBN + 32, r1);
-      tmem_wait_ld_regs(r0);
-      tmem_wait_ld_regs(r1);
+      uint32_t ra[16], rb[16];
+      tmem_ld16x256_x4(tl0 + kColS + b * kBN + half * 32, ra);
+      tmem_ld16x256_x4(tl16 + kColS + b * kBN + half * 32, rb);
+      tmem_wait_ld_n<16>(ra);
+      tmem_wait_ld_n<16>(rb);
       tc_fence_before();
       mbar_arrive(&bars->s_empty[b]);
-      const int64_t valid = a.nb - static_cast<int64_t>(t) * kBN;  // columns < valid are real
-      float x[64];
-      float tmax = -INFINITY;
+      float v[4][8];
+      unpack_rows(ra, rb, v);
+      if (static_cast<int64_t>(t + 1) * kBN > a.nb) {  // ragged last tile
+        const int64_t valid = a.nb - static_cast<int64_t>(t) * kBN;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const float s = __uint_as_float(j < 32 ? r0[j] : r1[j - 32]);
-        x[j] = j < valid ? s * sl2 : -INFINITY;
-        tmax = fmaxf(tmax, x[j]);
+        for (int c = 0; c < 8; ++c)
+          if (col_of(c) >= valid) v[0][c] = v[1][c] = v[2][c] = v[3][c] = -INFINITY;
       }
-      const float mn = fmaxf(m, tmax);  // finite: the first column of every tile is real
-      l *= exp2_approx(m - mn);
-      m = mn;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) l += exp2_approx(x[j] - m);
+      for (int i = 0; i < 4; ++i) {
+        float tmax = fmaxf(fmaxf(fmaxf(v[i][0], v[i][1]), fmaxf(v[i][2], v[i][3])),
+                           fmaxf(fmaxf(v[i][4], v[i][5]), fmaxf(v[i][6], v[i][7])));
+        const float mn = fmaxf(mr[i], tmax);
+        if (mn == -INFINITY) continue;  // no valid column seen yet by this thread
+        const float off = -mn * sl2;
+        l[i] *= exp2_approx(fmaf(mr[i], sl2, off));
+        mr[i] = mn;
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) {
+          const float2 x = __ffma2_rn(make_float2(v[i][c], v[i][c + 1]), make_float2(sl2, sl2),
+                                      make_float2(off, off));
+          acc = __fadd2_rn(acc, make_float2(exp2_approx(x.x), exp2_approx(x.y)));
+        }
+        l[i] += acc.x + acc.y;
+      }
     }
-    const float lse2 = row_ok ? m + log2f(l) : INFINITY;
-    if (ok && a.lse && row_ok) a.lse[static_cast<int64_t>(h) * a.L + row] = lse2 * kLn2;
+    // combine the statistics of the 4 threads of a quad and of the two column halves
+    float lse2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, mr[i], o);
+        const float l2 = __shfl_xor_sync(0xffffffffu, l[i], o);
+        const float mn = fmaxf(mr[i], m2);
+        const float w1 = mr[i] == -INFINITY ? 0.f : exp2_approx((mr[i] - mn) * sl2);
+        const float w2 = m2 == -INFINITY ? 0.f : exp2_approx((m2 - mn) * sl2);
+        l[i] = l[i] * w1 + l2 * w2;
+        mr[i] = mn;
+      }
+      if (tq == 0) stat[half * 128 + g * 32 + tr + 8 * i] = make_float2(mr[i], l[i]);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->stat);
+    if (ok) ok = mbar_wait(&bars->stat, 0, abort, lim);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int rl = g * 32 + tr + 8 * i;
+      const float2 s0 = stat[rl], s1 = stat[128 + rl];
+      const float mn = fmaxf(s0.x, s1.x);  // finite: column 0 is valid for every row
+      const float w0 = s0.x == -INFINITY ? 0.f : exp2_approx((s0.x - mn) * sl2);
+      const float w1 = s1.x == -INFINITY ? 0.f : exp2_approx((s1.x - mn) * sl2);
+      const int64_t row = q0 + rl;
+      lse2[i] = row < a.L ? mn * sl2 + log2f(s0.y * w0 + s1.y * w1) : INFINITY;
+      if (ok && a.lse && half == 0 && tq == 0 && row < a.L)
+        a.lse[static_cast<int64_t>(h) * a.L + row] = lse2[i] * kLn2;
+    }
 
     // pass B: probabilities, column sums, P to TMEM for the P*Vc product
     for (int t = 0; ok && t < nt; ++t) {
-      const int c = nt + t, b = c & 1;
-      if (!(ok = mbar_wait(&bars->s_full[b], (c >> 1) & 1, abort, lim))) break;
+      const int c2 = nt + t, b = c2 & 1;
+      if (!(ok = mbar_wait(&bars->s_full[b], (c2 >> 1) & 1, abort, lim))) break;
       tc_fence_after();
-      uint32_t r[2][32];
-      tmem_ld32(tl + kColS + b * kBN, r[0]);
-      tmem_ld32(tl + kColS + b * kBN + 32, r[1]);
-      tmem_wait_ld_regs(r[0]);
-      tmem_wait_ld_regs(r[1]);
+      uint32_t ra[16], rb[16];
+      tmem_ld16x256_x4(tl0 + kColS + b * kBN + half * 32, ra);
+      tmem_ld16x256_x4(tl16 + kColS + b * kBN + half * 32, rb);
+      tmem_wait_ld_n<16>(ra);
+      tmem_wait_ld_n<16>(rb);
       tc_fence_before();
       mbar_arrive(&bars->s_empty[b]);
-      const int64_t valid = a.nb - static_cast<int64_t>(t) * kBN;
+      float v[4][8];
+      unpack_rows(ra, rb, v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < 8; c += 2) {
+          const float2 x = __ffma2_rn(make_float2(v[i][c], v[i][c + 1]), make_float2(sl2, sl2),
+                                      make_float2(-lse2[i], -lse2[i]));
+          v[i][c] = exp2_approx(x.x);
+          v[i][c + 1] = exp2_approx(x.y);
+        }
+      if (static_cast<int64_t>(t + 1) * kBN > a.nb) {  // ragged last tile: P = 0 past nb
+        const int64_t valid = a.nb - static_cast<int64_t>(t) * kBN;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (col_of(c) >= valid) v[0][c] = v[1][c] = v[2][c] = v[3][c] = 0.f;
+      }
+      // bf16 P for the tensor cores, in the 16x128b store layout (same columns as the load)
+      uint32_t p0[8], p1[8];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        p0[2 * r] = pack_bf16(v[0][2 * r], v[0][2 * r + 1]);
+        p0[2 * r + 1] = pack_bf16(v[1][2 * r], v[1][2 * r + 1]);
+        p1[2 * r] = pack_bf16(v[2][2 * r], v[2][2 * r + 1]);
+        p1[2 * r + 1] = pack_bf16(v[3][2 * r], v[3][2 * r + 1]);
+      }
+      // column sums of the fp32 P: the thread's 4 rows, then the 8 row groups of the warp
+      float cs[8];
+#pragma unroll
+      for (int c = 0; c < 8; c += 2) {
+        const float2 s01 = __fadd2_rn(make_float2(v[0][c], v[0][c + 1]),
+                                      make_float2(v[1][c], v[1][c + 1]));
+        const float2 s23 = __fadd2_rn(make_float2(v[2][c], v[2][c + 1]),
+                                      make_float2(v[3][c], v[3][c + 1]));
+        const float2 s = __fadd2_rn(s01, s23);
+        cs[c] = s.x;
+        cs[c + 1] = s.y;
+      }
+#pragma unroll
+      for (int w = 4; w >= 1; w >>= 1) {  // lane bits 4, 3, 2 (the row group tr)
+        const bool upper = lane & (w << 2);
+#pragma unroll
+        for (int i = 0; i < w; ++i) {
+          const float send = upper ? cs[i] : cs[i + w];
+          const float keep = upper ? cs[i + w] : cs[i];
+          cs[i] = keep + __shfl_xor_sync(0xffffffffu, send, w << 2);
+        }
+      }
+      // cs[0] is now the 32-row sum of value column c = tr of this lane
       const int par = t & 1;
       if (!(ok = mbar_wait(&bars->red_empty[par], ((t >> 1) & 1) ^ 1, abort, lim))) break;
-      uint32_t pk[32];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float p[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float s = __uint_as_float(r[half][j]);
-          p[j] = (half * 32 + j) < valid ? exp2_approx(fmaf(s, sl2, -lse2)) : 0.f;
-        }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) pk[half * 16 + j] = pack_bf16(p[2 * j], p[2 * j + 1]);
-        // column sums over the warp's 32 rows: recursive halving leaves column `lane` here
-#pragma unroll
-        for (int w = 16; w >= 1; w >>= 1) {
-          const bool upper = lane & w;
-#pragma unroll
-          for (int i = 0; i < w; ++i) {
-            const float send = upper ? p[i] : p[i + w];
-            const float keep = upper ? p[i + w] : p[i];
-            p[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
-          }
-        }
-        red[(par * 4 + g) * 64 + half * 32 + lane] = p[0];
-      }
+      red[(par * 4 + g) * 64 + col_of(tr)] = cs[0];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->red_full[par]);
       const int pb = t & 1;
       if (!(ok = mbar_wait(&bars->p_empty[pb], ((t >> 1) & 1) ^ 1, abort, lim))) break;
-      tmem_st32(tl + kColP + pb * 32, pk);
-      tmem_wait_st_regs(pk);
+      tmem_st16x128_x4(tl0 + kColP + pb * 32 + half * 16, p0);
+      tmem_st16x128_x4(tl16 + kColP + pb * 32 + half * 16, p1);
+      tmem_wait_st_keep8(p0);
+      tmem_wait_st_keep8(p1);
       tc_fence_before();
       mbar_arrive(&bars->p_full[pb]);
     }
     if (ok && (ok = mbar_wait(&bars->o_full, 0, abort, lim))) {
       tc_fence_after();
-      uint32_t o0[32], o1[32];
-      tmem_ld32(tl + kColO, o0);
-      tmem_ld32(tl + kColO + 32, o1);
-      tmem_wait_ld_regs(o0);
-      tmem_wait_ld_regs(o1);
-      if (row_ok) {
-        float4* dst = reinterpret_cast<float4*>(a.o_cmp + (row * a.H + h) * 64);
+      uint32_t o[32];
+      tmem_ld32(tl0 + kColO + half * 32, o);
+      tmem_wait_ld_regs(o);
+      const int64_t row = q0 + g * 32 + lane;
+      if (row < a.L) {
+        float4* dst = reinterpret_cast<float4*>(a.o_cmp + (row * a.H + h) * 64 + half * 32);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          dst[j] = make_float4(__uint_as_float(o0[4 * j]), __uint_as_float(o0[4 * j + 1]),
-                               __uint_as_float(o0[4 * j + 2]), __uint_as_float(o0[4 * j + 3]));
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          dst[8 + j] = make_float4(__uint_as_float(o1[4 * j]), __uint_as_float(o1[4 * j + 1]),
-                                   __uint_as_float(o1[4 * j + 2]), __uint_as_float(o1[4 * j + 3]));
+          dst[j] = make_float4(__uint_as_float(o[4 * j]), __uint_as_float(o[4 * j + 1]),
+                               __uint_as_float(o[4 * j + 2]), __uint_as_float(o[4 * j + 3]));
       }
     }
     if (!ok) raise_abort(abort, a.status);

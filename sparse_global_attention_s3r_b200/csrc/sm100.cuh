@@ -153,6 +153,43 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// 16 lanes x 256 bits, 4 repetitions (32 columns): thread t receives, for repetition r,
+// r[4r+0..1] = lane (base + t/4), columns 8r + 2(t%4) + {0,1}, and
+// r[4r+2..3] = lane (base + 8 + t/4), the same columns.
+__device__ __forceinline__ void tmem_ld16x256_x4(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+// 16 lanes x 128 bits, 4 repetitions (16 columns): thread t supplies, for repetition r,
+// r[2r] -> lane (base + t/4), column 4r + t%4, and r[2r+1] -> lane (base + 8 + t/4), same column.
+__device__ __forceinline__ void tmem_st16x128_x4(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld_n(uint32_t (&r)[N]);
+template <>
+__device__ __forceinline__ void tmem_wait_ld_n<16>(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st_keep8(const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::"r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]),
+               "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // tcgen05.wait::ld that also marks the 32 destination registers of a preceding tmem_ld32 as
 // produced here, so the compiler cannot schedule their first use before the wait.
 __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
