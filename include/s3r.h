@@ -176,6 +176,27 @@ s3r_status s3r_sparse_attn_fwd(const s3r_params* params, const s3r_bf16* q, cons
                                int32_t* idx_out, void* workspace, size_t workspace_bytes,
                                s3r_stream stream);
 
+/* Size of the scratch array built into the library for s3r_sparse_attn_fwd_static (32 MiB). */
+#define S3R_STATIC_WORKSPACE_BYTES (32u << 20)
+
+/* The whole path, like s3r_sparse_attn_fwd, for callers that cannot allocate device memory (for
+ * example a host framework that owns all device memory and gives plugins no workspace, or a loop
+ * that must not allocate once running). The paper has no counterpart; this is a deployment
+ * variant. Instead of a caller-provided workspace it uses a fixed array of
+ * S3R_STATIC_WORKSPACE_BYTES inside the library, present on every GPU that loads the library
+ * until the process exits. It allocates nothing.
+ *   Sizes whose workspace (s3r_workspace_bytes) exceeds S3R_STATIC_WORKSPACE_BYTES are rejected
+ *   with S3R_ERR_WORKSPACE before anything is launched; other arguments as s3r_sparse_attn_fwd.
+ *   The first call on a device looks up the array's device address on that device (the current
+ *   one); make that first call before any stream capture.
+ *   All calls share the one array per device and it keeps the last call's contents (the parts
+ *   that must start at zero are cleared by every call). Calls whose executions overlap on the GPU
+ *   (different streams, or different host threads) race on it: serialise them. */
+s3r_status s3r_sparse_attn_fwd_static(const s3r_params* params, const s3r_bf16* q,
+                                      const s3r_bf16* k, const s3r_bf16* v,
+                                      const float* gate_logits, s3r_bf16* out, int32_t* idx_out,
+                                      s3r_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

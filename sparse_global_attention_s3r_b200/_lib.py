@@ -23,6 +23,7 @@ S3R_DEV_BAD_INDEX = 0x2
 S3R_FLAG_DEBUG_CHECKS = 0x1
 S3R_FLAG_TEST_TIMEOUT = 0x2
 S3R_MAX_BLOCKS = 49152
+S3R_STATIC_WORKSPACE_BYTES = 32 << 20
 STAGES = ("pool", "cmp", "topk", "sel_combine")  # S3R_STAGE_* order
 
 # every function the header declares, with its ctypes signature
@@ -40,6 +41,7 @@ EXPORTS = {
     "s3r_sel_attn": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P]),
     "s3r_gate_combine": (ctypes.c_int, [_P, _P, _P, _P, _P, _P]),
     "s3r_sparse_attn_fwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "s3r_sparse_attn_fwd_static": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
 }
 
 

@@ -183,6 +183,25 @@ def sparse_attn_fwd(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tens
     return out
 
 
+def sparse_attn_fwd_static(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                           gates: torch.Tensor, out: Optional[torch.Tensor] = None,
+                           idx_out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The whole path without a workspace argument: the library's built-in scratch array is used
+    (sizes up to S3R_STATIC_WORKSPACE_BYTES of workspace; see include/s3r.h)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, _lhd(cfg), torch.bfloat16)
+    _need(gates, "gates", (cfg.L, cfg.H, 2), torch.float32)
+    if out is None:
+        out = torch.empty(_lhd(cfg), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", _lhd(cfg), torch.bfloat16)
+    if idx_out is not None:
+        _need(idx_out, "idx_out", (cfg.H, cfg.nqb, cfg.topk), torch.int32)
+    p = cfg.params()
+    _lib.call("s3r_sparse_attn_fwd_static", ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
+              _ptr(gates), _ptr(out), _ptr(idx_out), _stream())
+    return out
+
+
 def read_device_status(word: torch.Tensor) -> int:
     """Synchronise the current stream, return and clear the device status word."""
     v = ctypes.c_uint32(0)

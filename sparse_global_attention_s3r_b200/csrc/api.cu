@@ -76,6 +76,53 @@ Workspace layout(const Problem& p) {
 }
 
 }  // namespace
+
+size_t fused_workspace_bytes(const s3r_params* params) {
+  Problem p;
+  if (derive(params, &p) != S3R_OK) return 0;
+  return layout(p).total;
+}
+
+// The whole path on a caller-provided workspace; shared by the fused entry points.
+int fused_forward(const s3r_params* params, const uint16_t* q, const uint16_t* k,
+                  const uint16_t* v, const float* gate_logits, uint16_t* out, int32_t* idx_out,
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  Problem p;
+  s3r_status st = derive(params, &p);
+  if (st != S3R_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate_logits) ||
+      !aligned16(out) || (idx_out && !aligned16(idx_out)))
+    return S3R_ERR_INVALID_ARG;
+  const Workspace w = layout(p);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < w.total)
+    return S3R_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base + w.status);
+  if (!p.status) p.status = status;
+  uint16_t* kc = reinterpret_cast<uint16_t*>(base + w.kc);
+  uint16_t* vc = reinterpret_cast<uint16_t*>(base + w.vc);
+  float* o_cmp = reinterpret_cast<float*>(base + w.o_cmp);
+  float* scores = reinterpret_cast<float*>(base + w.scores);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
+
+  void* const* ev = params->stage_events;
+  auto mark = [&](int i) {
+    return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), stream) : cudaSuccess;
+  };
+  if (cudaMemsetAsync(status, 0, 4, stream) != cudaSuccess) return S3R_ERR_CUDA;
+  if (mark(0) != cudaSuccess) return S3R_ERR_CUDA;
+  if ((st = launched(launch_pool_kv(p, k, v, kc, vc, stream))) != S3R_OK) return st;
+  if (mark(1) != cudaSuccess) return S3R_ERR_CUDA;
+  if ((st = launched(launch_cmp_attn_tc(p, q, kc, vc, nullptr, o_cmp, scores, stream))) != S3R_OK)
+    return st;
+  if (mark(2) != cudaSuccess) return S3R_ERR_CUDA;
+  if ((st = launched(launch_topk(p, scores, idx, stream))) != S3R_OK) return st;
+  if (mark(3) != cudaSuccess) return S3R_ERR_CUDA;
+  st = launched(launch_sel_attn(p, q, k, v, idx, nullptr, o_cmp, gate_logits, out, stream));
+  if (st != S3R_OK) return st;
+  return mark(4) == cudaSuccess ? S3R_OK : S3R_ERR_CUDA;
+}
+
 }  // namespace s3r
 
 using namespace s3r;
@@ -98,11 +145,7 @@ int s3r_version(void) { return 100; }
 
 uint64_t s3r_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
-size_t s3r_workspace_bytes(const s3r_params* params) {
-  Problem p;
-  if (derive(params, &p) != S3R_OK) return 0;
-  return layout(p).total;
-}
+size_t s3r_workspace_bytes(const s3r_params* params) { return fused_workspace_bytes(params); }
 
 uint32_t* s3r_workspace_status_word(void* workspace) {
   return static_cast<uint32_t*>(workspace);  // the status word is the first region
@@ -174,40 +217,8 @@ s3r_status s3r_sparse_attn_fwd(const s3r_params* params, const s3r_bf16* q, cons
                                const s3r_bf16* v, const float* gate_logits, s3r_bf16* out,
                                int32_t* idx_out, void* workspace, size_t workspace_bytes,
                                s3r_stream stream) {
-  Problem p;
-  s3r_status st = derive(params, &p);
-  if (st != S3R_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate_logits) ||
-      !aligned16(out) || (idx_out && !aligned16(idx_out)))
-    return S3R_ERR_INVALID_ARG;
-  const Workspace w = layout(p);
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < w.total)
-    return S3R_ERR_WORKSPACE;
-  uint8_t* base = static_cast<uint8_t*>(workspace);
-  uint32_t* status = reinterpret_cast<uint32_t*>(base + w.status);
-  if (!p.status) p.status = status;
-  uint16_t* kc = reinterpret_cast<uint16_t*>(base + w.kc);
-  uint16_t* vc = reinterpret_cast<uint16_t*>(base + w.vc);
-  float* o_cmp = reinterpret_cast<float*>(base + w.o_cmp);
-  float* scores = reinterpret_cast<float*>(base + w.scores);
-  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
-
-  void* const* ev = params->stage_events;
-  auto mark = [&](int i) {
-    return ev ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), stream) : cudaSuccess;
-  };
-  if (cudaMemsetAsync(status, 0, 4, stream) != cudaSuccess) return S3R_ERR_CUDA;
-  if (mark(0) != cudaSuccess) return S3R_ERR_CUDA;
-  if ((st = launched(launch_pool_kv(p, k, v, kc, vc, stream))) != S3R_OK) return st;
-  if (mark(1) != cudaSuccess) return S3R_ERR_CUDA;
-  if ((st = launched(launch_cmp_attn_tc(p, q, kc, vc, nullptr, o_cmp, scores, stream))) != S3R_OK)
-    return st;
-  if (mark(2) != cudaSuccess) return S3R_ERR_CUDA;
-  if ((st = launched(launch_topk(p, scores, idx, stream))) != S3R_OK) return st;
-  if (mark(3) != cudaSuccess) return S3R_ERR_CUDA;
-  st = launched(launch_sel_attn(p, q, k, v, idx, nullptr, o_cmp, gate_logits, out, stream));
-  if (st != S3R_OK) return st;
-  return mark(4) == cudaSuccess ? S3R_OK : S3R_ERR_CUDA;
+  return static_cast<s3r_status>(s3r::fused_forward(params, q, k, v, gate_logits, out, idx_out,
+                                                     workspace, workspace_bytes, stream));
 }
 
 }  // extern "C"

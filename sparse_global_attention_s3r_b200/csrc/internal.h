@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "s3r.h"
+
 namespace s3r {
 
 // Sizes of one call after validation; every count is derived here, never passed in.
@@ -36,5 +38,12 @@ cudaError_t launch_gate_combine(const Problem& p, const float* o_cmp, const floa
                                 const float* gates, uint16_t* out, cudaStream_t st);
 
 void count_launch();
+
+// Workspace bytes of the fused path (0 if params are invalid), and the fused path itself on a
+// caller-provided workspace (returns an s3r_status value).
+size_t fused_workspace_bytes(const s3r_params* params);
+int fused_forward(const s3r_params* params, const uint16_t* q, const uint16_t* k,
+                  const uint16_t* v, const float* gate_logits, uint16_t* out, int32_t* idx_out,
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 }  // namespace s3r

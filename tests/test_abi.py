@@ -24,7 +24,7 @@ def declared_functions():
 def test_library_exports_every_declared_function():
     lib = _lib.load()
     names = declared_functions()
-    assert len(names) == 12, names
+    assert len(names) == 13, names
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_lib.EXPORTS)
@@ -129,3 +129,14 @@ def test_compute_calls_need_cuda_tensors():
     k = torch.zeros(64, 1, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         api.compress_kv(cfg, k, k)
+
+
+def test_static_entry_point_rejects_oversized_and_bad_sizes_before_any_launch():
+    lib = _lib.load()
+    big = _params(L=300000, H=16, topk=8)
+    assert lib.s3r_workspace_bytes(ctypes.byref(big)) > _lib.S3R_STATIC_WORKSPACE_BYTES
+    assert lib.s3r_sparse_attn_fwd_static(ctypes.byref(big), A16, A16, A16, A16, A16, None,
+                                          None) == _lib.S3R_ERR_WORKSPACE
+    bad = _params(d=128)
+    assert lib.s3r_sparse_attn_fwd_static(ctypes.byref(bad), A16, A16, A16, A16, A16, None,
+                                          None) == _lib.S3R_ERR_UNSUPPORTED
