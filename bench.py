@@ -84,6 +84,23 @@ def algorithmic(cfg):
     }
 
 
+def rank_seed(base: int, rank: int) -> int:
+    """Seed of the independent layer a rank runs (weak scaling: one layer per GPU)."""
+    return base + 1000 * rank
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest value over all ranks (the job's step time); identity without a process group."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def physical_gpu(local: int) -> str:
     """nvidia-smi's name for CUDA device `local` of this process."""
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
@@ -246,7 +263,7 @@ def run_native(args, wl):
                                 device_id=dev)
 
     cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"])
-    seed = wl["seed"] + 1000 * rank  # an independent layer per GPU
+    seed = rank_seed(wl["seed"], rank)  # an independent layer per GPU
     x = synth.make_inputs(cfg.L, cfg.H, cfg.d, cfg.block, seed, device=dev)
     q, k, v, gates = x.q, x.k, x.v, x.gates
     sa = api.SparseAttention(cfg, dev)
@@ -274,11 +291,7 @@ def run_native(args, wl):
         torch.cuda.synchronize()
         launches = _lib.kernel_launches() - n0
     barrier()
-    ms = start.elapsed_time(end) / args.steps
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
     stage_ms = {n: statistics.mean(e.stage_ms()[n] for e in stage_ev) for n in _lib.STAGES}
 
     # end to end through pinned host buffers: H2D of the step's inputs, the call, D2H of out
@@ -294,10 +307,7 @@ def run_native(args, wl):
         sa.from_host(*host, out_h)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
     h2d = sum(t_.numel() * t_.element_size() for t_ in host)
     d2h = out_h.numel() * out_h.element_size()
     del host, out_h
