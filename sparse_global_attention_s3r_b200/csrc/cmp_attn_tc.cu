@@ -6,20 +6,23 @@
 //
 // Exact scores need normalised probabilities, so one launch makes two passes over the nb block
 // summaries of its 128-row query tile (two 64-row query blocks) and one head:
-//   pass A: S = Q Kc^T (tcgen05.mma into TMEM), running max / sum -> lse per row
+//   pass A: S = Q Kc^T (tcgen05.mma into TMEM), running sum of exp2 -> lse per row
 //   pass B: S again; P = exp2(S*scale*log2e - lse2) in fp32; the column sums of the fp32 P over
 //           each 64-row query block are that block's scores; bf16(P) is stored to TMEM and
 //           O_cmp += P Vc runs on the tensor cores with P as the TMEM operand.
+// Q is placed in TMEM once, so both products read their A operand from TMEM and shared memory
+// only serves the Kc/Vc tiles (a 128x64x16 MMA with A in shared memory would re-read 4 KB of Q
+// per instruction and be limited by shared-memory bandwidth).
 // Roles (352 threads, 11 warps):
-//   warp 0      TMA producer: Q once, then Kc (pass A) or Kc+Vc (pass B) 64-key tiles into a
-//               4-stage ring of 128-byte-swizzled shared-memory tiles
+//   warp 0      TMA producer: Kc (pass A) or Kc+Vc (pass B) 64-key tiles into a ring of
+//               128-byte-swizzled shared-memory tiles
 //   warp 1      TMEM owner (256 columns) and the single-thread tcgen05.mma issuer
 //   warps 2-9   softmax: warp w reads TMEM lane quadrant w%4 (32 rows) and column half
 //               (w-2)/4 (32 of the tile's 64 columns). With the 16x256b load shape a thread
 //               holds 4 rows x 8 columns, so a column sum is 3 in-thread adds plus 3 shuffle
 //               levels; P goes back with the matching 16x128b store shape.
 //   warp 10     adds the two row-quadrant partial column sums of each query block, writes scores
-// TMEM: S[2] (64 fp32 columns each), P[2] (64 bf16 = 32 columns each), O (64 fp32 columns).
+// TMEM columns: S[2] (64 fp32 each) | O (64 fp32) | Q (64 bf16 = 32) | P (64 bf16 = 32).
 // Every wait is an mbarrier wait bounded in time that also watches a CTA abort flag; on expiry
 // the kernel records S3R_DEV_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
 #include "s3r.h"
@@ -35,31 +38,40 @@ using namespace sm100;
 
 constexpr int kBM = 128;       // query rows per CTA (TMEM lanes)
 constexpr int kBN = 64;        // block summaries per tile
-constexpr int kStages = 4;     // shared-memory ring depth
+constexpr int kStages = 5;     // shared-memory ring depth
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = (3 + kSoftmaxWarps) * 32;  // producer, MMA, softmax x8, scores
 constexpr int kScoreWarp = 2 + kSoftmaxWarps;
-constexpr uint32_t kQBytes = kBM * 128;   // 16 KB
+constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
 constexpr uint32_t kKVBytes = kBN * 128;  // 8 KB
-constexpr uint32_t kColS = 0, kColP = 128, kColO = 192, kTmemCols = 256;
-constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0, 0);  // A=Q K-major, B=Kc K-major
+constexpr uint32_t kColS = 0, kColO = 128, kColQ = 192, kColP = 224, kTmemCols = 256;
+constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0, 0);  // A=Q (TMEM), B=Kc K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, 64, 0, 1);   // A=P (TMEM), B=Vc MN-major
+constexpr int kRed = 4;  // depth of the ring of per-tile partial column sums
+// pass A keeps a per-row reference max from the first tile; a row sum beyond 2^64 (or inf/nan)
+// means a later logit exceeded it by a lot, and only then is the reference moved
+constexpr float kSumLimit = 1.8446744073709552e19f;
+
+// Tuning: how many of a thread's 4 column pairs per row take the FMA-pipe polynomial 2^x instead
+// of MUFU.EX2 in pass B.
+#ifndef S3R_CMP_POLY_B
+#define S3R_CMP_POLY_B 1
+#endif
 
 struct __align__(8) Bars {
-  uint64_t q_full;
+  uint64_t q_ready;  // every softmax thread has stored its part of Q into TMEM
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_empty[2];
-  uint64_t red_full[2], red_empty[2];
+  uint64_t p_full, p_empty;
+  uint64_t red_full[kRed], red_empty[kRed];
   uint64_t stat;  // both column halves' row statistics of pass A are in shared memory
   uint64_t o_full, drain;
   uint64_t never;  // never signalled: waited on only under S3R_FLAG_TEST_TIMEOUT
 };
 
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKV = kQBytes;                           // stage s: K at +2s*8K, V +8K
-constexpr uint32_t kOffRed = kOffKV + kStages * 2 * kKVBytes;  // [2 par][4 quadrant][64] f32
-constexpr uint32_t kOffStat = kOffRed + 2 * 4 * 64 * 4;        // [2 halves][128 rows] float2
+constexpr uint32_t kOffKV = 0;                                 // stage s: K at +2s*8K, V +8K
+constexpr uint32_t kOffRed = kOffKV + kStages * 2 * kKVBytes;  // [kRed][4 quadrant][64] f32
+constexpr uint32_t kOffStat = kOffRed + kRed * 4 * 64 * 4;     // [2 halves][128 rows] float2
 constexpr uint32_t kOffBars = kOffStat + 2 * 128 * 8;
 constexpr uint32_t kOffMisc = kOffBars + sizeof(Bars);  // tmem base, abort flag
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
@@ -67,9 +79,10 @@ constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr uint32_t kSmemBytes = (kSmemUsed + 1024 > 80 * 1024 ? kSmemUsed + 1024 : 80 * 1024);
 
 struct CmpArgs {
-  float* lse;     // [H, L] natural log, may be null
-  float* o_cmp;   // [L, H, 64]
-  float* scores;  // [H, nqb, nb]
+  const uint16_t* q;  // [L, H, 64]
+  float* lse;         // [H, L] natural log, may be null
+  float* o_cmp;       // [L, H, 64]
+  float* scores;      // [H, nqb, nb]
   int64_t L, nb, nqb;
   int H;
   float scale_log2;
@@ -98,9 +111,24 @@ __device__ __forceinline__ void unpack_rows(const uint32_t (&a)[16], const uint3
     }
 }
 
+// sum over the 8 values of v of exp2(v * sl2 + off)
+__device__ __forceinline__ float exp2_sum8(const float (&v)[8], float sl2, float off) {
+  float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < 8; c += 2) {
+    const float2 x = __ffma2_rn(make_float2(v[c], v[c + 1]), make_float2(sl2, sl2),
+                                make_float2(off, off));
+    acc = __fadd2_rn(acc, make_float2(exp2_approx(x.x), exp2_approx(x.y)));
+  }
+  return acc.x + acc.y;
+}
+
+__device__ __forceinline__ float max8(const float (&v)[8]) {
+  return fmax3(fmax3(v[0], v[1], v[2]), fmax3(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+}
+
 __global__ void __launch_bounds__(kThreads, 2)
-    cmp_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
-                       const __grid_constant__ CUtensorMap tmK,
+    cmp_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const CmpArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_addr(smem_raw);
@@ -120,18 +148,20 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint64_t lim = a.limit_ns;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_ready, kSoftmaxThreads);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_empty[b], kSoftmaxWarps * 32);
-      mbar_init(&bars->p_full[b], kSoftmaxWarps * 32);
-      mbar_init(&bars->p_empty[b], 1);
-      mbar_init(&bars->red_full[b], kSoftmaxWarps);
-      mbar_init(&bars->red_empty[b], 1);
+      mbar_init(&bars->s_empty[b], kSoftmaxThreads);
+    }
+    mbar_init(&bars->p_full, kSoftmaxThreads);
+    mbar_init(&bars->p_empty, 1);
+    for (int r = 0; r < kRed; ++r) {
+      mbar_init(&bars->red_full[r], kSoftmaxWarps);
+      mbar_init(&bars->red_empty[r], 1);
     }
     mbar_init(&bars->stat, kSoftmaxWarps);
     mbar_init(&bars->o_full, 1);
@@ -141,7 +171,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
   }
@@ -156,8 +185,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       int issued = 0;
       bool ok = true;
-      mbar_arrive_expect_tx(&bars->q_full, kQBytes);
-      tma_load_2d(sbase + kOffQ, &tmQ, h * 64, static_cast<int32_t>(q0), &bars->q_full);
       for (int u = 0; u < 2 * nt; ++u) {
         const int stage = u % kStages, n = u / kStages;
         if (!mbar_wait(&bars->kv_empty[stage], (n & 1) ^ 1, abort, lim)) {
@@ -176,7 +203,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         raise_abort(abort, a.status);
         // let the copies already issued land before this CTA's shared memory is released
         int dummy = 0;
-        mbar_wait(&bars->q_full, 0, &dummy, lim);
         for (int u = issued - 1; u >= 0 && u >= issued - kStages; --u)
           mbar_wait(&bars->kv_full[u % kStages], (u / kStages) & 1, &dummy, lim);
       }
@@ -184,9 +210,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait(&bars->q_full, 0, abort, lim);
+      bool ok = mbar_wait(&bars->q_ready, 0, abort, lim);
       tc_fence_after();
-      const uint64_t dq = desc_sw128(sbase + kOffQ);
       auto qk = [&](int u, int c) -> bool {  // S[c&1] = Q Kc^T for ring use u
         const int stage = u % kStages;
         if (!mbar_wait(&bars->kv_full[stage], (u / kStages) & 1, abort, lim)) return false;
@@ -195,21 +220,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         const uint64_t dk = desc_sw128(sbase + kOffKV + stage * 2 * kKVBytes);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)  // 16 of d per step: 32 bytes into the swizzled row
-          mma_ss(tbase + kColS + b * kBN, dq + 2 * ks, dk + 2 * ks, kIdescQK, ks > 0);
+        for (int ks = 0; ks < 4; ++ks)  // 16 of d per step: 8 TMEM columns of Q, 32 B of Kc rows
+          mma_ts(tbase + kColS + b * kBN, tbase + kColQ + ks * 8, dk + 2 * ks, kIdescQK, ks > 0);
         return true;
       };
-      auto pv = [&](int t) -> bool {  // O += P[t&1] Vc for pass-B tile t
-        const int u = nt + t, stage = u % kStages, pb = t & 1;
-        if (!mbar_wait(&bars->p_full[pb], (t >> 1) & 1, abort, lim)) return false;
+      auto pv = [&](int t) -> bool {  // O += P Vc for pass-B tile t
+        const int u = nt + t, stage = u % kStages;
+        if (!mbar_wait(&bars->p_full, t & 1, abort, lim)) return false;
         tc_fence_after();
         const uint64_t dv = desc_sw128(sbase + kOffKV + stage * 2 * kKVBytes + kKVBytes);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)  // 16 keys per step: 16 rows x 128 B = 2048 B
-          mma_ts(tbase + kColO, tbase + kColP + pb * 32 + ks * 8, dv + 128 * ks, kIdescPV,
+          mma_ts(tbase + kColO, tbase + kColP + ks * 8, dv + 128 * ks, kIdescPV,
                  (t > 0 || ks > 0) ? 1u : 0u);
         tc_commit(&bars->kv_empty[stage]);
-        tc_commit(&bars->p_empty[pb]);
+        tc_commit(&bars->p_empty);
         return true;
       };
       for (int t = 0; ok && t < nt; ++t) {  // pass A
@@ -235,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (warp < kScoreWarp) {
     // ------------------------------------------------------------------ softmax warps
     const int g = warp & 3;             // TMEM lane quadrant this warp may access
-    const int half = (warp - 2) >> 2;   // which 32 of the tile's 64 columns
+    const int half = (warp - 2) >> 2;   // which 32 of the tile's 64 columns (and of Q's d)
     const int tq = lane & 3, tr = lane >> 2;
     const uint32_t tl0 = tbase + (static_cast<uint32_t>(g * 32) << 16);
     const uint32_t tl16 = tbase + (static_cast<uint32_t>(g * 32 + 16) << 16);
@@ -243,9 +268,29 @@ __global__ void __launch_bounds__(kThreads, 2)
     // column (within the tile) of value column c of this thread
     auto col_of = [&](int c) { return half * 32 + 8 * (c >> 1) + 2 * tq + (c & 1); };
     bool ok = true;
+
+    {  // Q row (this lane's row, this warp's 32 of d) into TMEM, the A operand of Q Kc^T
+      const int64_t row = q0 + g * 32 + lane;
+      uint32_t qv[16];
+      if (row < a.L) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + (row * a.H + h) * 64 + half * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 x = __ldg(src + j);
+          qv[4 * j] = x.x, qv[4 * j + 1] = x.y, qv[4 * j + 2] = x.z, qv[4 * j + 3] = x.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) qv[j] = 0u;
+      }
+      tmem_st32x16(tl0 + kColQ + half * 16, qv);
+      tmem_wait_st_keep16(qv);
+      tc_fence_before();
+      mbar_arrive(&bars->q_ready);
+    }
     if (a.flags & S3R_FLAG_TEST_TIMEOUT) ok = mbar_wait(&bars->never, 0, abort, lim);
 
-    // pass A: per-thread running max (raw logits) and sum over this thread's columns
+    // pass A: per row a reference max (raw logits) and the sum of exp2 relative to it
     float mr[4], l[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) mr[i] = -INFINITY, l[i] = 0.f;
@@ -268,23 +313,31 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int c = 0; c < 8; ++c)
           if (col_of(c) >= valid) v[0][c] = v[1][c] = v[2][c] = v[3][c] = -INFINITY;
       }
+      if (t == 0) {  // first tile: its row maxima become the reference (-inf if all masked)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float tmax = fmaxf(fmaxf(fmaxf(v[i][0], v[i][1]), fmaxf(v[i][2], v[i][3])),
-                           fmaxf(fmaxf(v[i][4], v[i][5]), fmaxf(v[i][6], v[i][7])));
-        const float mn = fmaxf(mr[i], tmax);
-        if (mn == -INFINITY) continue;  // no valid column seen yet by this thread
-        const float off = -mn * sl2;
-        l[i] *= exp2_approx(fmaf(mr[i], sl2, off));
-        mr[i] = mn;
-        float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < 8; c += 2) {
-          const float2 x = __ffma2_rn(make_float2(v[i][c], v[i][c + 1]), make_float2(sl2, sl2),
-                                      make_float2(off, off));
-          acc = __fadd2_rn(acc, make_float2(exp2_approx(x.x), exp2_approx(x.y)));
+        for (int i = 0; i < 4; ++i) {
+          mr[i] = max8(v[i]);
+          l[i] = mr[i] == -INFINITY ? 0.f : exp2_sum8(v[i], sl2, -mr[i] * sl2);
         }
-        l[i] += acc.x + acc.y;
+        continue;
+      }
+      // later tiles (tile 0 was full, so every reference is finite): straight-line sums for the
+      // four rows, one combined check for the rare row whose sum left the safe range
+      float sum[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sum[i] = l[i] + exp2_sum8(v[i], sl2, -mr[i] * sl2);
+      const bool safe = (sum[0] <= kSumLimit) & (sum[1] <= kSumLimit) & (sum[2] <= kSumLimit) &
+                        (sum[3] <= kSumLimit);
+      if (safe) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) l[i] = sum[i];
+      } else {  // a logit far above its reference: move the reference, redo this tile's sum
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float mn = fmaxf(mr[i], max8(v[i]));
+          l[i] = l[i] * exp2_approx((mr[i] - mn) * sl2) + exp2_sum8(v[i], sl2, -mn * sl2);
+          mr[i] = mn;
+        }
       }
     }
     // combine the statistics of the 4 threads of a quad and of the two column halves
@@ -339,8 +392,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int c = 0; c < 8; c += 2) {
           const float2 x = __ffma2_rn(make_float2(v[i][c], v[i][c + 1]), make_float2(sl2, sl2),
                                       make_float2(-lse2[i], -lse2[i]));
-          v[i][c] = exp2_approx(x.x);
-          v[i][c + 1] = exp2_approx(x.y);
+          if (c / 2 < S3R_CMP_POLY_B) {
+            const float2 e = exp2_poly5x2(x);
+            v[i][c] = e.x;
+            v[i][c + 1] = e.y;
+          } else {
+            v[i][c] = exp2_approx(x.x);
+            v[i][c + 1] = exp2_approx(x.y);
+          }
         }
       if (static_cast<int64_t>(t + 1) * kBN > a.nb) {  // ragged last tile: P = 0 past nb
         const int64_t valid = a.nb - static_cast<int64_t>(t) * kBN;
@@ -380,19 +439,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       // cs[0] is now the 32-row sum of value column c = tr of this lane
-      const int par = t & 1;
-      if (!(ok = mbar_wait(&bars->red_empty[par], ((t >> 1) & 1) ^ 1, abort, lim))) break;
+      const int par = t % kRed;
+      if (!(ok = mbar_wait(&bars->red_empty[par], ((t / kRed) & 1) ^ 1, abort, lim))) break;
       red[(par * 4 + g) * 64 + col_of(tr)] = cs[0];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->red_full[par]);
-      const int pb = t & 1;
-      if (!(ok = mbar_wait(&bars->p_empty[pb], ((t >> 1) & 1) ^ 1, abort, lim))) break;
-      tmem_st16x128_x4(tl0 + kColP + pb * 32 + half * 16, p0);
-      tmem_st16x128_x4(tl16 + kColP + pb * 32 + half * 16, p1);
+      // the single P buffer is free once the P*Vc product of tile t-1 has completed
+      if (!(ok = mbar_wait(&bars->p_empty, (t & 1) ^ 1, abort, lim))) break;
+      tmem_st16x128_x4(tl0 + kColP + half * 16, p0);
+      tmem_st16x128_x4(tl16 + kColP + half * 16, p1);
       tmem_wait_st_keep8(p0);
       tmem_wait_st_keep8(p1);
       tc_fence_before();
-      mbar_arrive(&bars->p_full[pb]);
+      mbar_arrive(&bars->p_full);
     }
     if (ok && (ok = mbar_wait(&bars->o_full, 0, abort, lim))) {
       tc_fence_after();
@@ -412,8 +471,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else {
     // ------------------------------------------------------------------ score writer
     for (int t = 0; t < nt; ++t) {
-      const int par = t & 1;
-      if (!mbar_wait(&bars->red_full[par], (t >> 1) & 1, abort, lim)) {
+      const int par = t % kRed;
+      if (!mbar_wait(&bars->red_full[par], (t / kRed) & 1, abort, lim)) {
         if (lane == 0) raise_abort(abort, a.status);
         break;
       }
@@ -447,17 +506,16 @@ __global__ void __launch_bounds__(kThreads, 2)
 cudaError_t launch_cmp_attn_tc(const Problem& p, const uint16_t* q, const uint16_t* kc,
                                const uint16_t* vc, float* lse, float* o_cmp, float* scores,
                                cudaStream_t st) {
-  CUtensorMap tq, tk, tv;
-  if (!make_tmap_head_rows(&tq, q, p.L, p.H, kBM) || !make_tmap_head_rows(&tk, kc, p.nb, p.H, kBN) ||
-      !make_tmap_head_rows(&tv, vc, p.nb, p.H, kBN))
+  CUtensorMap tk, tv;
+  if (!make_tmap_head_rows(&tk, kc, p.nb, p.H, kBN) || !make_tmap_head_rows(&tv, vc, p.nb, p.H, kBN))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(cmp_attn_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  CmpArgs a{lse, o_cmp, scores, p.L, p.nb, p.nqb, p.H, p.scale_log2, p.status,
+  CmpArgs a{q, lse, o_cmp, scores, p.L, p.nb, p.nqb, p.H, p.scale_log2, p.status,
             (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull, p.flags};
   dim3 grid(static_cast<unsigned>((p.L + kBM - 1) / kBM), p.H);
-  cmp_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
+  cmp_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tk, tv, a);
   count_launch();
   return cudaGetLastError();
 }

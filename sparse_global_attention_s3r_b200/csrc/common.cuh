@@ -61,6 +61,45 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
+// 2^x for two values on the FMA pipe (no MUFU): Cody-Waite reduction x = n + f with n the nearest
+// integer (f in [-1/2, 1/2]), a degree-5 minimax polynomial for 2^f fitted for this library
+// (relative error 7.5e-8 in exact arithmetic, 2.3e-7 evaluated in fp32, the accuracy of
+// ex2.approx), and 2^n added to the exponent field. x is clamped below at -126 (2^-126 ~ 1e-38
+// stands in for anything smaller, including -inf).
+__device__ __forceinline__ float2 exp2_poly5x2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound keeps round(x) in the low bits
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = make_float2(1.327647199e-03f, 1.327647199e-03f);
+  p = __ffma2_rn(p, f, make_float2(9.675541334e-03f, 9.675541334e-03f));
+  p = __ffma2_rn(p, f, make_float2(5.550713273e-02f, 5.550713273e-02f));
+  p = __ffma2_rn(p, f, make_float2(2.402211972e-01f, 2.402211972e-01f));
+  p = __ffma2_rn(p, f, make_float2(6.931469671e-01f, 6.931469671e-01f));
+  p = __ffma2_rn(p, f, make_float2(1.000000072e+00f, 1.000000072e+00f));
+  // the low mantissa bits of t hold n; shifted by 23 they land on the exponent field
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Round two non-negative finite floats to bf16 (nearest, ties to even) with integer operations
+// and pack them, `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16_int(float lo, float hi) {
+  uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+  a += 0x7FFFu + ((a >> 16) & 1u);
+  b += 0x7FFFu + ((b >> 16) & 1u);
+  return __byte_perm(a, b, 0x7632);
+}
+
+// max(a, b, c) in one instruction (sm_100 three-input max)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a tile of 128-byte rows
 // (64 bf16), XOR-swizzled so that 8 consecutive rows at one chunk hit 8 distinct bank groups.
 __device__ __forceinline__ uint32_t swz128(int row, int chunk) {
