@@ -53,9 +53,15 @@ constexpr int kRed = 4;  // depth of the ring of per-tile partial column sums
 constexpr float kSumLimit = 1.8446744073709552e19f;
 
 // Tuning: how many of a thread's 4 column pairs per row take the FMA-pipe polynomial 2^x instead
-// of MUFU.EX2 in pass B.
+// of MUFU.EX2, in pass A and in pass B. MUFU.EX2 sustains 16 per clock per SM and the FMA pipe
+// could evaluate about as many polynomials, but this kernel is latency-bound rather than
+// MUFU-bound (measured at 1000 views: 0/0 -> 285 ms, 0/1 -> 292 ms, 1/1 -> 309 ms), so both
+// default to 0.
+#ifndef S3R_CMP_POLY_A
+#define S3R_CMP_POLY_A 0
+#endif
 #ifndef S3R_CMP_POLY_B
-#define S3R_CMP_POLY_B 1
+#define S3R_CMP_POLY_B 0
 #endif
 
 struct __align__(8) Bars {
@@ -111,14 +117,19 @@ __device__ __forceinline__ void unpack_rows(const uint32_t (&a)[16], const uint3
     }
 }
 
-// sum over the 8 values of v of exp2(v * sl2 + off)
+// sum over the 8 values of v of exp2(v * sl2 + off); the first `npoly` column pairs use the
+// FMA-pipe polynomial, the others MUFU.EX2
+template <int npoly>
 __device__ __forceinline__ float exp2_sum8(const float (&v)[8], float sl2, float off) {
   float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < 8; c += 2) {
     const float2 x = __ffma2_rn(make_float2(v[c], v[c + 1]), make_float2(sl2, sl2),
                                 make_float2(off, off));
-    acc = __fadd2_rn(acc, make_float2(exp2_approx(x.x), exp2_approx(x.y)));
+    if (c / 2 < npoly)
+      acc = __fadd2_rn(acc, exp2_poly5x2(x));
+    else
+      acc = __fadd2_rn(acc, make_float2(exp2_approx(x.x), exp2_approx(x.y)));
   }
   return acc.x + acc.y;
 }
@@ -317,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           mr[i] = max8(v[i]);
-          l[i] = mr[i] == -INFINITY ? 0.f : exp2_sum8(v[i], sl2, -mr[i] * sl2);
+          l[i] = mr[i] == -INFINITY ? 0.f : exp2_sum8<S3R_CMP_POLY_A>(v[i], sl2, -mr[i] * sl2);
         }
         continue;
       }
@@ -325,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       // four rows, one combined check for the rare row whose sum left the safe range
       float sum[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) sum[i] = l[i] + exp2_sum8(v[i], sl2, -mr[i] * sl2);
+      for (int i = 0; i < 4; ++i) sum[i] = l[i] + exp2_sum8<S3R_CMP_POLY_A>(v[i], sl2, -mr[i] * sl2);
       const bool safe = (sum[0] <= kSumLimit) & (sum[1] <= kSumLimit) & (sum[2] <= kSumLimit) &
                         (sum[3] <= kSumLimit);
       if (safe) {
@@ -335,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float mn = fmaxf(mr[i], max8(v[i]));
-          l[i] = l[i] * exp2_approx((mr[i] - mn) * sl2) + exp2_sum8(v[i], sl2, -mn * sl2);
+          l[i] = l[i] * exp2_approx((mr[i] - mn) * sl2) + exp2_sum8<S3R_CMP_POLY_A>(v[i], sl2, -mn * sl2);
           mr[i] = mn;
         }
       }
