@@ -350,6 +350,9 @@ def run_native(args, wl):
     for n in _lib.STAGES:
         b_, u_ = work["stage_work"][n]
         s_ = stage_ms[n] / 1e3
+        if s_ < 1e-5:  # no launch in this stage (top-k selected inside the compressed stage)
+            stages[n] = {"ms": stage_ms[n], "launched": False}
+            continue
         stages[n] = {"ms": stage_ms[n],
                      ("GB/s" if b_ == "hbm" else "TFLOP/s"): u_ / s_ / (1e9 if b_ == "hbm" else 1e12)}
     line = {

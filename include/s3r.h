@@ -95,7 +95,8 @@ typedef struct {
 /* Stages of s3r_sparse_attn_fwd, in launch order (one kernel each). */
 #define S3R_STAGE_POOL 0        /* K/V block pooling */
 #define S3R_STAGE_CMP 1         /* compressed attention (lse pass, then O_cmp and block scores) */
-#define S3R_STAGE_TOPK 2        /* per-query-block top-k */
+#define S3R_STAGE_TOPK 2        /* per-query-block top-k; empty (no launch) when topk <= 32,
+                                   where the compressed stage selects the blocks on the fly */
 #define S3R_STAGE_SEL_COMBINE 3 /* selection attention fused with the gated combine */
 #define S3R_NUM_STAGES 4
 
@@ -165,7 +166,10 @@ s3r_status s3r_gate_combine(const s3r_params* params, const float* o_cmp, const 
                             const float* gate_logits, s3r_bf16* out, s3r_stream stream);
 
 /* The whole path in one call: pooling, compressed attention and scores, top-k, selection
- * attention fused with the gated combine.
+ * attention fused with the gated combine. For topk <= 32 the compressed-attention kernel keeps a
+ * running top-k of every query block while it produces the scores, so the [H, nqb, nb] score
+ * matrix is never written (3 kernel launches); larger topk materialise it in the workspace and run
+ * s3r_topk_blocks' kernel (4 launches). Both select the same blocks.
  *   q, k, v     [L, H, d] bf16; gate_logits [L, H, 2] fp32 (read)
  *   out         [L, H, d] bf16 (written)
  *   idx_out     [H, nqb, topk] int32 (written if not NULL)

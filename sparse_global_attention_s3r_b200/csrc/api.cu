@@ -50,6 +50,8 @@ s3r_status launched(cudaError_t e) { return e == cudaSuccess ? S3R_OK : S3R_ERR_
 // Workspace of the fused call, every region 256-byte aligned:
 //   status word | Kc [nb,H,d] bf16 | Vc | O_cmp [L,H,d] f32 | scores [H,nqb,nb] f32
 //   | idx [H,nqb,k] i32
+// The score matrix is only materialised when k > kFusedTopkMax; otherwise the compressed-branch
+// kernel selects the top-k on the fly and the scores region is empty.
 struct Workspace {
   size_t status, kc, vc, o_cmp, scores, idx, total;
 };
@@ -69,7 +71,7 @@ Workspace layout(const Problem& p) {
   w.kc = take(static_cast<size_t>(p.nb) * HD * 2);
   w.vc = take(static_cast<size_t>(p.nb) * HD * 2);
   w.o_cmp = take(static_cast<size_t>(p.L) * HD * 4);
-  w.scores = take(static_cast<size_t>(p.H) * p.nqb * p.nb * 4);
+  w.scores = take(p.k > kFusedTopkMax ? static_cast<size_t>(p.H) * p.nqb * p.nb * 4 : 0);
   w.idx = take(static_cast<size_t>(p.H) * p.nqb * p.k * 4);
   w.total = off;
   return w;
@@ -113,10 +115,12 @@ int fused_forward(const s3r_params* params, const uint16_t* q, const uint16_t* k
   if (mark(0) != cudaSuccess) return S3R_ERR_CUDA;
   if ((st = launched(launch_pool_kv(p, k, v, kc, vc, stream))) != S3R_OK) return st;
   if (mark(1) != cudaSuccess) return S3R_ERR_CUDA;
-  if ((st = launched(launch_cmp_attn_tc(p, q, kc, vc, nullptr, o_cmp, scores, stream))) != S3R_OK)
+  const bool fused_topk = p.k <= kFusedTopkMax;
+  if ((st = launched(launch_cmp_attn_tc(p, q, kc, vc, nullptr, o_cmp, fused_topk ? nullptr : scores,
+                                        fused_topk ? idx : nullptr, stream))) != S3R_OK)
     return st;
   if (mark(2) != cudaSuccess) return S3R_ERR_CUDA;
-  if ((st = launched(launch_topk(p, scores, idx, stream))) != S3R_OK) return st;
+  if (!fused_topk && (st = launched(launch_topk(p, scores, idx, stream))) != S3R_OK) return st;
   if (mark(3) != cudaSuccess) return S3R_ERR_CUDA;
   st = launched(launch_sel_attn(p, q, k, v, idx, nullptr, o_cmp, gate_logits, out, stream));
   if (st != S3R_OK) return st;
@@ -181,7 +185,7 @@ s3r_status s3r_cmp_attn_and_score(const s3r_params* params, const s3r_bf16* q,
   if (!aligned16(q) || !aligned16(k_cmp) || !aligned16(v_cmp) || !aligned16(o_cmp) ||
       !aligned16(lse) || !aligned16(scores))
     return S3R_ERR_INVALID_ARG;
-  return launched(launch_cmp_attn_tc(p, q, k_cmp, v_cmp, lse, o_cmp, scores, stream));
+  return launched(launch_cmp_attn_tc(p, q, k_cmp, v_cmp, lse, o_cmp, scores, nullptr, stream));
 }
 
 s3r_status s3r_topk_blocks(const s3r_params* params, const float* scores, int32_t* idx,

@@ -21,7 +21,11 @@
 //               (w-2)/4 (32 of the tile's 64 columns). With the 16x256b load shape a thread
 //               holds 4 rows x 8 columns, so a column sum is 3 in-thread adds plus 3 shuffle
 //               levels; P goes back with the matching 16x128b store shape.
-//   warp 10     adds the two row-quadrant partial column sums of each query block, writes scores
+//   warp 10     adds the two row-quadrant partial column sums of each query block; writes the
+//               scores and/or keeps each query block's running top-k (k <= 32) in registers:
+//               lane i holds the i-th largest key (score bits << 32 | ~block index), a tile's
+//               candidates are tested against the k-th key with one ballot and the rare winners
+//               are inserted by a warp-wide ordered shift, so the score matrix never exists
 // TMEM columns: S[2] (64 fp32 each) | O (64 fp32) | Q (64 bf16 = 32) | P (64 bf16 = 32).
 // Every wait is an mbarrier wait bounded in time that also watches a CTA abort flag; on expiry
 // the kernel records S3R_DEV_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
@@ -88,7 +92,9 @@ struct CmpArgs {
   const uint16_t* q;  // [L, H, 64]
   float* lse;         // [H, L] natural log, may be null
   float* o_cmp;       // [L, H, 64]
-  float* scores;      // [H, nqb, nb]
+  float* scores;      // [H, nqb, nb], may be null
+  int32_t* idx;       // [H, nqb, topk] streaming top-k output (topk <= 32), may be null
+  int topk;
   int64_t L, nb, nqb;
   int H;
   float scale_log2;
@@ -96,6 +102,24 @@ struct CmpArgs {
   uint64_t limit_ns;
   uint32_t flags;
 };
+
+// Insert this lane's candidate key c into the warp's sorted list (lane i holds the i-th largest
+// key; lanes 0..k-1 are the current top-k) if it beats the k-th key. Keys are unique.
+__device__ __forceinline__ void topk_offer(uint64_t& mine, uint64_t c, int k, int lane) {
+  uint64_t thr = __shfl_sync(0xffffffffu, mine, k - 1);
+  unsigned pending = __ballot_sync(0xffffffffu, c > thr);
+  while (pending) {
+    const int src = __ffs(pending) - 1;
+    const uint64_t cand = __shfl_sync(0xffffffffu, c, src);
+    const int pos = __popc(__ballot_sync(0xffffffffu, mine > cand));  // < k since cand > thr
+    const uint64_t up = __shfl_up_sync(0xffffffffu, mine, 1);
+    if (lane > pos) mine = up;
+    if (lane == pos) mine = cand;
+    thr = __shfl_sync(0xffffffffu, mine, k - 1);
+    pending &= ~(1u << src);
+    pending &= __ballot_sync(0xffffffffu, c > thr);
+  }
+}
 
 __device__ __forceinline__ void raise_abort(volatile int* abort, uint32_t* status) {
   *abort = 1;
@@ -480,28 +504,49 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     if (!ok) raise_abort(abort, a.status);
   } else {
-    // ------------------------------------------------------------------ score writer
+    // ------------------------------------------------------------------ scores / top-k
+    uint64_t best[2] = {0ull, 0ull};  // below every real key
+    bool ok = true;
     for (int t = 0; t < nt; ++t) {
       const int par = t % kRed;
       if (!mbar_wait(&bars->red_full[par], (t / kRed) & 1, abort, lim)) {
         if (lane == 0) raise_abort(abort, a.status);
+        ok = false;
         break;
       }
 #pragma unroll
       for (int qb = 0; qb < 2; ++qb) {
         const int64_t i = qtile * 2 + qb;
         if (i >= a.nqb) continue;
-        float* dst = a.scores + (static_cast<int64_t>(h) * a.nqb + i) * a.nb;
+        float* dst = a.scores ? a.scores + (static_cast<int64_t>(h) * a.nqb + i) * a.nb : nullptr;
+        uint64_t key[2];
 #pragma unroll
         for (int hc = 0; hc < 2; ++hc) {
           const int cc = hc * 32 + lane;
           const int64_t col = static_cast<int64_t>(t) * kBN + cc;
-          if (col < a.nb)
-            dst[col] = red[(par * 4 + 2 * qb) * 64 + cc] + red[(par * 4 + 2 * qb + 1) * 64 + cc];
+          const float sc =
+              red[(par * 4 + 2 * qb) * 64 + cc] + red[(par * 4 + 2 * qb + 1) * 64 + cc];
+          if (dst && col < a.nb) dst[col] = sc;
+          key[hc] = col < a.nb ? (static_cast<uint64_t>(__float_as_uint(sc)) << 32) |
+                                     static_cast<uint32_t>(~static_cast<uint32_t>(col))
+                               : 0ull;
+        }
+        if (a.idx) {
+          topk_offer(best[qb], key[0], a.topk, lane);
+          topk_offer(best[qb], key[1], a.topk, lane);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->red_empty[par]);
+    }
+    if (ok && a.idx) {
+#pragma unroll
+      for (int qb = 0; qb < 2; ++qb) {
+        const int64_t i = qtile * 2 + qb;
+        if (i < a.nqb && lane < a.topk)
+          a.idx[(static_cast<int64_t>(h) * a.nqb + i) * a.topk + lane] =
+              static_cast<int32_t>(~static_cast<uint32_t>(best[qb] & 0xFFFFFFFFull));
+      }
     }
   }
 
@@ -516,14 +561,15 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 cudaError_t launch_cmp_attn_tc(const Problem& p, const uint16_t* q, const uint16_t* kc,
                                const uint16_t* vc, float* lse, float* o_cmp, float* scores,
-                               cudaStream_t st) {
+                               int32_t* idx, cudaStream_t st) {
+  if (idx && p.k > kFusedTopkMax) return cudaErrorInvalidValue;
   CUtensorMap tk, tv;
   if (!make_tmap_head_rows(&tk, kc, p.nb, p.H, kBN) || !make_tmap_head_rows(&tv, vc, p.nb, p.H, kBN))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(cmp_attn_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  CmpArgs a{q, lse, o_cmp, scores, p.L, p.nb, p.nqb, p.H, p.scale_log2, p.status,
+  CmpArgs a{q, lse, o_cmp, scores, idx, p.k, p.L, p.nb, p.nqb, p.H, p.scale_log2, p.status,
             (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull, p.flags};
   dim3 grid(static_cast<unsigned>((p.L + kBM - 1) / kBM), p.H);
   cmp_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tk, tv, a);

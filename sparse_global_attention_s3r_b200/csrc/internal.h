@@ -23,10 +23,14 @@ struct Problem {
 // Each launcher enqueues one kernel on `st` and returns cudaGetLastError().
 cudaError_t launch_pool_kv(const Problem& p, const uint16_t* k, const uint16_t* v, uint16_t* kc,
                            uint16_t* vc, cudaStream_t st);
-// Compression branch in one launch (both passes): lse (may be null), O_cmp and scores.
+// Largest top-k the compressed-branch kernel selects on the fly (one key per lane of a warp).
+constexpr int kFusedTopkMax = 32;
+
+// Compression branch in one launch (both passes): O_cmp, and any of lse, scores (the block score
+// matrix) and idx (the per-query-block top-k, topk <= kFusedTopkMax), each may be null.
 cudaError_t launch_cmp_attn_tc(const Problem& p, const uint16_t* q, const uint16_t* kc,
                                const uint16_t* vc, float* lse, float* o_cmp, float* scores,
-                               cudaStream_t st);
+                               int32_t* idx, cudaStream_t st);
 cudaError_t launch_topk(const Problem& p, const float* scores, int32_t* idx, cudaStream_t st);
 // o_sel != nullptr: write the selection output (fp32). Otherwise fuse the gated combine:
 // read o_cmp and gates and write out (bf16).

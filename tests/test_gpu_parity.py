@@ -24,6 +24,7 @@ CASES = {  # name: (L, H, b, k, seed)
     "tail_of_one_row": (65, 1, 32, 3, 6),
     "dense_selection": (1000, 2, 64, 16, 7),  # k = nb
     "multi_tile_keys": (9000, 2, 32, 9, 8),  # nb = 282: several 64-key tiles + ragged tile
+    "k_above_32": (3000, 2, 32, 40, 9),  # the fused path materialises the scores for k > 32
 }
 
 
@@ -210,12 +211,27 @@ def test_dense_selection_equals_dense_attention(dev):
     check_close("dense", f64(o), ref, 2.0 ** -8 * np.abs(f64(x.v)).max() + 1e-6, rl2=4e-3)
 
 
-def test_launch_counter_counts_kernels(dev):
-    cfg, pb, x, d = inputs("tiny", dev)
+@pytest.mark.parametrize("name,launches", [("tiny", 3), ("k_above_32", 4)])
+def test_launch_counter_counts_kernels(dev, name, launches):
+    cfg, pb, x, d = inputs(name, dev)
     n0 = _lib.kernel_launches()
     api.sparse_attn_fwd(cfg, d["q"], d["k"], d["v"], d["gates"])
     torch.cuda.synchronize()
-    assert _lib.kernel_launches() - n0 == 4
+    assert _lib.kernel_launches() - n0 == launches
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_b32_odd_k", "multi_tile_keys", "dense_selection"])
+def test_streaming_topk_equals_the_topk_kernel(dev, name):
+    """The top-k the compressed kernel keeps on the fly equals s3r_topk_blocks on the same
+    (bit-identical) scores, order included."""
+    cfg, pb, x, d = inputs(name, dev)
+    kc, vc = api.compress_kv(cfg, d["k"], d["v"])
+    _, _, scores = api.cmp_attn_and_score(cfg, d["q"], kc, vc)
+    want = api.topk_blocks(cfg, scores)
+    got = torch.empty_like(want)
+    api.sparse_attn_fwd(cfg, d["q"], d["k"], d["v"], d["gates"], idx_out=got)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(got.cpu().numpy(), want.cpu().numpy())
 
 
 def test_bounded_wait_timeout_is_reported_and_the_context_survives(dev):
