@@ -1,0 +1,498 @@
+// sel_attn_tc.cu -- selection branch on the sm_100a tensor cores (tcgen05 + TMEM + TMA),
+// optionally fused with the gated aggregation.
+//
+// Speed3R (gist.science summary, "Methodologie" §1 "Selectie-tak"): fine-grained attention only
+// on the tokens of the top-k key blocks chosen by the compression branch; §2 "Gated Aggregation":
+// a per-token gate mixes the two branch outputs (two independent sigmoid gates here).
+//
+// One CTA = two 64-row query blocks of one head (a 128-row tile, one TMEM lane per row). The k
+// selected blocks of a query block form a list of k*b tokens, walked in steps of 64 tokens. Each
+// step gathers, with 2-D TMA boxes straight from K/V [L, H, 64], the next 64 tokens of each of the
+// two query blocks into one 128-token K tile and V tile (rows past L read as zeros). Then
+//   S = Q K^T       tcgen05.mma, M=128 x N=128: rows of query block 0 only use columns 0-63 (its
+//                   tokens), rows of block 1 columns 64-127
+//   O += P V        tcgen05.mma with bf16 P as the TMEM operand; the P columns of the other
+//                   block's tokens are zero (written once), so the product stays block-diagonal
+// The MMA work is twice what a 64-row tile would need, in exchange for the 128-lane layouts.
+// Softmax: one warp per TMEM lane quadrant (32 rows of one query block), 4 rows x 16 columns per
+// thread with the 16x256b load shape; the reference max of a row is fixed at the first step and
+// moves (with O and the row sum rescaled in TMEM once the previous product has completed) only if
+// a logit exceeds it by 32 in base-2 units, so the bf16 P stays below 2^32.
+// Roles (224 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-5 softmax
+// (warp w holds lane quadrant w%4), warp 6 idle. TMEM: S (128 cols) | O (64) | P (64 = 128 keys).
+// Every wait is bounded in time and watches a CTA abort flag (S3R_DEV_TIMEOUT on expiry).
+#include "s3r.h"
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+#include "tma_host.h"
+
+namespace s3r {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;                 // rows: two 64-row query blocks
+constexpr int kStep = 64;                // tokens per query block per step
+constexpr int kStages = 2;               // K/V tile ring depth
+constexpr int kThreads = 224;            // 7 warps
+constexpr int kSoftmaxThreads = 128;
+constexpr uint32_t kQBytes = kBM * 128;  // 16 KB
+constexpr uint32_t kTileBytes = 2 * kStep * 128;  // 128 tokens x 128 B = 16 KB (K or V)
+constexpr uint32_t kColS = 0, kColO = 128, kColP = 192, kTmemCols = 256;
+constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, 2 * kStep, 0, 0);  // Q K-major, K K-major
+constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, 64, 0, 1);          // P TMEM, V MN-major
+constexpr float kMoveRef = 32.f;  // base-2 margin before a row's reference max moves
+constexpr int kIdxCache = 256;    // selection lists up to this length are staged in shared memory
+
+struct __align__(8) Bars {
+  uint64_t q_full;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full, s_empty;
+  uint64_t p_full, p_empty;
+  uint64_t o_full, drain;
+};
+
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKV = kQBytes;  // stage s: K tile at +2s*16K, V tile at +16K
+constexpr uint32_t kOffIdx = kOffKV + kStages * 2 * kTileBytes;  // [2][kIdxCache] int32
+constexpr uint32_t kOffBars = kOffIdx + 2 * kIdxCache * 4;
+constexpr uint32_t kOffMisc = kOffBars + sizeof(Bars);
+constexpr uint32_t kSmemUsed = kOffMisc + 16;
+// more than a third of an SM's shared memory: at most two CTAs per SM, so TMEM always fits
+constexpr uint32_t kSmemBytes = (kSmemUsed + 1024 > 80 * 1024 ? kSmemUsed + 1024 : 80 * 1024);
+
+struct SelArgs {
+  const int32_t* idx;  // [H, nqb, topk]
+  float* o_sel;        // [L, H, 64] fp32, or null for the fused combine
+  const float* o_cmp;  // [L, H, 64] fp32 (fused combine)
+  const float* gates;  // [L, H, 2]  fp32 (fused combine)
+  uint16_t* out;       // [L, H, 64] bf16 (fused combine)
+  int64_t L, nb, nqb;
+  int64_t nb_full;  // key blocks that lie wholly below L
+  int H, b, lb, topk, nsteps;  // lb = log2(b)
+  float scale_log2;
+  uint32_t flags;
+  uint32_t* status;
+  uint64_t limit_ns;
+};
+
+__device__ __forceinline__ void raise_abort(volatile int* abort, uint32_t* status) {
+  *abort = 1;
+  set_status(status, S3R_DEV_TIMEOUT);
+}
+
+// Block index of entry s of a selection list, clamped into range (out-of-range entries are
+// loaded as block 0 and masked).
+__device__ __forceinline__ int64_t sel_block(const int32_t* list, int s, int k, int64_t nb,
+                                             bool& ok) {
+  if (s >= k) {
+    ok = false;
+    return 0;
+  }
+  const int64_t j = list[s];
+  ok = j >= 0 && j < nb;
+  return ok ? j : 0;
+}
+
+// 128 registers: two CTAs of 7 warps per SM (at most 4 warps x 4096 registers per SM
+// sub-partition, whose register file holds 16K)
+__global__ void __maxnreg__(128)
+    sel_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const SelArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_addr(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+  const uint32_t sbase = smem_addr(smem);
+  Bars* bars = reinterpret_cast<Bars*>(smem + kOffBars);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int64_t qt = blockIdx.x;
+  const int64_t q0 = qt * kBM;
+  const uint64_t lim = a.limit_ns;
+  const int ns = a.nsteps;
+  // the two query blocks' selection lists (a missing second block reuses the first one's)
+  const int32_t* glist[2];
+  int32_t* slist = reinterpret_cast<int32_t*>(smem + kOffIdx);
+  const bool cached = a.topk <= kIdxCache;
+  for (int qb = 0; qb < 2; ++qb) {
+    const int64_t i = qt * 2 + qb < a.nqb ? qt * 2 + qb : qt * 2;
+    glist[qb] = a.idx + (static_cast<int64_t>(h) * a.nqb + i) * a.topk;
+    if (cached)
+      for (int s = threadIdx.x; s < a.topk; s += kThreads) slist[qb * kIdxCache + s] = glist[qb][s];
+  }
+  const int32_t* list_of[2] = {cached ? slist : glist[0], cached ? slist + kIdxCache : glist[1]};
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_empty, kSoftmaxThreads);
+    mbar_init(&bars->p_full, kSoftmaxThreads);
+    mbar_init(&bars->p_empty, 1);
+    mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer (gather)
+    if (lane == 0) {
+      bool ok = true;
+      int issued = 0;
+      mbar_arrive_expect_tx(&bars->q_full, kQBytes);
+      tma_load_2d(sbase + kOffQ, &tmQ, h * 64, static_cast<int32_t>(q0), &bars->q_full);
+      const int box = a.b < kStep ? a.b : kStep;  // rows per TMA box: 32 for b = 32, else 64
+      for (int t = 0; t < ns; ++t) {
+        const int stage = t % kStages;
+        if (!mbar_wait(&bars->kv_empty[stage], ((t / kStages) & 1) ^ 1, abort, lim)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sk = sbase + kOffKV + stage * 2 * kTileBytes;
+        mbar_arrive_expect_tx(&bars->kv_full[stage], 2 * kTileBytes);
+        for (int qb = 0; qb < 2; ++qb) {
+          const int32_t* list = list_of[qb];
+          for (int part = 0; part < kStep / box; ++part) {
+            // position of this box in the query block's token list, and its first token
+            const int pos = t * kStep + part * box;
+            bool valid;
+            const int64_t j = sel_block(list, pos >> a.lb, a.topk, a.nb, valid);
+            const int64_t tok = j * a.b + (pos & (a.b - 1));
+            const uint32_t row_off = (qb * kStep + part * box) * 128;
+            tma_load_2d(sk + row_off, &tmK, h * 64, static_cast<int32_t>(tok), &bars->kv_full[stage]);
+            tma_load_2d(sk + kTileBytes + row_off, &tmV, h * 64, static_cast<int32_t>(tok),
+                        &bars->kv_full[stage]);
+          }
+        }
+        issued = t + 1;
+      }
+      if (!ok) {
+        raise_abort(abort, a.status);
+        int dummy = 0;
+        mbar_wait(&bars->q_full, 0, &dummy, lim);
+        for (int t = issued - 1; t >= 0 && t >= issued - kStages; --t)
+          mbar_wait(&bars->kv_full[t % kStages], (t / kStages) & 1, &dummy, lim);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(&bars->q_full, 0, abort, lim);
+      tc_fence_after();
+      const uint64_t dq = desc_sw128(sbase + kOffQ);
+      auto qk = [&](int t) -> bool {
+        const int stage = t % kStages;
+        if (!mbar_wait(&bars->kv_full[stage], (t / kStages) & 1, abort, lim)) return false;
+        if (!mbar_wait(&bars->s_empty, (t & 1) ^ 1, abort, lim)) return false;
+        tc_fence_after();
+        const uint64_t dk = desc_sw128(sbase + kOffKV + stage * 2 * kTileBytes);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ss(tbase + kColS, dq + 2 * ks, dk + 2 * ks, kIdescQK, ks > 0);
+        tc_commit(&bars->s_full);
+        return true;
+      };
+      auto pv = [&](int t) -> bool {
+        const int stage = t % kStages;
+        if (!mbar_wait(&bars->p_full, t & 1, abort, lim)) return false;
+        tc_fence_after();
+        const uint64_t dv = desc_sw128(sbase + kOffKV + stage * 2 * kTileBytes + kTileBytes);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)  // 128 keys in steps of 16: 16 rows x 128 B = 2048 B
+          mma_ts(tbase + kColO, tbase + kColP + ks * 8, dv + 128 * ks, kIdescPV,
+                 (t > 0 || ks > 0) ? 1u : 0u);
+        tc_commit(&bars->kv_empty[stage]);
+        tc_commit(&bars->p_empty);
+        return true;
+      };
+      for (int t = 0; ok && t < ns; ++t) {
+        if (!(ok = qk(t))) break;
+        if (t > 0 && !(ok = pv(t - 1))) break;
+      }
+      if (ok) ok = pv(ns - 1);
+      if (ok) {
+        tc_commit(&bars->o_full);
+      } else {
+        raise_abort(abort, a.status);
+        int dummy = 0;
+        tc_commit(&bars->drain);
+        mbar_wait(&bars->drain, 0, &dummy, lim);
+      }
+    }
+  } else if (warp <= 5) {
+    // ------------------------------------------------------------------ softmax warps
+    const int g = warp & 3;       // TMEM lane quadrant: rows 32g .. 32g+31
+    const int qb = g >> 1;        // which of the two query blocks these rows belong to
+    const int tq = lane & 3, tr = lane >> 2;
+    const uint32_t tl0 = tbase + (static_cast<uint32_t>(g * 32) << 16);
+    const uint32_t tl16 = tbase + (static_cast<uint32_t>(g * 32 + 16) << 16);
+    const float sl2 = a.scale_log2;
+    const int32_t* list = list_of[qb];
+    bool ok = true;
+
+    {  // the other query block's P columns of these rows stay zero for the whole kernel
+      const uint32_t z[32] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
+                              0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      tmem_st32(tl0 + kColP + (1 - qb) * 32, z);
+      tmem_wait_st_regs(z);
+    }
+
+    // value v[i][c]: row tr + 8i of the quadrant, column c of this thread within the step's 64
+    // columns of the query block: 32*(c/8) + 8*((c%8)/2) + 2*tq + c%2
+    auto col_of = [&](int c) { return 32 * (c >> 3) + 8 * ((c & 7) >> 1) + 2 * tq + (c & 1); };
+    float mr[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mr[i] = -INFINITY, l[i] = 0.f;
+
+    for (int t = 0; ok && t < ns; ++t) {
+      if (!(ok = mbar_wait(&bars->s_full, t & 1, abort, lim))) break;
+      tc_fence_after();
+      uint32_t r[4][16];
+      tmem_ld16x256_x4(tl0 + kColS + qb * 64, r[0]);
+      tmem_ld16x256_x4(tl16 + kColS + qb * 64, r[1]);
+      tmem_ld16x256_x4(tl0 + kColS + qb * 64 + 32, r[2]);
+      tmem_ld16x256_x4(tl16 + kColS + qb * 64 + 32, r[3]);
+      tmem_wait_ld_n<16>(r[0]);
+      tmem_wait_ld_n<16>(r[1]);
+      tmem_wait_ld_n<16>(r[2]);
+      tmem_wait_ld_n<16>(r[3]);
+      tc_fence_before();
+      mbar_arrive(&bars->s_empty);
+      float v[4][16];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int rep = 0; rep < 4; ++rep)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = hh * 8 + 2 * rep + e;
+            v[0][c] = __uint_as_float(r[2 * hh][4 * rep + e]);
+            v[1][c] = __uint_as_float(r[2 * hh][4 * rep + 2 + e]);
+            v[2][c] = __uint_as_float(r[2 * hh + 1][4 * rep + e]);
+            v[3][c] = __uint_as_float(r[2 * hh + 1][4 * rep + 2 + e]);
+          }
+      // columns whose token does not exist: past k*b, an out-of-range index, or past L. A
+      // 64-token step spans at most two selected blocks (b >= 32).
+      {
+        const int p0 = t * kStep;
+        const int s_lo = p0 >> a.lb, s_hi = (p0 + kStep - 1) >> a.lb;
+        bool ok_lo, ok_hi;
+        const int64_t j_lo = sel_block(list, s_lo, a.topk, a.nb, ok_lo);
+        const int64_t j_hi = sel_block(list, s_hi, a.topk, a.nb, ok_hi);
+        if ((a.flags & S3R_FLAG_DEBUG_CHECKS) && lane == 0 &&
+            ((!ok_lo && s_lo < a.topk) || (!ok_hi && s_hi < a.topk)))
+          set_status(a.status, S3R_DEV_BAD_INDEX);
+        // the same for the whole warp; false only on a list's last step or at the partial block
+        const bool all_valid = ok_lo && ok_hi && j_lo < a.nb_full && j_hi < a.nb_full;
+        if (!all_valid) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int pos = p0 + col_of(c);
+            const bool lo = (pos >> a.lb) == s_lo;
+            const bool valid = lo ? ok_lo : ok_hi;
+            const int64_t tok = (lo ? j_lo : j_hi) * a.b + (pos & (a.b - 1));
+            if (!valid || tok >= a.L) v[0][c] = v[1][c] = v[2][c] = v[3][c] = -INFINITY;
+          }
+        }
+      }
+      // row maxima of this step (the quad's 4 threads hold the same rows)
+      float tmax[4];
+      bool move = false;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float m = fmax3(fmax3(v[i][0], v[i][1], v[i][2]), fmax3(v[i][3], v[i][4], v[i][5]),
+                        fmax3(v[i][6], v[i][7], v[i][8]));
+        m = fmax3(m, fmax3(v[i][9], v[i][10], v[i][11]), fmax3(v[i][12], v[i][13], v[i][14]));
+        m = fmaxf(m, v[i][15]);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        tmax[i] = m;
+        move |= m * sl2 > mr[i] * sl2 + kMoveRef;  // true on the first step with a valid column
+      }
+      // P(t) may overwrite the P buffer (and O may be rescaled) once P*V of step t-1 completed
+      if (!(ok = mbar_wait(&bars->p_empty, (t & 1) ^ 1, abort, lim))) break;
+      if (__any_sync(0xffffffffu, move)) {  // rare after the first step: move references
+        float f[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float mn = tmax[i] * sl2 > mr[i] * sl2 + kMoveRef ? tmax[i] : mr[i];
+          f[i] = mr[i] == -INFINITY ? 0.f : exp2_approx((mr[i] - mn) * sl2);
+          l[i] *= f[i];
+          mr[i] = mn;
+        }
+        if (t > 0) {  // O rows of this warp (lane = row) times the factor of their row
+          const int src = 4 * (lane & 7);  // a thread of the quad that holds row `lane`
+          const float f0 = __shfl_sync(0xffffffffu, f[0], src);
+          const float f1 = __shfl_sync(0xffffffffu, f[1], src);
+          const float f2 = __shfl_sync(0xffffffffu, f[2], src);
+          const float f3 = __shfl_sync(0xffffffffu, f[3], src);
+          const int which = lane >> 3;
+          const float fr = which == 0 ? f0 : which == 1 ? f1 : which == 2 ? f2 : f3;
+          tc_fence_after();
+#pragma unroll 1
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t o[16];
+            tmem_ld32x16(tl0 + kColO + 16 * q4, o);
+            tmem_wait_ld_n<16>(o);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * fr);
+            tmem_st32x16(tl0 + kColO + 16 * q4, o);
+            tmem_wait_st_keep16(o);
+          }
+        }
+      }
+      // P = exp2(v * sl2 - ref * sl2), its row sums, and bf16 P for the tensor cores, one half of
+      // the columns at a time. 16x128b store layout: repetition rep covers TMEM columns
+      // 4rep..4rep+3 (keys 8rep.. of the half), lane tr -> register 2rep, lane tr+8 -> 2rep+1;
+      // value columns (hh*8 + 2rep, +1) are exactly keys 32hh + 8rep + 2tq + {0,1}.
+      float off[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) off[i] = mr[i] == -INFINITY ? 0.f : -mr[i] * sl2;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t a0[8], a1[8];
+#pragma unroll
+        for (int rep = 0; rep < 4; ++rep) {
+          const int c = hh * 8 + 2 * rep;
+          float e[4][2];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 x = __ffma2_rn(make_float2(v[i][c], v[i][c + 1]), make_float2(sl2, sl2),
+                                        make_float2(off[i], off[i]));
+            e[i][0] = exp2_approx(x.x);
+            e[i][1] = exp2_approx(x.y);
+            l[i] += e[i][0] + e[i][1];
+          }
+          a0[2 * rep] = pack_bf16(e[0][0], e[0][1]);
+          a0[2 * rep + 1] = pack_bf16(e[1][0], e[1][1]);
+          a1[2 * rep] = pack_bf16(e[2][0], e[2][1]);
+          a1[2 * rep + 1] = pack_bf16(e[3][0], e[3][1]);
+        }
+        // keys 64*qb + 32*hh .. : TMEM columns 32*qb + 16*hh of the P region
+        tmem_st16x128_x4(tl0 + kColP + qb * 32 + hh * 16, a0);
+        tmem_st16x128_x4(tl16 + kColP + qb * 32 + hh * 16, a1);
+        tmem_wait_st_keep8(a0);
+        tmem_wait_st_keep8(a1);
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->p_full);
+    }
+
+    // finish: O / l per row (lane = row for the 32x32b loads), then write O_sel or the combine
+    if (ok && (ok = mbar_wait(&bars->o_full, 0, abort, lim))) {
+      float lsum[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float s = l[i];
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        lsum[i] = s;
+      }
+      const int src = 4 * (lane & 7);
+      const float s0 = __shfl_sync(0xffffffffu, lsum[0], src);
+      const float s1 = __shfl_sync(0xffffffffu, lsum[1], src);
+      const float s2 = __shfl_sync(0xffffffffu, lsum[2], src);
+      const float s3 = __shfl_sync(0xffffffffu, lsum[3], src);
+      const int which = lane >> 3;
+      const float rs = which == 0 ? s0 : which == 1 ? s1 : which == 2 ? s2 : s3;
+      const float inv = rs > 0.f ? 1.f / rs : 0.f;
+      tc_fence_after();
+      uint32_t o[2][32];
+      tmem_ld32(tl0 + kColO, o[0]);
+      tmem_ld32(tl0 + kColO + 32, o[1]);
+      tmem_wait_ld_regs(o[0]);
+      tmem_wait_ld_regs(o[1]);
+      const int64_t row = q0 + g * 32 + lane;
+      if (row < a.L) {
+        const int64_t at = (row * a.H + h) * 64;
+        if (a.o_sel) {
+          float4* dst = reinterpret_cast<float4*>(a.o_sel + at);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            dst[j] = make_float4(__uint_as_float(o[j >> 3][(4 * j) & 31]) * inv,
+                                 __uint_as_float(o[j >> 3][(4 * j + 1) & 31]) * inv,
+                                 __uint_as_float(o[j >> 3][(4 * j + 2) & 31]) * inv,
+                                 __uint_as_float(o[j >> 3][(4 * j + 3) & 31]) * inv);
+        } else {
+          const float2 gl = *reinterpret_cast<const float2*>(a.gates + (row * a.H + h) * 2);
+          const float gc = 1.f / (1.f + expf(-gl.x));
+          const float gs = 1.f / (1.f + expf(-gl.y));
+          const float4* oc = reinterpret_cast<const float4*>(a.o_cmp + at);
+          uint4* dst = reinterpret_cast<uint4*>(a.out + at);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 c0 = oc[2 * j], c1 = oc[2 * j + 1];
+            const uint32_t* os = &o[j >> 2][(8 * j) & 31];
+            uint4 w;
+            w.x = pack_bf16(gc * c0.x + gs * (__uint_as_float(os[0]) * inv),
+                            gc * c0.y + gs * (__uint_as_float(os[1]) * inv));
+            w.y = pack_bf16(gc * c0.z + gs * (__uint_as_float(os[2]) * inv),
+                            gc * c0.w + gs * (__uint_as_float(os[3]) * inv));
+            w.z = pack_bf16(gc * c1.x + gs * (__uint_as_float(os[4]) * inv),
+                            gc * c1.y + gs * (__uint_as_float(os[5]) * inv));
+            w.w = pack_bf16(gc * c1.z + gs * (__uint_as_float(os[6]) * inv),
+                            gc * c1.w + gs * (__uint_as_float(os[7]) * inv));
+            dst[j] = w;
+          }
+        }
+      }
+    }
+    if (!ok) raise_abort(abort, a.status);
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tbase, kTmemCols);
+}
+
+}  // namespace
+
+cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, const int32_t* idx, float* o_sel,
+                            const float* o_cmp, const float* gates, uint16_t* out,
+                            cudaStream_t st) {
+  const int box = p.b < kStep ? p.b : kStep;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_head_rows(&tq, q, p.L, p.H, kBM) || !make_tmap_head_rows(&tk, k, p.L, p.H, box) ||
+      !make_tmap_head_rows(&tv, v, p.L, p.H, box))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(sel_attn_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  // two CTAs of about 85 KB each: ask for the largest shared-memory carveout
+  e = cudaFuncSetAttribute(sel_attn_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  const int64_t ntok = static_cast<int64_t>(p.k) * p.b;
+  const int lb = p.b == 32 ? 5 : p.b == 64 ? 6 : 7;
+  SelArgs a{idx, o_sel, o_cmp, gates, out, p.L, p.nb, p.nqb, p.L / p.b, p.H, p.b, lb, p.k,
+            static_cast<int>((ntok + kStep - 1) / kStep), p.scale_log2, p.flags, p.status,
+            (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull};
+  dim3 grid(static_cast<unsigned>((p.L + kBM - 1) / kBM), p.H);
+  sel_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace s3r
