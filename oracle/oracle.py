@@ -38,6 +38,7 @@ class _Params(ctypes.Structure):
         ("scale", ctypes.c_double),
         ("exact_pool", ctypes.c_int32),
         ("threads", ctypes.c_int32),
+        ("forced", ctypes.c_int32),
     ]
 
 
@@ -58,7 +59,7 @@ def lib():
         for name, args in {
             "s3r_ref_pool": [p, p, p],
             "s3r_ref_cmp": [p, p, p, p, p, ctypes.c_int64, p, p, p],
-            "s3r_ref_topk": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, p, p, p],
+            "s3r_ref_topk": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, p, p, p],
             "s3r_ref_sel": [p, p, p, p, p, ctypes.c_int64, p, p],
             "s3r_ref_combine": [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, p, p, p, p],
         }.items():
@@ -80,6 +81,7 @@ class Problem:
     topk: int
     qblock: int = 64
     scale: Optional[float] = None  # None -> 1/sqrt(d)
+    forced: int = 0  # leading key blocks kept in every selection list (VGGT reference frame)
 
     @property
     def nb(self) -> int:
@@ -88,6 +90,11 @@ class Problem:
     @property
     def nqb(self) -> int:
         return -(-self.L // self.qblock)
+
+    @property
+    def nsel(self) -> int:
+        """Length of a selection list: the forced blocks, then the top-k."""
+        return self.forced + self.topk
 
     @property
     def softmax_scale(self) -> float:
@@ -103,7 +110,7 @@ class Problem:
 
 def _params(pb: Problem, exact_pool: bool = False, threads: int = 0) -> _Params:
     return _Params(pb.L, pb.H, pb.d, pb.block, pb.qblock, pb.topk, pb.softmax_scale,
-                   1 if exact_pool else 0, threads)
+                   1 if exact_pool else 0, threads, pb.forced)
 
 
 def _ptr(a: np.ndarray) -> ctypes.c_void_p:
@@ -162,21 +169,24 @@ def cmp_attn(pb: Problem, q_bits, kc, vc, qblocks=None, threads: int = 0):
     return lse, o, sc
 
 
-def topk(scores: np.ndarray, k: int):
-    """Top-k along the last axis: (idx int32 [..., k], gap [...]); ties -> lower index first."""
+def topk(scores: np.ndarray, k: int, forced: int = 0):
+    """Selection lists along the last axis: (idx int32 [..., forced + k], gap [...]).
+
+    The lists open with blocks 0 .. forced-1; the top-k (ties -> lower index first) ranks only the
+    other blocks, and gap is the k-th minus the (k+1)-th of those."""
     s = np.ascontiguousarray(scores, dtype=np.float64)
     lead = s.shape[:-1]
     n = s.shape[-1]
     rows = int(np.prod(lead)) if lead else 1
-    idx = np.empty(lead + (k,), np.int32)
+    idx = np.empty(lead + (forced + k,), np.int32)
     gap = np.empty(lead, np.float64)
-    rc = lib().s3r_ref_topk(rows, n, k, _ptr(s), _ptr(idx), _ptr(gap))
+    rc = lib().s3r_ref_topk(rows, n, k, forced, _ptr(s), _ptr(idx), _ptr(gap))
     assert rc == 0, rc
     return idx, gap
 
 
 def sel_attn(pb: Problem, q_bits, k_bits, v_bits, idx, qblocks=None, threads: int = 0):
-    """Selection branch over the chosen query blocks with the given idx [H, nq, topk]."""
+    """Selection branch over the chosen query blocks with the given idx [H, nq, forced + topk]."""
     q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
     k_bits = np.ascontiguousarray(k_bits, dtype=np.uint16)
     v_bits = np.ascontiguousarray(v_bits, dtype=np.uint16)
@@ -184,7 +194,7 @@ def sel_attn(pb: Problem, q_bits, k_bits, v_bits, idx, qblocks=None, threads: in
     qa, nq = _qb_array(qblocks)
     if qa is None:
         nq = pb.nqb
-    assert idx.shape == (pb.H, nq, pb.topk), idx.shape
+    assert idx.shape == (pb.H, nq, pb.nsel), idx.shape
     R = pb.rows_of(qblocks).size
     o = np.empty((R, pb.H, pb.d), np.float64)
     rc = lib().s3r_ref_sel(ctypes.byref(_params(pb, threads=threads)), _ptr(q_bits), _ptr(k_bits),
@@ -213,9 +223,9 @@ class Result:
     lse: np.ndarray      # [H, R]
     o_cmp: np.ndarray    # [R, H, d]
     scores: np.ndarray   # [H, nq, nb]
-    idx: np.ndarray      # [H, nq, topk] the oracle's own top-k
+    idx: np.ndarray      # [H, nq, forced + topk] the oracle's own selection lists
     gap: np.ndarray      # [H, nq]
-    idx_used: np.ndarray  # [H, nq, topk] the indices the selection branch ran on
+    idx_used: np.ndarray  # [H, nq, forced + topk] the indices the selection branch ran on
     o_sel: np.ndarray    # [R, H, d]
     out: np.ndarray      # [R, H, d]
 
@@ -234,7 +244,7 @@ def sparse_attn(pb: Problem, q_bits, k_bits, v_bits, gates, qblocks=None, idx_gi
     else:
         kc, vc = pooled
     lse, o_cmp, scores = cmp_attn(pb, q_bits, kc, vc, qblocks, threads)
-    idx, gap = topk(scores, pb.topk)
+    idx, gap = topk(scores, pb.topk, pb.forced)
     use = idx if idx_given is None else np.ascontiguousarray(idx_given, np.int32)
     o_sel = sel_attn(pb, q_bits, k_bits, v_bits, use, qblocks, threads)
     rows = pb.rows_of(qblocks)

@@ -27,7 +27,10 @@
  *   s3r_ref_pool        closed forms (constant blocks, linear ramps, ragged tail).
  *   s3r_ref_cmp         uniform-key closed form, a hand-derived worked example (tests/golden),
  *                       row-probability sums, library attention (torch SDPA, fp64).
- *   s3r_ref_topk        brute force over every k-subset; torch.topk on tie-free rows.
+ *   s3r_ref_topk        brute force over every k-subset; torch.topk on tie-free rows; with forced
+ *                       blocks, brute force over the subsets of the other blocks, and the forced
+ *                       blocks' own scores have no effect.
+ *   s3r_ref_sel         with forced blocks, dense attention when F + k = nb.
  *   s3r_ref_sel         dense attention (torch SDPA, fp64) when k = nb; brute force per query.
  *   s3r_ref_combine     gate limits and the zero-logit midpoint.
  *   whole pipeline      composition of the pinned steps plus permutation invariances.
@@ -296,6 +299,7 @@ static int scored_cmp(const void* a, const void* b) {
 typedef struct {
   int64_t n;
   int32_t k;
+  int32_t forced;
   const double* scores;
   int32_t* idx;
   double* gap;
@@ -303,21 +307,26 @@ typedef struct {
 
 static void topk_task(void* vctx, int64_t r) {
   const topk_ctx* c = (const topk_ctx*)vctx;
-  scored* a = (scored*)malloc(sizeof(scored) * (size_t)c->n);
-  for (int64_t j = 0; j < c->n; ++j) {
-    a[j].score = c->scores[r * c->n + j];
-    a[j].index = j;
+  int32_t* out = c->idx + r * ((int64_t)c->forced + c->k);
+  /* the always-kept blocks open the list, in ascending order */
+  for (int32_t f = 0; f < c->forced; ++f) out[f] = f;
+  /* the other blocks compete on their scores */
+  const int64_t m = c->n - c->forced;
+  scored* a = (scored*)malloc(sizeof(scored) * (size_t)m);
+  for (int64_t j = 0; j < m; ++j) {
+    a[j].score = c->scores[r * c->n + c->forced + j];
+    a[j].index = c->forced + j;
   }
-  qsort(a, (size_t)c->n, sizeof(scored), scored_cmp);
-  for (int32_t t = 0; t < c->k; ++t) c->idx[r * c->k + t] = (int32_t)a[t].index;
-  if (c->gap) c->gap[r] = c->k < c->n ? a[c->k - 1].score - a[c->k].score : INFINITY;
+  qsort(a, (size_t)m, sizeof(scored), scored_cmp);
+  for (int32_t t = 0; t < c->k; ++t) out[c->forced + t] = (int32_t)a[t].index;
+  if (c->gap) c->gap[r] = c->k < m ? a[c->k - 1].score - a[c->k].score : INFINITY;
   free(a);
 }
 
-int s3r_ref_topk(int64_t rows, int64_t n, int32_t k, const double* scores, int32_t* idx,
-                 double* gap) {
-  if (rows < 0 || n < 1 || k < 1 || k > n || !scores || !idx) return -1;
-  topk_ctx c = {n, k, scores, idx, gap};
+int s3r_ref_topk(int64_t rows, int64_t n, int32_t k, int32_t forced, const double* scores,
+                 int32_t* idx, double* gap) {
+  if (rows < 0 || n < 1 || forced < 0 || k < 1 || k > n - forced || !scores || !idx) return -1;
+  topk_ctx c = {n, k, forced, scores, idx, gap};
   parallel_for(rows, 0, topk_task, &c);
   return 0;
 }
@@ -344,13 +353,14 @@ static void sel_task(void* vctx, int64_t task) {
   const int64_t nb = ceil_div(p->L, p->block);
   const int64_t H = p->H, d = p->d, HD = H * d;
   const int64_t h = task / rm->nq, i = task % rm->nq;
-  const int32_t* sel = c->idx + (h * rm->nq + i) * p->topk;
+  const int32_t n_list = p->forced + p->topk; /* always-kept blocks, then the top-k */
+  const int32_t* sel = c->idx + (h * rm->nq + i) * n_list;
 
   /* the token set T: every token of every selected block, each block once, tokens < L */
   char* chosen = (char*)calloc((size_t)nb, 1);
-  int64_t* tokens = (int64_t*)malloc(sizeof(int64_t) * (size_t)p->topk * (size_t)p->block);
+  int64_t* tokens = (int64_t*)malloc(sizeof(int64_t) * (size_t)n_list * (size_t)p->block);
   int64_t nt = 0;
-  for (int32_t s = 0; s < p->topk; ++s) {
+  for (int32_t s = 0; s < n_list; ++s) {
     int64_t j = sel[s];
     if (j < 0 || j >= nb) {
       c->bad_index = 1;
@@ -390,7 +400,8 @@ static void sel_task(void* vctx, int64_t task) {
 
 int s3r_ref_sel(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                 const int64_t* qblocks, int64_t nq, const int32_t* idx, double* o_sel) {
-  if (check_params(p) || !q || !k || !v || !idx || !o_sel || p->topk < 1) return -1;
+  if (check_params(p) || !q || !k || !v || !idx || !o_sel || p->topk < 1 || p->forced < 0)
+    return -1;
   row_map rm;
   int rc = row_map_make(p, qblocks, nq, &rm);
   if (rc) return rc;

@@ -19,7 +19,7 @@
  *   lse          [H, R]      double          R = rows of the chosen query blocks (see below)
  *   o_cmp, o_sel [R, H, d]   double
  *   scores       [H, nq, nb] double          nq = number of chosen query blocks
- *   idx          [H, nq, k]  int32
+ *   idx          [H, nq, F + k] int32   F = forced blocks (0 unless the reference-frame variant)
  * A call may restrict the query side to a list of query-block indices ("sampled mode"); its row
  * outputs are then the rows of those blocks, concatenated in list order. A NULL list means every
  * query block 0 .. ceil(L / qblock) - 1.
@@ -46,6 +46,9 @@ typedef struct {
   int32_t exact_pool; /* 0: pooled K/V are rounded to bf16 (RNE) like a tensor-core operand;
                          1: keep the exact fp64 mean (used by the closed-form checks) */
   int32_t threads;  /* worker threads, 0 = all online cores */
+  int32_t forced;   /* F: key blocks 0 .. F-1 open every selection list (the VGGT variant keeps the
+                       reference frame's tokens for every query); the top-k then picks k more
+                       among blocks F .. nb-1, so a list holds F + k blocks. 0 = plain top-k. */
 } s3r_ref_params;
 
 /* Number of cores the oracle uses when params.threads == 0. */
@@ -64,14 +67,18 @@ int s3r_ref_pool(const s3r_ref_params* p, const uint16_t* x, double* out);
 int s3r_ref_cmp(const s3r_ref_params* p, const uint16_t* q, const double* kc, const double* vc,
                 const int64_t* qblocks, int64_t nq, double* lse, double* o_cmp, double* scores);
 
-/* Per-row top-k of a [rows, n] score matrix: the k largest, in descending score order, equal
- * scores by lower index. gap[r] = k-th largest minus (k+1)-th largest (+inf when k == n).
- * gap may be NULL. */
-int s3r_ref_topk(int64_t rows, int64_t n, int32_t k, const double* scores, int32_t* idx,
-                 double* gap);
+/* Per-row selection lists from a [rows, n] score matrix, F + k entries per row ([rows, F + k]):
+ * first the forced blocks 0 .. F-1 in ascending order, then the k largest scores among columns
+ * F .. n-1 in descending score order, equal scores by lower index. gap[r] = k-th largest minus
+ * (k+1)-th largest of those columns (+inf when k == n - F). gap may be NULL. F = 0 is the plain
+ * top-k. (Speed3R, "Methodologie" §3: for VGGT the reference-frame tokens are always kept while
+ * the rest is sparsified.) */
+int s3r_ref_topk(int64_t rows, int64_t n, int32_t k, int32_t forced, const double* scores,
+                 int32_t* idx, double* gap);
 
-/* Selection branch: exact softmax attention of each chosen query row over the tokens of the k
- * key blocks idx[h, i, :] of its query block (tokens >= L excluded). */
+/* Selection branch: exact softmax attention of each chosen query row over the tokens of the
+ * F + k key blocks idx[h, i, :] of its query block (tokens >= L excluded; a block listed twice
+ * counts once). */
 int s3r_ref_sel(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                 const int64_t* qblocks, int64_t nq, const int32_t* idx, double* o_sel);
 

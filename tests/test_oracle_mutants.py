@@ -49,6 +49,16 @@ MUTANTS = {
         "const double g_cmp = sigmoid((double)gates[(r * H + h) * 2 + 0]);",
         "const double g_cmp = sigmoid((double)gates[(r * H + h) * 2 + 1]);"),
     "round_bf16_truncates": ("double r = nearbyint(scaled);", "double r = trunc(scaled);"),
+    "topk_forced_offset_dropped": (
+        "a[j].index = c->forced + j;", "a[j].index = j;"),
+    "topk_forced_blocks_compete": (
+        "a[j].score = c->scores[r * c->n + c->forced + j];",
+        "a[j].score = c->scores[r * c->n + j];"),
+    "topk_forced_list_not_opened": (
+        "for (int32_t f = 0; f < c->forced; ++f) out[f] = f;",
+        "for (int32_t f = 0; f < c->forced; ++f) out[f] = c->forced;"),
+    "sel_list_skips_forced_blocks": (
+        "const int32_t n_list = p->forced + p->topk;", "const int32_t n_list = p->topk;"),
 }
 
 

@@ -282,6 +282,44 @@ def test_topk_matches_library_topk_without_ties():
         np.testing.assert_array_equal(idx, want)
 
 
+def test_topk_with_forced_blocks_by_brute_force():
+    """VGGT variant (reference-frame blocks always kept): the lists open with blocks 0..F-1 in
+    order, and the remaining k entries are the best k-subset of blocks F..n-1 by brute force,
+    ordered by descending score, ties by lower index; the gap is taken among those blocks."""
+    rng = np.random.default_rng(5)
+    n = 9
+    for trial in range(40):
+        row = rng.integers(0, 4, size=n).astype(np.float64)
+        for forced in range(0, 4):
+            for k in range(1, n - forced + 1):
+                rest = range(forced, n)
+                best = max(itertools.combinations(rest, k),
+                           key=lambda c: (sum(row[list(c)]), tuple(-x for x in c)))
+                idx, gap = O.topk(row[None], k, forced)
+                assert idx.shape == (1, forced + k)
+                assert idx[0, :forced].tolist() == list(range(forced))
+                assert idx[0, forced:].tolist() == sorted(best, key=lambda j: (-row[j], j))
+                srt = np.sort(row[forced:])[::-1]
+                assert gap[0] == (math.inf if k == n - forced else srt[k - 1] - srt[k])
+
+
+def test_topk_forced_blocks_scores_have_no_effect():
+    """Raising or lowering the forced blocks' own scores changes no list: they are kept without
+    competing, and they never take one of the k places."""
+    g = torch.Generator().manual_seed(9)
+    s = torch.rand(30, 50, generator=g, dtype=torch.float64).numpy()
+    for forced, k in ((1, 5), (7, 12), (20, 30)):
+        base, gap = O.topk(s, k, forced)
+        for fill in (1e9, -1e9, 0.0):
+            t = s.copy()
+            t[:, :forced] = fill
+            idx, gap2 = O.topk(t, k, forced)
+            np.testing.assert_array_equal(idx, base)
+            np.testing.assert_array_equal(gap2, gap)
+        # forced = 0 is the plain top-k
+    np.testing.assert_array_equal(O.topk(s, 5, 0)[0], O.topk(s, 5)[0])
+
+
 # --------------------------------------------------------------------------------------------
 # selection branch
 # --------------------------------------------------------------------------------------------
@@ -316,6 +354,53 @@ def test_sel_matches_library_attention_under_block_mask(L, b, k):
                 mask[64 * i:64 * i + 64, j * b:min(L, j * b + b)] = True
         want = sdpa64(qv[:, h:h + 1], kv[:, h:h + 1], vv[:, h:h + 1], pb.softmax_scale, mask[None, None])
         np.testing.assert_allclose(o[:, h:h + 1], want, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("L,b,forced", [(1000, 64, 3), (777, 32, 10), (900, 128, 1)])
+def test_sel_forced_plus_topk_covering_every_block_equals_dense_attention(L, b, forced):
+    """With F forced blocks and k = nb - F the lists cover every block: the selection branch is
+    dense attention (library SDPA in fp64), whatever order the top-k part has."""
+    H, d = 2, 64
+    pb0, q, kk, v = _setup(L, H, d, b, 1, 53, qscale=1.0)
+    nb = pb0.nb
+    pb = O.Problem(L, H, d, b, nb - forced, forced=forced)
+    rng = np.random.default_rng(forced)
+    lists = [np.concatenate([np.arange(forced), forced + rng.permutation(nb - forced)])
+             for _ in range(H * pb.nqb)]
+    idx = np.stack(lists).reshape(H, pb.nqb, nb).astype(np.int32)
+    o = O.sel_attn(pb, q, kk, v, idx)
+    want = sdpa64(values_of(q), values_of(kk), values_of(v), pb.softmax_scale)
+    np.testing.assert_allclose(o, want, rtol=0, atol=1e-13)
+
+
+def test_pipeline_with_forced_blocks_attends_to_the_reference_frame():
+    """Whole path of the VGGT variant on 4 views of 160 tokens, b = 32: the reference frame
+    (view 0, blocks 0..4) opens every list; the selection output equals masked library attention
+    over the forced tokens plus the blocks of the oracle's own top-k; the compression branch and
+    the scores are those of the plain path."""
+    P, N, H, d, b, k = 160, 4, 2, 64, 32, 3
+    L = P * N
+    forced = -(-P // b)
+    pb, q, kk, v = _setup(L, H, d, b, k, 57, qscale=0.8)
+    pbf = O.Problem(L, H, d, b, k, forced=forced)
+    gates = _gates(L, H, 58)
+    plain = O.sparse_attn(pb, q, kk, v, gates)
+    res = O.sparse_attn(pbf, q, kk, v, gates)
+    np.testing.assert_array_equal(res.scores, plain.scores)
+    np.testing.assert_array_equal(res.o_cmp, plain.o_cmp)
+    assert res.idx.shape == (H, pbf.nqb, forced + k)
+    assert (res.idx[..., :forced] == np.arange(forced)).all()
+    assert (res.idx[..., forced:] >= forced).all()
+    qv, kv, vv = values_of(q), values_of(kk), values_of(v)
+    for h in range(H):
+        mask = np.zeros((L, L), bool)
+        for i in range(pbf.nqb):
+            for j in res.idx[h, i]:
+                mask[64 * i:64 * i + 64, j * b:min(L, j * b + b)] = True
+        assert mask[:, :P].all()
+        want = sdpa64(qv[:, h:h + 1], kv[:, h:h + 1], vv[:, h:h + 1], pbf.softmax_scale,
+                      mask[None, None])
+        np.testing.assert_allclose(res.o_sel[:, h:h + 1], want, rtol=0, atol=1e-13)
 
 
 def test_sel_block_order_and_duplicates_do_not_matter():
