@@ -62,6 +62,40 @@ def load_peaks():
     return p
 
 
+# MUFU.EX2 issue rate of one SM per clock (4 sub-partitions x 4 lanes; 15.8 measured with a
+# dependent-free ex2.approx loop over all 148 SMs at 1965 MHz) and the SM count of a B200.
+EX2_PER_CLK_SM = 16
+SM_COUNT = 148
+
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the kernel that bounds
+# the step, from one ncu capture of the default workload (python bench.py --steps 2 --warmup 3
+# --no-cpu-baseline), with the SHA-256 of the sources that kernel was built from: once any of them
+# changes, the figure no longer describes the kernel and the roofline reports null.
+TRAFFIC = {}
+
+
+def _sources_sha(paths):
+    import hashlib
+
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(stage: str, workload: str):
+    rec = TRAFFIC.get(stage)
+    if not rec or rec["workload"] != workload:
+        return None
+    try:
+        if _sources_sha(rec["sources"]) != rec["sha256"]:
+            return None
+    except OSError:
+        return None
+    return rec["bytes"]
+
+
 def algorithmic(cfg):
     """Algorithmic work per call: FLOPs of Q.Kc^T + P.Vc (once) and of the selection's
     Q.K^T + P.V over the tokens actually selected; bytes of each stage's compulsory traffic."""
@@ -72,6 +106,7 @@ def algorithmic(cfg):
     cmp_flops = 4.0 * L * nb * d * H
     sel_flops = 4.0 * L * sel_tokens * d * H
     return {
+        "cmp_exp2": 2.0 * L * nb * H,  # one per (query, summary) pair in each of the two passes
         "cmp_flops": cmp_flops,
         "sel_flops": sel_flops,
         "flops": cmp_flops + sel_flops,
@@ -343,9 +378,18 @@ def run_native(args, wl):
         roof = {"bound": "tensor", "achieved": units / dom_s / 1e12,
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = measured_traffic(dom, args.workload)
     roof["kernel"] = dom
     roof["peak_source"] = peaks["source"] + (" sustained bf16" if bound == "tensor" else " copy")
+    if dom == "cmp":
+        # the compressed branch needs two exponentials per (query, summary) pair; their unit,
+        # not the tensor pipe, is the tighter bound
+        ex2_peak = EX2_PER_CLK_SM * SM_COUNT * peaks.get("sm_max_mhz", 1965.0) * 1e6
+        ach = work["cmp_exp2"] / dom_s
+        roof["co_bound"] = {"bound": "alu", "what": "exp2 on the MUFU pipe",
+                            "achieved": ach / 1e12, "peak": ex2_peak / 1e12, "unit": "Texp2/s",
+                            "frac": ach / ex2_peak,
+                            "peak_source": "16 ex2 per clock per SM x 148 SMs x max SM clock"}
     stages = {}
     for n in _lib.STAGES:
         b_, u_ = work["stage_work"][n]

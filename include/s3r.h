@@ -23,8 +23,10 @@
  *   P[q,j]               = exp(s[q,j] - lse[h,q])                      (fp32)
  *   O_cmp[q,h,:]         = sum_j P[q,j] * Vc[j,h,:]
  *   scores[h,i,j]        = sum over the valid rows q of query block i of P[q,j]
- *   idx[h,i,:]           = the topk block indices with the largest scores[h,i,:], ties broken
- *                          toward the lower index
+ *   idx[h,i,:]           = the selection list of query block i, F + topk entries: the forced
+ *                          blocks 0 .. F-1 (F = params.forced, usually 0), then the topk block
+ *                          indices j >= F with the largest scores[h,i,j], ties broken toward the
+ *                          lower index
  *   O_sel[q,h,:]         = softmax-weighted sum of V[t,h,:] over the tokens t < L of the
  *                          blocks idx[h,i,:] of q's query block, weights softmax_t(scale*<Q,K[t]>)
  *   out[q,h,:]           = sigmoid(g[q,h,0]) * O_cmp[q,h,:] + sigmoid(g[q,h,1]) * O_sel[q,h,:]
@@ -85,6 +87,10 @@ typedef struct {
   int32_t topk;   /* k, blocks selected per query block, 1 <= k <= nb (k = nb: dense selection) */
   float scale;    /* softmax scale; <= 0 selects 1/sqrt(d) */
   uint32_t flags; /* S3R_FLAG_* */
+  int32_t forced; /* F >= 0: key blocks 0 .. F-1 open every selection list without competing,
+                     and topk more are chosen among blocks F .. nb-1 (topk <= nb - F). The VGGT
+                     variant keeps the reference frame's tokens for every query ("Methodologie"
+                     §3): with P tokens per view, F = ceil(P / b). 0 = plain top-k. */
   uint32_t* dev_status; /* optional device word that receives S3R_DEV_* bits (may be NULL) */
   void* const* stage_events; /* optional: S3R_NUM_STAGES + 1 cudaEvent_t handles that
                                 s3r_sparse_attn_fwd records on `stream` at the stage boundaries
@@ -143,16 +149,17 @@ s3r_status s3r_cmp_attn_and_score(const s3r_params* params, const s3r_bf16* q,
 
 /* Per-query-block top-k ("Selectie-tak": "Top-k selectie").
  *   scores [H, nqb, nb] fp32 (read), non-negative, not NaN
- *   idx    [H, nqb, topk] int32 (written). The set is exact: score bits compared as unsigned
- *          integers, equal scores broken toward the lower block index. For topk <= 2048 the
- *          entries are ordered by descending score, ties by ascending index; for larger topk
- *          they are in ascending index order. */
+ *   idx    [H, nqb, forced + topk] int32 (written): blocks 0 .. forced-1, then the top-k of
+ *          blocks forced .. nb-1. The set is exact: score bits compared as unsigned integers,
+ *          equal scores broken toward the lower block index. For topk <= 2048 the top-k entries
+ *          are ordered by descending score, ties by ascending index; for larger topk they are in
+ *          ascending index order. */
 s3r_status s3r_topk_blocks(const s3r_params* params, const float* scores, int32_t* idx,
                            s3r_stream stream);
 
 /* Selection branch ("Selectie-tak": fine attention on the selected tokens).
- *   q, k, v [L, H, d] bf16 (read); idx [H, nqb, topk] int32 (read): distinct block indices in
- *           [0, nb) per row (entries outside that range are skipped; with
+ *   q, k, v [L, H, d] bf16 (read); idx [H, nqb, forced + topk] int32 (read): distinct block
+ *           indices in [0, nb) per row (entries outside that range are skipped; with
  *           S3R_FLAG_DEBUG_CHECKS they also raise S3R_DEV_BAD_INDEX)
  *   o_sel   [L, H, d] fp32 (written) */
 s3r_status s3r_sel_attn(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,
@@ -172,7 +179,7 @@ s3r_status s3r_gate_combine(const s3r_params* params, const float* o_cmp, const 
  * s3r_topk_blocks' kernel (4 launches). Both select the same blocks.
  *   q, k, v     [L, H, d] bf16; gate_logits [L, H, 2] fp32 (read)
  *   out         [L, H, d] bf16 (written)
- *   idx_out     [H, nqb, topk] int32 (written if not NULL)
+ *   idx_out     [H, nqb, forced + topk] int32 (written if not NULL)
  *   workspace   device buffer of at least s3r_workspace_bytes(params) bytes, 256-byte aligned;
  *               its contents on entry do not matter. */
 s3r_status s3r_sparse_attn_fwd(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,

@@ -57,6 +57,7 @@ class Params(ctypes.Structure):
         ("topk", ctypes.c_int32),
         ("scale", ctypes.c_float),
         ("flags", ctypes.c_uint32),
+        ("forced", ctypes.c_int32),
         ("dev_status", ctypes.c_void_p),
         ("stage_events", ctypes.c_void_p),
     ]

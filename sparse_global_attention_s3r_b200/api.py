@@ -24,7 +24,10 @@ QBLOCK = 64
 
 @dataclass(frozen=True)
 class Config:
-    """Sizes of one call: L tokens (N views x P tokens), H heads, d, block size b, top-k."""
+    """Sizes of one call: L tokens (N views x P tokens), H heads, d, block size b, top-k.
+
+    forced: leading key blocks kept in every selection list (VGGT's reference frame: with P
+    tokens per view, ceil(P / b)); the top-k then picks topk more among the other blocks."""
 
     L: int
     H: int
@@ -34,6 +37,12 @@ class Config:
     scale: Optional[float] = None  # None -> 1/sqrt(d)
     debug_checks: bool = False
     test_timeout: bool = False  # testing only: exercise the bounded-wait timeout path
+    forced: int = 0
+
+    @property
+    def nsel(self) -> int:
+        """Selection list length: forced blocks, then the top-k."""
+        return self.forced + self.topk
 
     @property
     def nb(self) -> int:
@@ -48,6 +57,7 @@ class Config:
                            0.0 if self.scale is None else float(self.scale),
                            (_lib.S3R_FLAG_DEBUG_CHECKS if self.debug_checks else 0)
                            | (_lib.S3R_FLAG_TEST_TIMEOUT if self.test_timeout else 0),
+                           self.forced,
                            None if dev_status is None else dev_status.data_ptr(),
                            None if stage_events is None else ctypes.addressof(stage_events))
 
@@ -101,7 +111,7 @@ def cmp_attn_and_score(cfg: Config, q: torch.Tensor, kc: torch.Tensor, vc: torch
 def topk_blocks(cfg: Config, scores: torch.Tensor,
                 dev_status: Optional[torch.Tensor] = None) -> torch.Tensor:
     _need(scores, "scores", (cfg.H, cfg.nqb, cfg.nb), torch.float32)
-    idx = torch.empty((cfg.H, cfg.nqb, cfg.topk), dtype=torch.int32, device=scores.device)
+    idx = torch.empty((cfg.H, cfg.nqb, cfg.nsel), dtype=torch.int32, device=scores.device)
     p = cfg.params(dev_status)
     _lib.call("s3r_topk_blocks", ctypes.byref(p), _ptr(scores), _ptr(idx), _stream())
     return idx
@@ -111,7 +121,7 @@ def sel_attn(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx
              dev_status: Optional[torch.Tensor] = None) -> torch.Tensor:
     for n, t in (("q", q), ("k", k), ("v", v)):
         _need(t, n, _lhd(cfg), torch.bfloat16)
-    _need(idx, "idx", (cfg.H, cfg.nqb, cfg.topk), torch.int32)
+    _need(idx, "idx", (cfg.H, cfg.nqb, cfg.nsel), torch.int32)
     o = torch.empty(_lhd(cfg), dtype=torch.float32, device=q.device)
     p = cfg.params(dev_status)
     _lib.call("s3r_sel_attn", ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o),
@@ -176,7 +186,7 @@ def sparse_attn_fwd(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tens
         out = torch.empty(_lhd(cfg), dtype=torch.bfloat16, device=q.device)
     _need(out, "out", _lhd(cfg), torch.bfloat16)
     if idx_out is not None:
-        _need(idx_out, "idx_out", (cfg.H, cfg.nqb, cfg.topk), torch.int32)
+        _need(idx_out, "idx_out", (cfg.H, cfg.nqb, cfg.nsel), torch.int32)
     p = cfg.params(dev_status, None if stage_events is None else stage_events.handles)
     _lib.call("s3r_sparse_attn_fwd", ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(gates),
               _ptr(out), _ptr(idx_out), _ptr(workspace), workspace.numel(), _stream())
@@ -195,7 +205,7 @@ def sparse_attn_fwd_static(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: tor
         out = torch.empty(_lhd(cfg), dtype=torch.bfloat16, device=q.device)
     _need(out, "out", _lhd(cfg), torch.bfloat16)
     if idx_out is not None:
-        _need(idx_out, "idx_out", (cfg.H, cfg.nqb, cfg.topk), torch.int32)
+        _need(idx_out, "idx_out", (cfg.H, cfg.nqb, cfg.nsel), torch.int32)
     p = cfg.params()
     _lib.call("s3r_sparse_attn_fwd_static", ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
               _ptr(gates), _ptr(out), _ptr(idx_out), _stream())
@@ -223,7 +233,7 @@ class SparseAttention:
         self.device = torch.device(device or "cuda")
         self.workspace = alloc_workspace(cfg, self.device)
         self.out = torch.empty(_lhd(cfg), dtype=torch.bfloat16, device=self.device)
-        self.idx = torch.empty((cfg.H, cfg.nqb, cfg.topk), dtype=torch.int32, device=self.device)
+        self.idx = torch.empty((cfg.H, cfg.nqb, cfg.nsel), dtype=torch.int32, device=self.device)
         self._dev_in = None
 
     def __call__(self, q, k, v, gates) -> torch.Tensor:

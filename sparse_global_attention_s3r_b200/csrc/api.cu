@@ -32,10 +32,12 @@ s3r_status derive(const s3r_params* prm, Problem* out) {
   p.b = prm->block;
   p.qb = prm->qblock;
   p.k = prm->topk;
+  p.F = prm->forced;
+  p.nsel = p.F + p.k;
   p.nb = (p.L + p.b - 1) / p.b;
   p.nqb = (p.L + p.qb - 1) / p.qb;
   if (p.nb > S3R_MAX_BLOCKS) return S3R_ERR_UNSUPPORTED;
-  if (p.k > p.nb) return S3R_ERR_INVALID_ARG;
+  if (p.F < 0 || p.k > p.nb - p.F) return S3R_ERR_INVALID_ARG;
   p.scale = prm->scale > 0.f ? prm->scale : 1.0f / std::sqrt(static_cast<float>(p.d));
   p.scale_log2 = static_cast<float>(static_cast<double>(p.scale) * 1.4426950408889634);
   p.flags = prm->flags;
@@ -72,7 +74,7 @@ Workspace layout(const Problem& p) {
   w.vc = take(static_cast<size_t>(p.nb) * HD * 2);
   w.o_cmp = take(static_cast<size_t>(p.L) * HD * 4);
   w.scores = take(p.k > kFusedTopkMax ? static_cast<size_t>(p.H) * p.nqb * p.nb * 4 : 0);
-  w.idx = take(static_cast<size_t>(p.H) * p.nqb * p.k * 4);
+  w.idx = take(static_cast<size_t>(p.H) * p.nqb * p.nsel * 4);
   w.total = off;
   return w;
 }

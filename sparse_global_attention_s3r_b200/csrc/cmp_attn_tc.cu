@@ -13,7 +13,7 @@
 // Q is placed in TMEM once, so both products read their A operand from TMEM and shared memory
 // only serves the Kc/Vc tiles (a 128x64x16 MMA with A in shared memory would re-read 4 KB of Q
 // per instruction and be limited by shared-memory bandwidth).
-// Roles (352 threads, 11 warps):
+// Roles (384 threads, 12 warps):
 //   warp 0      TMA producer: Kc (pass A) or Kc+Vc (pass B) 64-key tiles into a ring of
 //               128-byte-swizzled shared-memory tiles
 //   warp 1      TMEM owner (256 columns) and the single-thread tcgen05.mma issuer
@@ -21,11 +21,12 @@
 //               (w-2)/4 (32 of the tile's 64 columns). With the 16x256b load shape a thread
 //               holds 4 rows x 8 columns, so a column sum is 3 in-thread adds plus 3 shuffle
 //               levels; P goes back with the matching 16x128b store shape.
-//   warp 10     adds the two row-quadrant partial column sums of each query block; writes the
-//               scores and/or keeps each query block's running top-k (k <= 32) in registers:
-//               lane i holds the i-th largest key (score bits << 32 | ~block index), a tile's
-//               candidates are tested against the k-th key with one ballot and the rare winners
-//               are inserted by a warp-wide ordered shift, so the score matrix never exists
+//   warps 10-11 one per query block of the tile: add the two row-quadrant partial column sums;
+//               write the scores and/or keep the query block's running top-k (k <= 32) in
+//               registers: lane i holds the i-th largest key (score bits << 32 | ~block index),
+//               a tile's candidates are tested against the k-th key with one ballot and the
+//               winners are inserted by a warp-wide ordered shift, so the score matrix never
+//               exists; blocks below `forced` never compete
 // TMEM columns: S[2] (64 fp32 each) | O (64 fp32) | Q (64 bf16 = 32) | P (64 bf16 = 32).
 // Every wait is an mbarrier wait bounded in time that also watches a CTA abort flag; on expiry
 // the kernel records S3R_DEV_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
@@ -44,14 +45,14 @@ constexpr int kBM = 128;       // query rows per CTA (TMEM lanes)
 constexpr int kBN = 64;        // block summaries per tile
 constexpr int kStages = 5;     // shared-memory ring depth
 constexpr int kSoftmaxWarps = 8;
-constexpr int kThreads = (3 + kSoftmaxWarps) * 32;  // producer, MMA, softmax x8, scores
+constexpr int kThreads = (4 + kSoftmaxWarps) * 32;  // producer, MMA, softmax x8, scores x2
 constexpr int kScoreWarp = 2 + kSoftmaxWarps;
 constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
 constexpr uint32_t kKVBytes = kBN * 128;  // 8 KB
 constexpr uint32_t kColS = 0, kColO = 128, kColQ = 192, kColP = 224, kTmemCols = 256;
 constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0, 0);  // A=Q (TMEM), B=Kc K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, 64, 0, 1);   // A=P (TMEM), B=Vc MN-major
-constexpr int kRed = 4;  // depth of the ring of per-tile partial column sums
+constexpr int kRed = 8;  // depth of the ring of per-tile partial column sums
 // pass A keeps a per-row reference max from the first tile; a row sum beyond 2^64 (or inf/nan)
 // means a later logit exceeded it by a lot, and only then is the reference moved
 constexpr float kSumLimit = 1.8446744073709552e19f;
@@ -93,8 +94,9 @@ struct CmpArgs {
   float* lse;         // [H, L] natural log, may be null
   float* o_cmp;       // [L, H, 64]
   float* scores;      // [H, nqb, nb], may be null
-  int32_t* idx;       // [H, nqb, topk] streaming top-k output (topk <= 32), may be null
+  int32_t* idx;       // [H, nqb, forced + topk] selection lists (topk <= 32), may be null
   int topk;
+  int forced;         // blocks 0 .. forced-1 open every list and do not compete
   int64_t L, nb, nqb;
   int H;
   float scale_log2;
@@ -103,21 +105,22 @@ struct CmpArgs {
   uint32_t flags;
 };
 
-// Insert this lane's candidate key c into the warp's sorted list (lane i holds the i-th largest
-// key; lanes 0..k-1 are the current top-k) if it beats the k-th key. Keys are unique.
+// Offer one candidate key c per lane to the warp's sorted list (lane i holds the i-th largest
+// key; lanes 0..k-1 are the current top-k). Keys are unique. Candidates above the k-th key are
+// inserted one at a time by an ordered shift. The threshold is not re-read between insertions:
+// a candidate that an earlier one pushed below the k-th key lands at a position >= k (or drops
+// off the end), which leaves the top-k unchanged, so each insertion costs three collectives.
 __device__ __forceinline__ void topk_offer(uint64_t& mine, uint64_t c, int k, int lane) {
-  uint64_t thr = __shfl_sync(0xffffffffu, mine, k - 1);
+  const uint64_t thr = __shfl_sync(0xffffffffu, mine, k - 1);
   unsigned pending = __ballot_sync(0xffffffffu, c > thr);
   while (pending) {
     const int src = __ffs(pending) - 1;
+    pending &= pending - 1;
     const uint64_t cand = __shfl_sync(0xffffffffu, c, src);
-    const int pos = __popc(__ballot_sync(0xffffffffu, mine > cand));  // < k since cand > thr
+    const int pos = __popc(__ballot_sync(0xffffffffu, mine > cand));
     const uint64_t up = __shfl_up_sync(0xffffffffu, mine, 1);
     if (lane > pos) mine = up;
     if (lane == pos) mine = cand;
-    thr = __shfl_sync(0xffffffffu, mine, k - 1);
-    pending &= ~(1u << src);
-    pending &= __ballot_sync(0xffffffffu, c > thr);
   }
 }
 
@@ -196,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(&bars->p_empty, 1);
     for (int r = 0; r < kRed; ++r) {
       mbar_init(&bars->red_full[r], kSoftmaxWarps);
-      mbar_init(&bars->red_empty[r], 1);
+      mbar_init(&bars->red_empty[r], 2);  // one arrival per score warp
     }
     mbar_init(&bars->stat, kSoftmaxWarps);
     mbar_init(&bars->o_full, 1);
@@ -505,7 +508,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (!ok) raise_abort(abort, a.status);
   } else {
     // ------------------------------------------------------------------ scores / top-k
-    uint64_t best[2] = {0ull, 0ull};  // below every real key
+    // one warp per query block of the tile, so the two running lists grow in parallel
+    const int qb = warp - kScoreWarp;
+    const int64_t i = qtile * 2 + qb;
+    float* dst = a.scores && i < a.nqb ? a.scores + (static_cast<int64_t>(h) * a.nqb + i) * a.nb
+                                       : nullptr;
+    uint64_t best = 0ull;  // below every real key
     bool ok = true;
     for (int t = 0; t < nt; ++t) {
       const int par = t % kRed;
@@ -514,39 +522,33 @@ __global__ void __launch_bounds__(kThreads, 2)
         ok = false;
         break;
       }
+      float sc[2];
 #pragma unroll
-      for (int qb = 0; qb < 2; ++qb) {
-        const int64_t i = qtile * 2 + qb;
-        if (i >= a.nqb) continue;
-        float* dst = a.scores ? a.scores + (static_cast<int64_t>(h) * a.nqb + i) * a.nb : nullptr;
-        uint64_t key[2];
-#pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-          const int cc = hc * 32 + lane;
-          const int64_t col = static_cast<int64_t>(t) * kBN + cc;
-          const float sc =
-              red[(par * 4 + 2 * qb) * 64 + cc] + red[(par * 4 + 2 * qb + 1) * 64 + cc];
-          if (dst && col < a.nb) dst[col] = sc;
-          key[hc] = col < a.nb ? (static_cast<uint64_t>(__float_as_uint(sc)) << 32) |
-                                     static_cast<uint32_t>(~static_cast<uint32_t>(col))
-                               : 0ull;
-        }
-        if (a.idx) {
-          topk_offer(best[qb], key[0], a.topk, lane);
-          topk_offer(best[qb], key[1], a.topk, lane);
-        }
+      for (int hc = 0; hc < 2; ++hc) {
+        const int cc = hc * 32 + lane;
+        sc[hc] = red[(par * 4 + 2 * qb) * 64 + cc] + red[(par * 4 + 2 * qb + 1) * 64 + cc];
       }
-      __syncwarp();
+      __syncwarp();  // the ring slot is read: hand it back before the (slower) list updates
       if (lane == 0) mbar_arrive(&bars->red_empty[par]);
-    }
-    if (ok && a.idx) {
+      if (i >= a.nqb) continue;
 #pragma unroll
-      for (int qb = 0; qb < 2; ++qb) {
-        const int64_t i = qtile * 2 + qb;
-        if (i < a.nqb && lane < a.topk)
-          a.idx[(static_cast<int64_t>(h) * a.nqb + i) * a.topk + lane] =
-              static_cast<int32_t>(~static_cast<uint32_t>(best[qb] & 0xFFFFFFFFull));
+      for (int hc = 0; hc < 2; ++hc) {
+        const int64_t col = static_cast<int64_t>(t) * kBN + hc * 32 + lane;
+        if (dst && col < a.nb) dst[col] = sc[hc];
+        if (a.idx) {
+          const uint64_t key = col < a.nb && col >= a.forced
+                                   ? (static_cast<uint64_t>(__float_as_uint(sc[hc])) << 32) |
+                                         static_cast<uint32_t>(~static_cast<uint32_t>(col))
+                                   : 0ull;
+          topk_offer(best, key, a.topk, lane);
+        }
       }
+    }
+    if (ok && a.idx && i < a.nqb) {
+      int32_t* list = a.idx + (static_cast<int64_t>(h) * a.nqb + i) * (a.forced + a.topk);
+      for (int f = lane; f < a.forced; f += 32) list[f] = f;
+      if (lane < a.topk)
+        list[a.forced + lane] = static_cast<int32_t>(~static_cast<uint32_t>(best & 0xFFFFFFFFull));
     }
   }
 
@@ -569,7 +571,7 @@ cudaError_t launch_cmp_attn_tc(const Problem& p, const uint16_t* q, const uint16
   cudaError_t e = cudaFuncSetAttribute(cmp_attn_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  CmpArgs a{q, lse, o_cmp, scores, idx, p.k, p.L, p.nb, p.nqb, p.H, p.scale_log2, p.status,
+  CmpArgs a{q, lse, o_cmp, scores, idx, p.k, p.F, p.L, p.nb, p.nqb, p.H, p.scale_log2, p.status,
             (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull, p.flags};
   dim3 grid(static_cast<unsigned>((p.L + kBM - 1) / kBM), p.H);
   cmp_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tk, tv, a);

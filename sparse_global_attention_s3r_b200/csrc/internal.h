@@ -12,7 +12,9 @@ namespace s3r {
 struct Problem {
   int64_t L;        // tokens
   int H, d, b, qb;  // heads, head dim (64), key-block size, query-block rows (64)
-  int k;            // top-k
+  int k;            // top-k (blocks chosen by score)
+  int F;            // leading key blocks kept in every selection list (0 = none)
+  int nsel;         // selection list length F + k
   int64_t nb, nqb;  // key blocks, query blocks
   float scale;      // softmax scale
   float scale_log2; // scale * log2(e): logits in base-2 units

@@ -63,7 +63,7 @@ constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr uint32_t kSmemBytes = (kSmemUsed + 1024 > 80 * 1024 ? kSmemUsed + 1024 : 80 * 1024);
 
 struct SelArgs {
-  const int32_t* idx;  // [H, nqb, topk]
+  const int32_t* idx;  // [H, nqb, topk] (topk here = list length: forced blocks + top-k)
   float* o_sel;        // [L, H, 64] fp32, or null for the fused combine
   const float* o_cmp;  // [L, H, 64] fp32 (fused combine)
   const float* gates;  // [L, H, 2]  fp32 (fused combine)
@@ -484,9 +484,9 @@ cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t*
   e = cudaFuncSetAttribute(sel_attn_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  const int64_t ntok = static_cast<int64_t>(p.k) * p.b;
+  const int64_t ntok = static_cast<int64_t>(p.nsel) * p.b;
   const int lb = p.b == 32 ? 5 : p.b == 64 ? 6 : 7;
-  SelArgs a{idx, o_sel, o_cmp, gates, out, p.L, p.nb, p.nqb, p.L / p.b, p.H, p.b, lb, p.k,
+  SelArgs a{idx, o_sel, o_cmp, gates, out, p.L, p.nb, p.nqb, p.L / p.b, p.H, p.b, lb, p.nsel,
             static_cast<int>((ntok + kStep - 1) / kStep), p.scale_log2, p.flags, p.status,
             (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull};
   dim3 grid(static_cast<unsigned>((p.L + kBM - 1) / kBM), p.H);

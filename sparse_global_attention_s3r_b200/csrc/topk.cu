@@ -20,6 +20,8 @@
 // of the elements equal to T the lowest indices, found by an in-order block prefix count. For
 // k <= kSortMax the winners are bitonic-sorted as above; larger k are emitted in ascending index
 // order.
+// With F forced blocks (the VGGT variant's always-kept reference frame) the list opens with
+// blocks 0 .. F-1 and the top-k runs over the rest of the row only.
 #include "common.cuh"
 #include "internal.h"
 
@@ -82,7 +84,8 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int& 
 }
 
 __global__ void __launch_bounds__(kThreads)
-    topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, int nb, int k) {
+    topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, int row_len,
+                int first, int k) {
   // dynamic shared memory: [kWarps][256] histograms (reused as the sort buffer), then [nb] keys
   extern __shared__ __align__(16) uint32_t smem_dyn[];
   int(*hist)[256] = reinterpret_cast<int(*)[256]>(smem_dyn);
@@ -93,10 +96,14 @@ __global__ void __launch_bounds__(kThreads)
   __shared__ uint32_t s_max[kThreads];
   __shared__ int s_count;
 
+  // blocks 0 .. first-1 open the list without competing; the top-k ranks the other nb of the row
+  const int nb = row_len - first;
   const int64_t row = blockIdx.x;
-  const uint32_t* src = reinterpret_cast<const uint32_t*>(scores + row * nb);
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(scores + row * row_len + first);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int32_t* out = idx + row * k;
+  int32_t* out = idx + row * (first + k);
+  for (int f = tid; f < first; f += kThreads) out[f] = f;
+  out += first;
   uint64_t* sort_buf = reinterpret_cast<uint64_t*>(smem_dyn);  // aliases the histograms
 
   uint32_t my_max = 0;
@@ -154,7 +161,7 @@ __global__ void __launch_bounds__(kThreads)
       __syncthreads();
       bitonic_sort_desc(sort_buf, n2);
       for (int e = tid; e < k; e += kThreads)
-        out[e] = static_cast<int32_t>(~static_cast<uint32_t>(sort_buf[e] & 0xFFFFFFFFull));
+        out[e] = first + static_cast<int32_t>(~static_cast<uint32_t>(sort_buf[e] & 0xFFFFFFFFull));
       return;
     }
     // too many candidates (degenerate row): fall through to the exact radix select
@@ -211,7 +218,7 @@ __global__ void __launch_bounds__(kThreads)
       if (sorted_out)
         sort_buf[pos] = (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(j));
       else
-        out[pos] = j;
+        out[pos] = first + j;
     }
     eq_base += eq_total;
     out_base += take_total;
@@ -224,7 +231,7 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
   bitonic_sort_desc(sort_buf, n2);
   for (int e = tid; e < k; e += kThreads)
-    out[e] = static_cast<int32_t>(~static_cast<uint32_t>(sort_buf[e] & 0xFFFFFFFFull));
+    out[e] = first + static_cast<int32_t>(~static_cast<uint32_t>(sort_buf[e] & 0xFFFFFFFFull));
 }
 
 }  // namespace
@@ -242,7 +249,7 @@ cudaError_t launch_topk(const Problem& p, const float* scores, int32_t* idx, cud
   if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(p.H) * p.nqb;
   topk_kernel<<<static_cast<unsigned>(rows), kThreads, smem, st>>>(scores, idx,
-                                                                   static_cast<int>(p.nb), p.k);
+                                                                   static_cast<int>(p.nb), p.F, p.k);
   count_launch();
   return cudaGetLastError();
 }

@@ -56,11 +56,17 @@ def check_close(name, gpu, ref, atol, rl2=None):
 
 
 def check_selection(gpu_idx: np.ndarray, ref_idx: np.ndarray, gap: np.ndarray,
-                    scores: np.ndarray, k: int) -> dict:
-    """Index parity of one top-k selection [H, nq, k] against the oracle.
+                    scores: np.ndarray, k: int, forced: int = 0) -> dict:
+    """Index parity of one selection [H, nq, forced + k] against the oracle.
 
-    Where the oracle's gap exceeds GAP_EXACT the sets must be equal; everywhere, every selected
-    block must be score-optimal within tau of the oracle's k-th best score."""
+    The forced blocks 0 .. forced-1 must open every list. Of the rest (the top-k among blocks
+    forced .. nb-1): where the oracle's gap exceeds GAP_EXACT the sets must be equal; everywhere,
+    every selected block must be score-optimal within tau of the oracle's k-th best score."""
+    if forced:
+        assert (gpu_idx[..., :forced] == np.arange(forced)).all(), "forced blocks missing"
+        assert (ref_idx[..., :forced] == np.arange(forced)).all()
+        gpu_idx, ref_idx = gpu_idx[..., forced:] - forced, ref_idx[..., forced:] - forced
+        scores = scores[..., forced:]
     gs = np.sort(gpu_idx, -1)
     rs = np.sort(ref_idx, -1)
     sep = gap > GAP_EXACT

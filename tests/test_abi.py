@@ -60,6 +60,8 @@ A16_NOT256 = ctypes.c_void_p((1 << 20) + 16)
     (dict(H=0), _lib.S3R_ERR_INVALID_ARG),
     (dict(topk=0), _lib.S3R_ERR_INVALID_ARG),
     (dict(topk=17), _lib.S3R_ERR_INVALID_ARG),  # nb = 16
+    (dict(topk=4, forced=13), _lib.S3R_ERR_INVALID_ARG),  # forced + topk > nb
+    (dict(forced=-1), _lib.S3R_ERR_INVALID_ARG),
     (dict(scale=float("nan")), _lib.S3R_ERR_INVALID_ARG),
     (dict(scale=float("inf")), _lib.S3R_ERR_INVALID_ARG),
     (dict(L=_lib.S3R_MAX_BLOCKS * 32 + 1, block=32, topk=1), _lib.S3R_ERR_UNSUPPORTED),
@@ -112,14 +114,15 @@ def r256(x):
     return (x + 255) // 256 * 256
 
 
-@pytest.mark.parametrize("L,H,b,k", [(1024, 2, 64, 4), (1374000, 16, 64, 32), (274800, 16, 32, 8588),
-                                     (1, 1, 128, 1)])
-def test_workspace_size_matches_layout(L, H, b, k):
-    cfg = api.Config(L=L, H=H, block=b, topk=k)
+@pytest.mark.parametrize("L,H,b,k,F", [(1024, 2, 64, 4, 0), (1374000, 16, 64, 32, 0),
+                                       (274800, 16, 32, 8588, 0), (1, 1, 128, 1, 0),
+                                       (43968, 16, 64, 16, 22), (43968, 16, 64, 40, 22)])
+def test_workspace_size_matches_layout(L, H, b, k, F):
+    cfg = api.Config(L=L, H=H, block=b, topk=k, forced=F)
     nb, nqb, d = cfg.nb, cfg.nqb, 64
     scores = H * nqb * nb * 4 if k > 32 else 0  # materialised only when k exceeds 32
     want = (r256(4) + 2 * r256(nb * H * d * 2) + r256(L * H * d * 4)
-            + r256(scores) + r256(H * nqb * k * 4))
+            + r256(scores) + r256(H * nqb * (F + k) * 4))
     assert api.workspace_bytes(cfg) == want
 
 

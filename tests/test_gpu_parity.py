@@ -152,7 +152,7 @@ def test_gate_combine(dev, name):
 
 
 def _fused(cfg, d):
-    idx = torch.empty((cfg.H, cfg.nqb, cfg.topk), dtype=torch.int32, device=d["q"].device)
+    idx = torch.empty((cfg.H, cfg.nqb, cfg.nsel), dtype=torch.int32, device=d["q"].device)
     out = api.sparse_attn_fwd(cfg, d["q"], d["k"], d["v"], d["gates"], idx_out=idx)
     torch.cuda.synchronize()
     return f64(out), idx.cpu().numpy()
@@ -247,3 +247,64 @@ def test_bounded_wait_timeout_is_reported_and_the_context_survives(dev):
     assert api.read_device_status(word) == 0
     rlse, ro, rs = O.cmp_attn(pb, O.bf16_bits(x.q), f64(kc), f64(vc))
     check_close("lse after a timeout", f64(lse), rlse, 2e-5)
+
+
+# --------------------------------------------------------------------------------------------
+# VGGT variant: the reference frame's blocks open every selection list
+# --------------------------------------------------------------------------------------------
+
+FORCED = {  # name: (L, H, b, k, forced, seed)
+    "vggt_4_views": (4 * 1374, 2, 64, 16, 22, 20),  # P = 1374 tokens per view, F = ceil(P/b)
+    "forced_b32_odd_list": (2000, 2, 32, 5, 6, 21),  # F + k odd: the last step is half empty
+    "forced_k_above_32": (3000, 2, 32, 36, 5, 22),  # top-k kernel on the materialised scores
+    "forced_plus_k_is_nb": (1000, 2, 64, 12, 4, 23),  # F + k = nb: dense selection
+}
+
+
+def forced_inputs(name, device):
+    L, H, b, k, F, seed = FORCED[name]
+    x = synth.make_inputs(L, H, 64, b, seed)
+    cfg = api.Config(L=L, H=H, block=b, topk=k, forced=F)
+    pb = O.Problem(L, H, 64, b, k, forced=F)
+    d = {n: getattr(x, n).to(device) for n in ("q", "k", "v", "gates")}
+    return cfg, pb, x, d
+
+
+@pytest.mark.parametrize("name", list(FORCED))
+def test_forced_whole_path(dev, name):
+    cfg, pb, x, d = forced_inputs(name, dev)
+    out, idx = _fused(cfg, d)
+    assert idx.shape == (cfg.H, cfg.nqb, cfg.forced + cfg.topk)
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    ref = O.sparse_attn(pb, *bits, x.gates.numpy())
+    stats = check_selection(idx, ref.idx, ref.gap, ref.scores, cfg.topk, cfg.forced)
+    cond = O.sparse_attn(pb, *bits, x.gates.numpy(), idx_given=idx, pooled=(ref.kc, ref.vc))
+    check_output(out, cond.out)
+    if stats["sets_equal"] == 1.0:
+        check_output(out, ref.out)
+
+
+@pytest.mark.parametrize("name", list(FORCED))
+def test_forced_topk_blocks_bit_exact(dev, name):
+    cfg, pb, x, d = forced_inputs(name, dev)
+    kc, vc = O.pool(pb, O.bf16_bits(x.k)), O.pool(pb, O.bf16_bits(x.v))
+    _, _, rs = O.cmp_attn(pb, O.bf16_bits(x.q), kc, vc)
+    s32 = rs.astype(np.float32)
+    for scores in (s32, np.round(s32 * 4) / 4):
+        scores = np.ascontiguousarray(scores, np.float32)
+        got = api.topk_blocks(cfg, torch.from_numpy(scores).to(dev)).cpu().numpy()
+        want, _ = O.topk(scores.astype(np.float64), cfg.topk, cfg.forced)
+        np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("name", ["vggt_4_views", "forced_b32_odd_list"])
+def test_forced_sel_attn(dev, name):
+    cfg, pb, x, d = forced_inputs(name, dev)
+    rng = np.random.default_rng(FORCED[name][-1])
+    F, k = cfg.forced, cfg.topk
+    idx = np.stack([np.stack([np.concatenate([np.arange(F), F + rng.permutation(cfg.nb - F)[:k]])
+                              for _ in range(cfg.nqb)]) for _ in range(cfg.H)]).astype(np.int32)
+    o = api.sel_attn(cfg, d["q"], d["k"], d["v"], torch.from_numpy(idx).to(dev))
+    torch.cuda.synchronize()
+    ref = O.sel_attn(pb, O.bf16_bits(x.q), O.bf16_bits(x.k), O.bf16_bits(x.v), idx)
+    check_close("o_sel", f64(o), ref, 2.0 ** -8 * np.abs(f64(x.v)).max() + 1e-6, rl2=4e-3)
