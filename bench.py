@@ -111,7 +111,8 @@ def algorithmic(cfg):
         "sel_flops": sel_flops,
         "flops": cmp_flops + sel_flops,
         "stage_work": {
-            "pool": ("hbm", 2.0 * (L + nb) * H * d * 2),                       # bytes
+            # K, V read; Kc, Vc and the head-major copies of K, V (nb*b rows) written
+            "pool": ("hbm", 2.0 * (L + nb + nb * b) * H * d * 2),              # bytes
             "cmp": ("tensor", cmp_flops),                                     # flops
             "topk": ("hbm", H * nqb * (nb * 4.0 + k * 4.0)),                  # bytes
             "sel_combine": ("tensor", sel_flops),                             # flops

@@ -2,6 +2,7 @@
 // of the fused call, and the launch sequence. The operation and its conventions are defined in
 // include/s3r.h.
 #include <atomic>
+#include <climits>
 #include <cmath>
 
 #include "internal.h"
@@ -50,15 +51,23 @@ s3r_status derive(const s3r_params* prm, Problem* out) {
 s3r_status launched(cudaError_t e) { return e == cudaSuccess ? S3R_OK : S3R_ERR_CUDA; }
 
 // Workspace of the fused call, every region 256-byte aligned:
-//   status word | Kc [nb,H,d] bf16 | Vc | O_cmp [L,H,d] f32 | scores [H,nqb,nb] f32
-//   | idx [H,nqb,k] i32
+//   status word | Kc [nb,H,d] bf16 | Vc | Kh [H,nb*b,d] bf16 | Vh | O_cmp [L,H,d] f32
+//   | scores [H,nqb,nb] f32 | idx [H,nqb,forced+k] i32
+// Kh, Vh are head-major copies of K and V written by the pooling pass, from which the selection
+// branch gathers each selected block as contiguous rows.
 // The score matrix is only materialised when k > kFusedTopkMax; otherwise the compressed-branch
 // kernel selects the top-k on the fly and the scores region is empty.
 struct Workspace {
-  size_t status, kc, vc, o_cmp, scores, idx, total;
+  size_t status, kc, vc, kh, vh, o_cmp, scores, idx, total;
 };
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// The head-major copies are addressed with 32-bit TMA row coordinates (H * nb*b rows); beyond
+// that the selection branch gathers from K and V themselves.
+bool use_head_major(const Problem& p) {
+  return static_cast<int64_t>(p.H) * p.nb * p.b <= INT32_MAX;
+}
 
 Workspace layout(const Problem& p) {
   Workspace w{};
@@ -72,6 +81,9 @@ Workspace layout(const Problem& p) {
   w.status = take(4);
   w.kc = take(static_cast<size_t>(p.nb) * HD * 2);
   w.vc = take(static_cast<size_t>(p.nb) * HD * 2);
+  const size_t copy = use_head_major(p) ? static_cast<size_t>(p.nb) * p.b * HD * 2 : 0;
+  w.kh = take(copy);
+  w.vh = take(copy);
   w.o_cmp = take(static_cast<size_t>(p.L) * HD * 4);
   w.scores = take(p.k > kFusedTopkMax ? static_cast<size_t>(p.H) * p.nqb * p.nb * 4 : 0);
   w.idx = take(static_cast<size_t>(p.H) * p.nqb * p.nsel * 4);
@@ -105,6 +117,9 @@ int fused_forward(const s3r_params* params, const uint16_t* q, const uint16_t* k
   if (!p.status) p.status = status;
   uint16_t* kc = reinterpret_cast<uint16_t*>(base + w.kc);
   uint16_t* vc = reinterpret_cast<uint16_t*>(base + w.vc);
+  const bool hm = use_head_major(p);
+  uint16_t* kh = hm ? reinterpret_cast<uint16_t*>(base + w.kh) : nullptr;
+  uint16_t* vh = hm ? reinterpret_cast<uint16_t*>(base + w.vh) : nullptr;
   float* o_cmp = reinterpret_cast<float*>(base + w.o_cmp);
   float* scores = reinterpret_cast<float*>(base + w.scores);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
@@ -115,7 +130,7 @@ int fused_forward(const s3r_params* params, const uint16_t* q, const uint16_t* k
   };
   if (cudaMemsetAsync(status, 0, 4, stream) != cudaSuccess) return S3R_ERR_CUDA;
   if (mark(0) != cudaSuccess) return S3R_ERR_CUDA;
-  if ((st = launched(launch_pool_kv(p, k, v, kc, vc, stream))) != S3R_OK) return st;
+  if ((st = launched(launch_pool_kv(p, k, v, kc, vc, kh, vh, stream))) != S3R_OK) return st;
   if (mark(1) != cudaSuccess) return S3R_ERR_CUDA;
   const bool fused_topk = p.k <= kFusedTopkMax;
   if ((st = launched(launch_cmp_attn_tc(p, q, kc, vc, nullptr, o_cmp, fused_topk ? nullptr : scores,
@@ -124,7 +139,8 @@ int fused_forward(const s3r_params* params, const uint16_t* q, const uint16_t* k
   if (mark(2) != cudaSuccess) return S3R_ERR_CUDA;
   if (!fused_topk && (st = launched(launch_topk(p, scores, idx, stream))) != S3R_OK) return st;
   if (mark(3) != cudaSuccess) return S3R_ERR_CUDA;
-  st = launched(launch_sel_attn(p, q, k, v, idx, nullptr, o_cmp, gate_logits, out, stream));
+  st = launched(launch_sel_attn(p, q, hm ? kh : k, hm ? vh : v, hm, idx, nullptr, o_cmp, gate_logits,
+                                out, stream));
   if (st != S3R_OK) return st;
   return mark(4) == cudaSuccess ? S3R_OK : S3R_ERR_CUDA;
 }
@@ -175,7 +191,7 @@ s3r_status s3r_compress_kv(const s3r_params* params, const s3r_bf16* k, const s3
   if (st != S3R_OK) return st;
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_cmp) || !aligned16(v_cmp))
     return S3R_ERR_INVALID_ARG;
-  return launched(launch_pool_kv(p, k, v, k_cmp, v_cmp, stream));
+  return launched(launch_pool_kv(p, k, v, k_cmp, v_cmp, nullptr, nullptr, stream));
 }
 
 s3r_status s3r_cmp_attn_and_score(const s3r_params* params, const s3r_bf16* q,
@@ -206,7 +222,7 @@ s3r_status s3r_sel_attn(const s3r_params* params, const s3r_bf16* q, const s3r_b
   if (st != S3R_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o_sel))
     return S3R_ERR_INVALID_ARG;
-  return launched(launch_sel_attn(p, q, k, v, idx, o_sel, nullptr, nullptr, nullptr, stream));
+  return launched(launch_sel_attn(p, q, k, v, false, idx, o_sel, nullptr, nullptr, nullptr, stream));
 }
 
 s3r_status s3r_gate_combine(const s3r_params* params, const float* o_cmp, const float* o_sel,

@@ -193,9 +193,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_empty[b], kSoftmaxThreads);
+      mbar_init(&bars->s_empty[b], kSoftmaxWarps);
     }
-    mbar_init(&bars->p_full, kSoftmaxThreads);
+    mbar_init(&bars->p_full, kSoftmaxWarps);
     mbar_init(&bars->p_empty, 1);
     for (int r = 0; r < kRed; ++r) {
       mbar_init(&bars->red_full[r], kSoftmaxWarps);
@@ -342,7 +342,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       tmem_wait_ld_n<16>(ra);
       tmem_wait_ld_n<16>(rb);
       tc_fence_before();
-      mbar_arrive(&bars->s_empty[b]);
+      __syncwarp();  // one arrival per warp: its lanes' TMEM loads have all completed
+      if (lane == 0) mbar_arrive(&bars->s_empty[b]);
       float v[4][8];
       unpack_rows(ra, rb, v);
       if (static_cast<int64_t>(t + 1) * kBN > a.nb) {  // ragged last tile
@@ -421,7 +422,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       tmem_wait_ld_n<16>(ra);
       tmem_wait_ld_n<16>(rb);
       tc_fence_before();
-      mbar_arrive(&bars->s_empty[b]);
+      __syncwarp();  // one arrival per warp: its lanes' TMEM loads have all completed
+      if (lane == 0) mbar_arrive(&bars->s_empty[b]);
       float v[4][8];
       unpack_rows(ra, rb, v);
 #pragma unroll
@@ -489,7 +491,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       tmem_wait_st_keep8(p0);
       tmem_wait_st_keep8(p1);
       tc_fence_before();
-      mbar_arrive(&bars->p_full);
+      __syncwarp();  // one arrival per warp: its lanes' TMEM stores have all completed
+      if (lane == 0) mbar_arrive(&bars->p_full);
     }
     if (ok && (ok = mbar_wait(&bars->o_full, 0, abort, lim))) {
       tc_fence_after();

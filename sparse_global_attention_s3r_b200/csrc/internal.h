@@ -23,8 +23,9 @@ struct Problem {
 };
 
 // Each launcher enqueues one kernel on `st` and returns cudaGetLastError().
+// kh, vh (nullable): head-major copies [H, nb*b, 64] of K and V written in the same pass.
 cudaError_t launch_pool_kv(const Problem& p, const uint16_t* k, const uint16_t* v, uint16_t* kc,
-                           uint16_t* vc, cudaStream_t st);
+                           uint16_t* vc, uint16_t* kh, uint16_t* vh, cudaStream_t st);
 // Largest top-k the compressed-branch kernel selects on the fly (one key per lane of a warp).
 constexpr int kFusedTopkMax = 32;
 
@@ -36,8 +37,9 @@ cudaError_t launch_cmp_attn_tc(const Problem& p, const uint16_t* q, const uint16
 cudaError_t launch_topk(const Problem& p, const float* scores, int32_t* idx, cudaStream_t st);
 // o_sel != nullptr: write the selection output (fp32). Otherwise fuse the gated combine:
 // read o_cmp and gates and write out (bf16).
+// k, v: [L, H, 64] token-major, or (head_major) the [H, nb*b, 64] copies of launch_pool_kv.
 cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t* k,
-                            const uint16_t* v, const int32_t* idx, float* o_sel,
+                            const uint16_t* v, bool head_major, const int32_t* idx, float* o_sel,
                             const float* o_cmp, const float* gates, uint16_t* out,
                             cudaStream_t st);
 cudaError_t launch_gate_combine(const Problem& p, const float* o_cmp, const float* o_sel,

@@ -8,6 +8,10 @@
 // walks the b rows of its block, so a warp reads 512 contiguous bytes per row and the block's
 // whole [b, H*d] slab is read exactly once. fp32 accumulation, one IEEE division by the valid
 // count, round-to-nearest-even to bf16. Algorithmic traffic: 2 * (L + nb) * H * d * 2 bytes.
+// Optionally the same pass also writes head-major copies Kh, Vh [H, nb*b, 64] of K and V (rows
+// past L zero), so that the selection branch can gather a selected block of one head as b
+// contiguous 128-byte rows rather than rows H*128 bytes apart; that adds 2 * nb*b * H*d * 2 bytes
+// of writes.
 #include "common.cuh"
 #include "internal.h"
 
@@ -27,9 +31,12 @@ __device__ __forceinline__ void add_bf16x8(float acc[8], const uint4& x) {
 
 __global__ void __launch_bounds__(kPoolThreads)
     pool_kv_kernel(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
-                   uint16_t* __restrict__ kc, uint16_t* __restrict__ vc, int64_t L, int HD, int b) {
+                   uint16_t* __restrict__ kc, uint16_t* __restrict__ vc,
+                   uint16_t* __restrict__ kh, uint16_t* __restrict__ vh, int64_t L, int64_t Lp,
+                   int HD, int b) {
   const uint16_t* src = blockIdx.z ? v : k;
   uint16_t* dst = blockIdx.z ? vc : kc;
+  uint16_t* hm = blockIdx.z ? vh : kh;  // head-major copy [H, Lp, 64] or null
   const int chunk = blockIdx.x * kPoolThreads + threadIdx.x;  // 16-byte chunk within a row
   const int chunks = HD / 8;
   if (chunk >= chunks) return;
@@ -37,6 +44,9 @@ __global__ void __launch_bounds__(kPoolThreads)
   const int64_t t0 = j * b;
   const int n = static_cast<int>(min(static_cast<int64_t>(b), L - t0));
   const uint4* p = reinterpret_cast<const uint4*>(src + t0 * HD) + chunk;
+  // head chunk >> 3, 16-byte piece chunk & 7 of its 128-byte row; rows are 8 uint4 apart
+  uint4* hp = hm ? reinterpret_cast<uint4*>(hm + ((chunk >> 3) * Lp + t0) * 64) + (chunk & 7)
+                 : nullptr;
 
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   int t = 0;
@@ -44,10 +54,20 @@ __global__ void __launch_bounds__(kPoolThreads)
     uint4 x[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) x[u] = __ldg(p + static_cast<int64_t>(t + u) * chunks);
+    if (hp) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) hp[(t + u) * 8] = x[u];
+    }
 #pragma unroll
     for (int u = 0; u < 8; ++u) add_bf16x8(acc, x[u]);
   }
-  for (; t < n; ++t) add_bf16x8(acc, __ldg(p + static_cast<int64_t>(t) * chunks));
+  for (; t < n; ++t) {
+    const uint4 x = __ldg(p + static_cast<int64_t>(t) * chunks);
+    if (hp) hp[t * 8] = x;
+    add_bf16x8(acc, x);
+  }
+  if (hp)
+    for (; t < b; ++t) hp[t * 8] = make_uint4(0u, 0u, 0u, 0u);  // padding rows of the last block
 
   const float fn = static_cast<float>(n);
   uint4 o;
@@ -61,10 +81,10 @@ __global__ void __launch_bounds__(kPoolThreads)
 }  // namespace
 
 cudaError_t launch_pool_kv(const Problem& p, const uint16_t* k, const uint16_t* v, uint16_t* kc,
-                           uint16_t* vc, cudaStream_t st) {
+                           uint16_t* vc, uint16_t* kh, uint16_t* vh, cudaStream_t st) {
   const int HD = p.H * p.d;
   dim3 grid((HD / 8 + kPoolThreads - 1) / kPoolThreads, static_cast<unsigned>(p.nb), 2);
-  pool_kv_kernel<<<grid, kPoolThreads, 0, st>>>(k, v, kc, vc, p.L, HD, p.b);
+  pool_kv_kernel<<<grid, kPoolThreads, 0, st>>>(k, v, kc, vc, kh, vh, p.L, p.nb * p.b, HD, p.b);
   count_launch();
   return cudaGetLastError();
 }

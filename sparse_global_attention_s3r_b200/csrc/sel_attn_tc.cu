@@ -21,6 +21,8 @@
 // Roles (224 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-5 softmax
 // (warp w holds lane quadrant w%4), warp 6 idle. TMEM: S (128 cols) | O (64) | P (64 = 128 keys).
 // Every wait is bounded in time and watches a CTA abort flag (S3R_DEV_TIMEOUT on expiry).
+#include <climits>
+
 #include "s3r.h"
 #include "common.cuh"
 #include "internal.h"
@@ -70,6 +72,8 @@ struct SelArgs {
   uint16_t* out;       // [L, H, 64] bf16 (fused combine)
   int64_t L, nb, nqb;
   int64_t nb_full;  // key blocks that lie wholly below L
+  int kv_xh, kv_yh;  // K/V box of head h, token tok at (h*kv_xh, h*kv_yh + tok): token-major
+                     // [L, H, 64] is (64, 0), the head-major [H, nb*b, 64] copy is (0, nb*b)
   int H, b, lb, topk, nsteps;  // lb = log2(b)
   float scale_log2;
   uint32_t flags;
@@ -134,8 +138,8 @@ __global__ void __maxnreg__(128)
       mbar_init(&bars->kv_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_empty, kSoftmaxThreads);
-    mbar_init(&bars->p_full, kSoftmaxThreads);
+    mbar_init(&bars->s_empty, kSoftmaxThreads / 32);
+    mbar_init(&bars->p_full, kSoftmaxThreads / 32);
     mbar_init(&bars->p_empty, 1);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->drain, 1);
@@ -178,9 +182,9 @@ __global__ void __maxnreg__(128)
             const int64_t j = sel_block(list, pos >> a.lb, a.topk, a.nb, valid);
             const int64_t tok = j * a.b + (pos & (a.b - 1));
             const uint32_t row_off = (qb * kStep + part * box) * 128;
-            tma_load_2d(sk + row_off, &tmK, h * 64, static_cast<int32_t>(tok), &bars->kv_full[stage]);
-            tma_load_2d(sk + kTileBytes + row_off, &tmV, h * 64, static_cast<int32_t>(tok),
-                        &bars->kv_full[stage]);
+            const int32_t x = h * a.kv_xh, y = static_cast<int32_t>(h * a.kv_yh + tok);
+            tma_load_2d(sk + row_off, &tmK, x, y, &bars->kv_full[stage]);
+            tma_load_2d(sk + kTileBytes + row_off, &tmV, x, y, &bars->kv_full[stage]);
           }
         }
         issued = t + 1;
@@ -276,7 +280,8 @@ __global__ void __maxnreg__(128)
       tmem_wait_ld_n<16>(r[2]);
       tmem_wait_ld_n<16>(r[3]);
       tc_fence_before();
-      mbar_arrive(&bars->s_empty);
+      __syncwarp();  // one arrival per warp: its lanes' TMEM loads have all completed
+      if (lane == 0) mbar_arrive(&bars->s_empty);
       float v[4][16];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
@@ -394,7 +399,8 @@ __global__ void __maxnreg__(128)
         tmem_wait_st_keep8(a1);
       }
       tc_fence_before();
-      mbar_arrive(&bars->p_full);
+      __syncwarp();  // one arrival per warp: its lanes' TMEM stores have all completed
+      if (lane == 0) mbar_arrive(&bars->p_full);
     }
 
     // finish: O / l per row (lane = row for the 32x32b loads), then write O_sel or the combine
@@ -469,14 +475,19 @@ __global__ void __maxnreg__(128)
 }  // namespace
 
 cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t* k,
-                            const uint16_t* v, const int32_t* idx, float* o_sel,
+                            const uint16_t* v, bool head_major, const int32_t* idx, float* o_sel,
                             const float* o_cmp, const float* gates, uint16_t* out,
                             cudaStream_t st) {
   const int box = p.b < kStep ? p.b : kStep;
+  const int64_t Lp = p.nb * p.b;
+  if (head_major && p.H * Lp > INT32_MAX) return cudaErrorInvalidValue;  // TMA coordinates
   CUtensorMap tq, tk, tv;
-  if (!make_tmap_head_rows(&tq, q, p.L, p.H, kBM) || !make_tmap_head_rows(&tk, k, p.L, p.H, box) ||
-      !make_tmap_head_rows(&tv, v, p.L, p.H, box))
-    return cudaErrorInvalidValue;
+  const bool maps =
+      make_tmap_head_rows(&tq, q, p.L, p.H, kBM) &&
+      (head_major ? make_tmap_rows64(&tk, k, p.H * Lp, box) && make_tmap_rows64(&tv, v, p.H * Lp, box)
+                  : make_tmap_head_rows(&tk, k, p.L, p.H, box) &&
+                        make_tmap_head_rows(&tv, v, p.L, p.H, box));
+  if (!maps) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(sel_attn_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -486,7 +497,8 @@ cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t*
   if (e != cudaSuccess) return e;
   const int64_t ntok = static_cast<int64_t>(p.nsel) * p.b;
   const int lb = p.b == 32 ? 5 : p.b == 64 ? 6 : 7;
-  SelArgs a{idx, o_sel, o_cmp, gates, out, p.L, p.nb, p.nqb, p.L / p.b, p.H, p.b, lb, p.nsel,
+  SelArgs a{idx, o_sel, o_cmp, gates, out, p.L, p.nb, p.nqb, p.L / p.b,
+            head_major ? 0 : 64, head_major ? static_cast<int>(Lp) : 0, p.H, p.b, lb, p.nsel,
             static_cast<int>((ntok + kStep - 1) / kStep), p.scale_log2, p.flags, p.status,
             (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull};
   dim3 grid(static_cast<unsigned>((p.L + kBM - 1) / kBM), p.H);

@@ -121,7 +121,8 @@ def test_workspace_size_matches_layout(L, H, b, k, F):
     cfg = api.Config(L=L, H=H, block=b, topk=k, forced=F)
     nb, nqb, d = cfg.nb, cfg.nqb, 64
     scores = H * nqb * nb * 4 if k > 32 else 0  # materialised only when k exceeds 32
-    want = (r256(4) + 2 * r256(nb * H * d * 2) + r256(L * H * d * 4)
+    copies = 2 * r256(nb * b * H * d * 2) if H * nb * b <= 2**31 - 1 else 0  # head-major K, V
+    want = (r256(4) + 2 * r256(nb * H * d * 2) + copies + r256(L * H * d * 4)
             + r256(scores) + r256(H * nqb * (F + k) * 4))
     assert api.workspace_bytes(cfg) == want
 
