@@ -71,7 +71,13 @@ SM_COUNT = 148
 # the step, from one ncu capture of the default workload (python bench.py --steps 2 --warmup 3
 # --no-cpu-baseline), with the SHA-256 of the sources that kernel was built from: once any of them
 # changes, the figure no longer describes the kernel and the roofline reports null.
-TRAFFIC = {}
+TRAFFIC = {
+    "cmp": {"workload": "n1000", "bytes": 3004117760 + 5630263040,
+             "sources": ["sparse_global_attention_s3r_b200/csrc/cmp_attn_tc.cu",
+                         "sparse_global_attention_s3r_b200/csrc/common.cuh",
+                         "sparse_global_attention_s3r_b200/csrc/sm100.cuh"],
+             "sha256": "03f6d30ab8794617f4072b8b8c86c4b81a876495bec52d65bc8ebb97d3fa9d12"},
+}
 
 
 def _sources_sha(paths):
