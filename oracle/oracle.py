@@ -39,6 +39,10 @@ class _Params(ctypes.Structure):
         ("exact_pool", ctypes.c_int32),
         ("threads", ctypes.c_int32),
         ("forced", ctypes.c_int32),
+        ("grid_h", ctypes.c_int32),
+        ("grid_w", ctypes.c_int32),
+        ("special", ctypes.c_int32),
+        ("win_h", ctypes.c_int32),
     ]
 
 
@@ -62,10 +66,14 @@ def lib():
             "s3r_ref_topk": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, p, p, p],
             "s3r_ref_sel": [p, p, p, p, p, ctypes.c_int64, p, p],
             "s3r_ref_combine": [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, p, p, p, p],
+            "s3r_ref_block_tokens": [p, ctypes.c_int64, p],
         }.items():
             fn = getattr(L, name)
             fn.restype = ctypes.c_int
             fn.argtypes = args
+        L.s3r_ref_num_blocks.restype = ctypes.c_int64
+        L.s3r_ref_num_blocks.argtypes = [ctypes.c_void_p]
+        L.s3r_ref_block_tokens.restype = ctypes.c_int64
         _LIB = L
     return _LIB
 
@@ -82,10 +90,27 @@ class Problem:
     qblock: int = 64
     scale: Optional[float] = None  # None -> 1/sqrt(d)
     forced: int = 0  # leading key blocks kept in every selection list (VGGT reference frame)
+    # 2-D windows (grid_h > 0): views of `special` tokens + a grid_h x grid_w patch grid, key
+    # blocks = the special tokens of a view, then win_h x (block / win_h) windows of its grid
+    grid_h: int = 0
+    grid_w: int = 0
+    special: int = 0
+    win_h: int = 0
 
     @property
     def nb(self) -> int:
-        return -(-self.L // self.block)
+        if self.grid_h == 0:
+            return -(-self.L // self.block)
+        n = lib().s3r_ref_num_blocks(ctypes.byref(_params(self)))
+        assert n > 0, "invalid 2-D geometry"
+        return int(n)
+
+    def block_tokens(self, j: int) -> np.ndarray:
+        """Tokens of key block j, ascending."""
+        out = np.empty(self.block, np.int64)
+        n = lib().s3r_ref_block_tokens(ctypes.byref(_params(self)), j, _ptr(out))
+        assert n >= 0, n
+        return out[:n].copy()
 
     @property
     def nqb(self) -> int:
@@ -110,7 +135,8 @@ class Problem:
 
 def _params(pb: Problem, exact_pool: bool = False, threads: int = 0) -> _Params:
     return _Params(pb.L, pb.H, pb.d, pb.block, pb.qblock, pb.topk, pb.softmax_scale,
-                   1 if exact_pool else 0, threads, pb.forced)
+                   1 if exact_pool else 0, threads, pb.forced, pb.grid_h, pb.grid_w, pb.special,
+                   pb.win_h)
 
 
 def _ptr(a: np.ndarray) -> ctypes.c_void_p:

@@ -16,7 +16,9 @@
  *   §4 "Efficient Kernel": top-k and softmax are computed together, so the scores are softmax
  *      probabilities.
  * Where the pages leave a step open, the reading taken is the plainest one the rest supports:
- * 1-D blocks of b consecutive tokens of the flattened sequence, the last block partial; pooled
+ * 1-D blocks of b consecutive tokens of the flattened sequence, the last block partial (or, as an
+ * option, 2-D windows of each view's patch grid with the view's special tokens as a block of
+ * their own: the "spatial downsampling" read literally); pooled
  * means divide by the count of valid tokens; scores are per head; probabilities are summed over
  * the rows of a query block that lie inside the sequence; ties in the top-k go to the lower block
  * index; two independent sigmoid gates, one per branch.
@@ -31,6 +33,11 @@
  *                       blocks, brute force over the subsets of the other blocks, and the forced
  *                       blocks' own scores have no effect.
  *   s3r_ref_sel         with forced blocks, dense attention when F + k = nb.
+ *   2-D windows         every token in exactly one block, blocks are patch rectangles cut only
+ *                       at the grid edges; one-patch-high windows reproduce the 1-D path bit for
+ *                       bit; a ramp pools to its value at the window centre; selection equals
+ *                       SDPA under the window mask; patches permuted within windows change
+ *                       nothing.
  *   s3r_ref_sel         dense attention (torch SDPA, fp64) when k = nb; brute force per query.
  *   s3r_ref_combine     gate limits and the zero-logit midpoint.
  *   whole pipeline      composition of the pinned steps plus permutation invariances.
@@ -125,10 +132,65 @@ static void parallel_for(int64_t ntasks, int threads, task_fn fn, void* ctx) {
 /* argument checks shared by the entry points of this file                                     */
 /* ------------------------------------------------------------------------------------------ */
 
+static int check_geometry(const s3r_ref_params* p) {
+  if (p->grid_h == 0) return 0; /* 1-D blocks */
+  if (p->grid_h < 1 || p->grid_w < 1 || p->special < 0 || p->special > p->block) return -1;
+  if (p->win_h < 1 || p->block % p->win_h != 0) return -1;
+  const int64_t P = (int64_t)p->special + (int64_t)p->grid_h * p->grid_w;
+  return p->L % P == 0 ? 0 : -1;
+}
+
 static int check_params(const s3r_ref_params* p) {
   if (!p) return -1;
   if (p->L < 1 || p->H < 1 || p->d < 1 || p->block < 1 || p->qblock < 1) return -1;
-  return 0;
+  return check_geometry(p);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* key-block geometry: which tokens each key block holds                                       */
+/* ------------------------------------------------------------------------------------------ */
+
+/* blocks of one view under 2-D windows: the special-token block, then the windows */
+static int64_t blocks_per_view(const s3r_ref_params* p) {
+  const int64_t win_w = p->block / p->win_h;
+  const int64_t rows = ceil_div(p->grid_h, p->win_h), cols = ceil_div(p->grid_w, win_w);
+  return (p->special > 0 ? 1 : 0) + rows * cols;
+}
+
+int64_t s3r_ref_num_blocks(const s3r_ref_params* p) {
+  if (check_params(p)) return 0;
+  if (p->grid_h == 0) return ceil_div(p->L, p->block);
+  const int64_t P = (int64_t)p->special + (int64_t)p->grid_h * p->grid_w;
+  return (p->L / P) * blocks_per_view(p);
+}
+
+int64_t s3r_ref_block_tokens(const s3r_ref_params* p, int64_t j, int64_t* out) {
+  if (check_params(p) || !out || j < 0 || j >= s3r_ref_num_blocks(p)) return -1;
+  int64_t n = 0;
+  if (p->grid_h == 0) { /* b consecutive tokens, the last block cut at L */
+    for (int64_t t = j * p->block; t < (j + 1) * p->block && t < p->L; ++t) out[n++] = t;
+    return n;
+  }
+  const int64_t P = (int64_t)p->special + (int64_t)p->grid_h * p->grid_w;
+  const int64_t per_view = blocks_per_view(p);
+  const int64_t view = j / per_view;
+  int64_t m = j % per_view; /* block within the view */
+  const int64_t first = view * P;
+  if (p->special > 0) {
+    if (m == 0) { /* the view's camera / register tokens */
+      for (int64_t t = 0; t < p->special; ++t) out[n++] = first + t;
+      return n;
+    }
+    m -= 1;
+  }
+  /* window (wr, wc) of the view's patch grid: patch rows wr*win_h.., columns wc*win_w.. */
+  const int64_t win_w = p->block / p->win_h;
+  const int64_t cols = ceil_div(p->grid_w, win_w);
+  const int64_t wr = m / cols, wc = m % cols;
+  for (int64_t r = wr * p->win_h; r < (wr + 1) * p->win_h && r < p->grid_h; ++r)
+    for (int64_t c = wc * win_w; c < (wc + 1) * win_w && c < p->grid_w; ++c)
+      out[n++] = first + p->special + r * p->grid_w + c;
+  return n;
 }
 
 /* Rows of the chosen query blocks: first row and count of each, and their concatenated offset. */
@@ -187,21 +249,21 @@ static void pool_task(void* vctx, int64_t j) {
   const pool_ctx* c = (const pool_ctx*)vctx;
   const s3r_ref_params* p = c->p;
   const int64_t HD = (int64_t)p->H * p->d;
-  int64_t t0 = j * p->block;
-  int64_t t1 = t0 + p->block < p->L ? t0 + p->block : p->L;
-  double n = (double)(t1 - t0);
+  int64_t* tok = (int64_t*)malloc(sizeof(int64_t) * (size_t)p->block);
+  const int64_t n = s3r_ref_block_tokens(p, j, tok);
   for (int64_t e = 0; e < HD; ++e) {
     double sum = 0.0;
-    for (int64_t t = t0; t < t1; ++t) sum += bf16_value(c->x[t * HD + e]);
-    double mean = sum / n;
+    for (int64_t a = 0; a < n; ++a) sum += bf16_value(c->x[tok[a] * HD + e]);
+    double mean = sum / (double)n;
     c->out[j * HD + e] = p->exact_pool ? mean : s3r_ref_round_bf16(mean);
   }
+  free(tok);
 }
 
 int s3r_ref_pool(const s3r_ref_params* p, const uint16_t* x, double* out) {
   if (check_params(p) || !x || !out) return -1;
   pool_ctx c = {p, x, out};
-  parallel_for(ceil_div(p->L, p->block), p->threads, pool_task, &c);
+  parallel_for(s3r_ref_num_blocks(p), p->threads, pool_task, &c);
   return 0;
 }
 
@@ -224,7 +286,7 @@ static void cmp_task(void* vctx, int64_t task) {
   const cmp_ctx* c = (const cmp_ctx*)vctx;
   const s3r_ref_params* p = c->p;
   const row_map* rm = c->rm;
-  const int64_t nb = ceil_div(p->L, p->block);
+  const int64_t nb = s3r_ref_num_blocks(p);
   const int64_t H = p->H, d = p->d, HD = H * d;
   const int64_t h = task / rm->nq, i = task % rm->nq;
   double* s = (double*)malloc(sizeof(double) * (size_t)nb);
@@ -350,7 +412,7 @@ static void sel_task(void* vctx, int64_t task) {
   sel_ctx* c = (sel_ctx*)vctx;
   const s3r_ref_params* p = c->p;
   const row_map* rm = c->rm;
-  const int64_t nb = ceil_div(p->L, p->block);
+  const int64_t nb = s3r_ref_num_blocks(p);
   const int64_t H = p->H, d = p->d, HD = H * d;
   const int64_t h = task / rm->nq, i = task % rm->nq;
   const int32_t n_list = p->forced + p->topk; /* always-kept blocks, then the top-k */
@@ -368,7 +430,7 @@ static void sel_task(void* vctx, int64_t task) {
     }
     if (chosen[j]) continue;
     chosen[j] = 1;
-    for (int64_t t = j * p->block; t < (j + 1) * p->block && t < p->L; ++t) tokens[nt++] = t;
+    nt += s3r_ref_block_tokens(p, j, tokens + nt);
   }
   double* s = (double*)malloc(sizeof(double) * (size_t)(nt > 0 ? nt : 1));
 

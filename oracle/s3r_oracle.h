@@ -14,7 +14,8 @@
  *
  * Conventions (all arrays dense, row-major):
  *   Q, K, V      [L, H, d]   bf16, passed as their raw 16-bit patterns (uint16_t)
- *   pooled K/V   [nb, H, d]  double          nb  = ceil(L / block)
+ *   pooled K/V   [nb, H, d]  double          nb  = ceil(L / block) for 1-D blocks, else the
+ *                                           number of 2-D windows (see s3r_ref_params)
  *   gates        [L, H, 2]   float           [...,0] compression gate logit, [...,1] selection
  *   lse          [H, R]      double          R = rows of the chosen query blocks (see below)
  *   o_cmp, o_sel [R, H, d]   double
@@ -49,7 +50,23 @@ typedef struct {
   int32_t forced;   /* F: key blocks 0 .. F-1 open every selection list (the VGGT variant keeps the
                        reference frame's tokens for every query); the top-k then picks k more
                        among blocks F .. nb-1, so a list holds F + k blocks. 0 = plain top-k. */
+  /* Key-block geometry. grid_h == 0: 1-D blocks, block j = tokens [j*b, min((j+1)*b, L)).
+   * grid_h > 0: 2-D windows on each view's patch grid ("spatial downsampling", Methodologie §1).
+   * The sequence is N = L / P views of P = special + grid_h * grid_w tokens each: `special`
+   * leading tokens (camera and register tokens), then the grid_h x grid_w patches in row-major
+   * order. Each view contributes, in this order, one block holding its special tokens (when
+   * special > 0) and the windows of win_h x (b / win_h) patches that tile its grid from the
+   * top-left, row by row; windows at the right and bottom edges hold only the patches inside
+   * the grid. Blocks are numbered view by view. Query blocks stay 64 consecutive tokens. */
+  int32_t grid_h, grid_w, special, win_h;
 } s3r_ref_params;
+
+/* Number of key blocks nb of the geometry in p (0 if the geometry is invalid). */
+int64_t s3r_ref_num_blocks(const s3r_ref_params* p);
+
+/* Tokens of key block j in ascending order, written to out (room for p->block entries);
+ * returns their count, or -1 for a bad argument. */
+int64_t s3r_ref_block_tokens(const s3r_ref_params* p, int64_t j, int64_t* out);
 
 /* Number of cores the oracle uses when params.threads == 0. */
 int s3r_ref_hardware_threads(void);
@@ -57,8 +74,9 @@ int s3r_ref_hardware_threads(void);
 /* Round a double to the nearest bfloat16 value (ties to even), returned as a double. */
 double s3r_ref_round_bf16(double x);
 
-/* Compression branch, step 1: block means of x over the valid tokens of each block.
- * out[j,h,c] = (1/n_j) sum_{t in block j, t < L} x[t,h,c], n_j = number of valid tokens. */
+/* Compression branch, step 1: block means of x over the tokens of each block.
+ * out[j,h,c] = (1/n_j) sum_{t in block j} x[t,h,c], n_j = number of tokens of block j (1-D: the
+ * tokens below L). */
 int s3r_ref_pool(const s3r_ref_params* p, const uint16_t* x, double* out);
 
 /* Compression branch, step 2: attention of each chosen query row to all nb block summaries,

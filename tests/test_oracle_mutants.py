@@ -18,7 +18,7 @@ SRC = os.path.join(ROOT, "oracle", "s3r_oracle.c")
 
 MUTANTS = {
     "pool_divides_by_block_size": (
-        "double n = (double)(t1 - t0);", "double n = (double)p->block;"),
+        "double mean = sum / (double)n;", "double mean = sum / (double)p->block;"),
     "pool_skips_bf16_rounding": (
         "p->exact_pool ? mean : s3r_ref_round_bf16(mean)", "mean"),
     "lse_drops_the_max": (
@@ -57,6 +57,13 @@ MUTANTS = {
     "topk_forced_list_not_opened": (
         "for (int32_t f = 0; f < c->forced; ++f) out[f] = f;",
         "for (int32_t f = 0; f < c->forced; ++f) out[f] = c->forced;"),
+    "window_spills_past_grid_edge": (
+        "c < (wc + 1) * win_w && c < p->grid_w; ++c)", "c < (wc + 1) * win_w; ++c)"),
+    "window_forgets_special_offset": (
+        "out[n++] = first + p->special + r * p->grid_w + c;", "out[n++] = first + r * p->grid_w + c;"),
+    "window_index_ignores_special_block": ("    m -= 1;\n", "\n"),
+    "window_rows_use_grid_width": (
+        "const int64_t wr = m / cols, wc = m % cols;", "const int64_t wr = m / p->grid_w, wc = m % cols;"),
     "sel_list_skips_forced_blocks": (
         "const int32_t n_list = p->forced + p->topk;", "const int32_t n_list = p->topk;"),
 }

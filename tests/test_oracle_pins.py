@@ -556,3 +556,138 @@ def test_scale_applies_to_both_branches():
     # and the scale matters: a different scale changes the compressed output
     e = O.sparse_attn(O.Problem(L, H, d, b, k, scale=0.6), q, kk, v, gates)
     assert np.abs(e.o_cmp - a.o_cmp).max() > 1e-6
+
+
+# --------------------------------------------------------------------------------------------
+# 2-D windows on each view's patch grid
+# --------------------------------------------------------------------------------------------
+
+def _geo(N, special, gh, gw, b, win_h, H=2, k=3, forced=0):
+    P = special + gh * gw
+    return O.Problem(N * P, H, 64, b, k, forced=forced, grid_h=gh, grid_w=gw, special=special,
+                     win_h=win_h)
+
+
+def test_2d_blocks_partition_each_view_into_rectangles():
+    """Every token lies in exactly one key block; a block never spans two views; the special
+    tokens of a view form one block; every other block is a rectangle of at most win_h x win_w
+    patches whose sides are cut only by the grid's right and bottom edges."""
+    for N, special, gh, gw, b, wh in [(3, 5, 37, 37, 64, 8), (2, 0, 10, 13, 32, 4),
+                                      (2, 3, 9, 17, 128, 8), (1, 1, 5, 5, 32, 1)]:
+        pb = _geo(N, special, gh, gw, b, wh)
+        P, ww = special + gh * gw, b // wh
+        seen = np.zeros(pb.L, np.int64)
+        for j in range(pb.nb):
+            t = pb.block_tokens(j)
+            assert 0 < t.size <= b and np.all(np.diff(t) > 0)
+            seen[t] += 1
+            view = t // P
+            assert np.all(view == view[0])
+            off = t - view[0] * P
+            if off[0] < special:
+                np.testing.assert_array_equal(off, np.arange(special))
+                continue
+            r, c = (off - special) // gw, (off - special) % gw
+            rows, cols = np.unique(r), np.unique(c)
+            assert rows.size * cols.size == t.size  # a full rectangle of patches
+            assert np.all(np.diff(rows) == 1) and np.all(np.diff(cols) == 1)
+            assert rows[0] % wh == 0 and cols[0] % ww == 0
+            assert rows.size == min(wh, gh - rows[0]) and cols.size == min(ww, gw - cols[0])
+        assert np.all(seen == 1)
+
+
+def test_2d_windows_of_one_patch_row_equal_1d_blocks():
+    """Windows one patch high and b wide on a grid b-multiple wide, with no special tokens, are
+    exactly the 1-D blocks of b consecutive tokens: the whole path must agree bit for bit."""
+    N, gh, gw, b, k = 2, 6, 128, 64, 3
+    pb2 = _geo(N, 0, gh, gw, b, 1, k=k)
+    pb1 = O.Problem(pb2.L, 2, 64, b, k)
+    assert pb2.nb == pb1.nb
+    q, kk, v = (rand_bits((pb2.L, 2, 64), s, 0.7) for s in (91, 92, 93))
+    g = _gates(pb2.L, 2, 94)
+    a, c = O.sparse_attn(pb2, q, kk, v, g), O.sparse_attn(pb1, q, kk, v, g)
+    for name in ("kc", "vc", "lse", "o_cmp", "scores", "idx", "o_sel", "out"):
+        np.testing.assert_array_equal(getattr(a, name), getattr(c, name), err_msg=name)
+
+
+def test_2d_pooling_of_a_ramp_is_the_ramp_at_the_window_centre():
+    """K = alpha*row + beta*col + e over the patches and a constant over the special tokens: the
+    mean over a (possibly cut) window is the ramp at the mean row and mean column of its patches,
+    computed here from the window corners alone."""
+    N, special, gh, gw, b, wh = 2, 4, 11, 13, 32, 4
+    ww = b // wh
+    pb = _geo(N, special, gh, gw, b, wh, H=1)
+    P = special + gh * gw
+    x = np.zeros((pb.L, 1, 64))
+    e = (np.arange(64) % 4) / 2.0  # every value below is a multiple of 1/2 under 32: exact in bf16
+    for view in range(N):
+        x[view * P:view * P + special, 0, :] = 3.0 + e
+        for r in range(gh):
+            for c in range(gw):
+                x[view * P + special + r * gw + c, 0, :] = 2.0 * r + 0.5 * c + e
+    got = O.pool(pb, bits_of(x), exact=True)
+    per_view = 1 + (-(-gh // wh)) * (-(-gw // ww))
+    for j in range(pb.nb):
+        m = j % per_view
+        if m == 0:
+            np.testing.assert_array_equal(got[j, 0], 3.0 + e)
+            continue
+        wr, wc = divmod(m - 1, -(-gw // ww))
+        r0, r1 = wr * wh, min(gh, wr * wh + wh) - 1
+        c0, c1 = wc * ww, min(gw, wc * ww + ww) - 1
+        want = 2.0 * (r0 + r1) / 2 + 0.5 * (c0 + c1) / 2 + e
+        np.testing.assert_allclose(got[j, 0], want, rtol=0, atol=1e-12)
+
+
+def test_2d_selection_matches_library_attention_under_window_mask():
+    """Selection over windows, cut edge windows and special blocks included: SDPA with a boolean
+    mask admitting exactly the selected windows' tokens for the rows of each query block."""
+    pb = _geo(2, 5, 9, 11, 32, 4, H=2, k=4)
+    q, kk, v = (rand_bits((pb.L, 2, 64), s, 1.0 / 8) for s in (95, 96, 97))
+    rng = np.random.default_rng(7)
+    idx = np.stack([np.stack([rng.permutation(pb.nb)[:pb.topk] for _ in range(pb.nqb)])
+                    for _ in range(2)]).astype(np.int32)
+    o = O.sel_attn(pb, q, kk, v, idx)
+    qv, kv, vv = values_of(q), values_of(kk), values_of(v)
+    for h in range(2):
+        mask = np.zeros((pb.L, pb.L), bool)
+        for i in range(pb.nqb):
+            for j in idx[h, i]:
+                mask[64 * i:64 * i + 64, pb.block_tokens(int(j))] = True
+        want = sdpa64(qv[:, h:h + 1], kv[:, h:h + 1], vv[:, h:h + 1], pb.softmax_scale,
+                      mask[None, None])
+        np.testing.assert_allclose(o[:, h:h + 1], want, rtol=0, atol=1e-13)
+
+
+def test_2d_invariance_patches_permuted_within_windows():
+    """Re-ordering the patches inside every window (K and V together) changes nothing but the
+    summation order of the pooled means."""
+    pb = _geo(2, 5, 9, 11, 32, 4, H=2, k=4)
+    q, kk, v = (rand_bits((pb.L, 2, 64), s, 0.7) for s in (98, 99, 100))
+    g = _gates(pb.L, 2, 101)
+    perm = np.arange(pb.L)
+    rng = np.random.default_rng(3)
+    for j in range(pb.nb):
+        t = pb.block_tokens(j)
+        perm[t] = rng.permutation(t)
+    a = O.sparse_attn(pb, q, kk, v, g)
+    b_ = O.sparse_attn(pb, q, kk[perm], v[perm], g)
+    np.testing.assert_allclose(a.kc, b_.kc, atol=1e-2 * np.abs(a.kc).max())
+    np.testing.assert_allclose(a.scores, b_.scores, rtol=1e-5, atol=1e-9)
+    np.testing.assert_allclose(a.out, b_.out, rtol=1e-3, atol=1e-5)
+
+
+def test_2d_reference_view_forced_covers_every_token_of_view_zero():
+    """VGGT variant on windows: forcing the first view's blocks (its special block and all its
+    windows) puts every token of view 0, and no token of another view, among the forced tokens."""
+    N, special, gh, gw, b, wh = 3, 5, 9, 11, 32, 4
+    pb0 = _geo(N, special, gh, gw, b, wh)
+    per_view = pb0.nb // N
+    pb = _geo(N, special, gh, gw, b, wh, k=3, forced=per_view)
+    P = special + gh * gw
+    q, kk, v = (rand_bits((pb.L, 2, 64), s, 0.7) for s in (102, 103, 104))
+    res = O.sparse_attn(pb, q, kk, v, _gates(pb.L, 2, 105))
+    toks = np.concatenate([pb.block_tokens(j) for j in range(per_view)])
+    np.testing.assert_array_equal(np.sort(toks), np.arange(P))
+    assert (res.idx[..., :per_view] == np.arange(per_view)).all()
+    assert (res.idx[..., per_view:] >= per_view).all()
