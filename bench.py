@@ -44,6 +44,13 @@ WORKLOADS = {
                    L=43968, H=16, block=64, topk=16, seed=1),
     "tiny": dict(desc="tiny: N=4 x P=256, L=1024, H=2, d=64, b=64, top-k=4",
                  L=1024, H=2, block=64, topk=4, seed=0),
+    # the same 1000 views with key blocks as 2-D windows: each view's 5 camera/register tokens,
+    # then 8 x 8 windows of its 37 x 37 patch grid (26 blocks a view, 26,000 in all)
+    "n1000_windows": dict(desc="1000-view sequence with 2-D key windows: N=1000 x P=1374 "
+                               "(5 special tokens + 37x37 patches), 8x8-patch windows, L=1,374,000, "
+                               "H=16, d=64, b=64, top-k=32, 1 layer",
+                          L=1374000, H=16, block=64, topk=32, seed=3,
+                          geo=dict(grid_h=37, grid_w=37, special=5, win_h=8)),
 }
 
 METRIC = "sparse global-attn tokens/s at 1000 views"
@@ -106,8 +113,8 @@ def algorithmic(cfg):
     """Algorithmic work per call: FLOPs of Q.Kc^T + P.Vc (once) and of the selection's
     Q.K^T + P.V over the tokens actually selected; bytes of each stage's compulsory traffic."""
     L, H, d, b, k, nb, nqb = cfg.L, cfg.H, cfg.d, cfg.block, cfg.topk, cfg.nb, cfg.nqb
-    # tokens selected per query block: k full blocks, except that the ragged last block (if it is
-    # selected) is shorter; count it as a full block less the tail (upper bound when unselected)
+    # tokens selected per query block: k blocks of b (an upper bound: the ragged last 1-D block,
+    # and 2-D windows cut at a grid edge or a view's special-token block, hold fewer)
     sel_tokens = k * b
     cmp_flops = 4.0 * L * nb * d * H
     sel_flops = 4.0 * L * sel_tokens * d * H
@@ -220,7 +227,8 @@ def oracle_sample(cfg, host_bits, gates_np, n_blocks: int, seed: int):
 
     from oracle import oracle as O
 
-    pb = O.Problem(cfg.L, cfg.H, cfg.d, cfg.block, cfg.topk)
+    pb = O.Problem(cfg.L, cfg.H, cfg.d, cfg.block, cfg.topk, forced=cfg.forced, grid_h=cfg.grid_h,
+                   grid_w=cfg.grid_w, special=cfg.special, win_h=cfg.win_h)
     rng = np.random.default_rng(seed)
     blocks = sorted(set(rng.choice(cfg.nqb - 1, size=max(0, min(n_blocks, cfg.nqb) - 1),
                                    replace=False).tolist()
@@ -250,7 +258,7 @@ def run_reference(args, wl):
     from oracle import oracle as O
     from sparse_global_attention_s3r_b200 import api, synth
 
-    cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"])
+    cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"], **wl.get("geo", {}))
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     x = synth.make_inputs(cfg.L, cfg.H, cfg.d, cfg.block, wl["seed"], device=dev)
     bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
@@ -272,7 +280,8 @@ def run_reference(args, wl):
         "ms_per_step": 1e3 * cfg.L / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl["desc"], "L": cfg.L, "H": cfg.H, "d": cfg.d,
-                   "block": cfg.block, "topk": cfg.topk, "qblock": 64, "seed": wl["seed"]},
+                   "block": cfg.block, "topk": cfg.topk, "qblock": 64, "seed": wl["seed"],
+                   **wl.get("geo", {})},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": desc + f"; median of {args.steps} samples of "
                                           f"{statistics.median(secs):.1f} s"},
@@ -304,7 +313,7 @@ def run_native(args, wl):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
 
-    cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"])
+    cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"], **wl.get("geo", {}))
     seed = rank_seed(wl["seed"], rank)  # an independent layer per GPU
     x = synth.make_inputs(cfg.L, cfg.H, cfg.d, cfg.block, seed, device=dev)
     q, k, v, gates = x.q, x.k, x.v, x.gates
@@ -336,23 +345,28 @@ def run_native(args, wl):
     ms_max = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
     stage_ms = {n: statistics.mean(e.stage_ms()[n] for e in stage_ev) for n in _lib.STAGES}
 
-    # end to end through pinned host buffers: H2D of the step's inputs, the call, D2H of out
+    # end to end through the public API from pinned host memory: every step copies all of its
+    # inputs in and its output out. HostPipeline overlaps the copy-in of step i+1 and the
+    # copy-out of step i-1 with the kernels of step i (two sets of device buffers, two copy
+    # streams); the timed region runs from before the first copy-in to after the last copy-out.
     host = [t_.cpu().pin_memory() for t_ in (q, k, v, gates)]
-    out_h = torch.empty(sa.out.shape, dtype=sa.out.dtype).pin_memory()
-    e2e_steps = max(1, min(args.steps, 3))
-    sa.from_host(*host, out_h)
-    torch.cuda.synchronize()
+    outs_h = [torch.empty(sa.out.shape, dtype=sa.out.dtype).pin_memory() for _ in range(2)]
+    del sa
+    pipe = api.HostPipeline(cfg, dev)
+    e2e_steps = max(2, args.steps)
+    pipe.submit(*host, outs_h[0])
+    pipe.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(e2e_steps):
-        sa.from_host(*host, out_h)
-    e1.record()
-    torch.cuda.synchronize()
+    for s_ in range(e2e_steps):
+        pipe.submit(*host, outs_h[s_ % 2], after=e0 if s_ == 0 else None)
+    e1.record(pipe.copy_out)
+    pipe.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
     h2d = sum(t_.numel() * t_.element_size() for t_ in host)
-    d2h = out_h.numel() * out_h.element_size()
-    del host, out_h
+    d2h = outs_h[0].numel() * outs_h[0].element_size()
+    del host, outs_h, pipe
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -412,7 +426,7 @@ def run_native(args, wl):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": wl["desc"], "L": cfg.L, "H": cfg.H, "d": cfg.d, "block": cfg.block,
-                   "topk": cfg.topk, "qblock": 64, "seed": wl["seed"],
+                   "topk": cfg.topk, "qblock": 64, "seed": wl["seed"], **wl.get("geo", {}),
                    "parallelism": "independent layer per GPU" if world > 1 else "single GPU",
                    "l2": "inputs exceed L2 (each of Q/K/V is %.2f GB > 126 MB); no flush" %
                          (q.numel() * 2 / 1e9)},
@@ -422,7 +436,10 @@ def run_native(args, wl):
         "stage_ms": stages,
         "roofline": roof,
         "e2e": {"value": cfg.L * world / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "steps": e2e_steps,
+                "how": "HostPipeline: pinned host inputs copied in and outputs copied out every "
+                       "step, overlapped with the neighbouring steps' kernels"},
         "cpu_baseline": cpu,
         "gpu_launches": launches,
         "clocks": clocks.summary(),

@@ -90,7 +90,17 @@ typedef struct {
   int32_t forced; /* F >= 0: key blocks 0 .. F-1 open every selection list without competing,
                      and topk more are chosen among blocks F .. nb-1 (topk <= nb - F). The VGGT
                      variant keeps the reference frame's tokens for every query ("Methodologie"
-                     §3): with P tokens per view, F = ceil(P / b). 0 = plain top-k. */
+                     §3): with P tokens per view, F = ceil(P / b) (with 2-D windows: the
+                     number of blocks of one view). 0 = plain top-k. */
+  /* Key-block geometry. grid_h = 0: 1-D blocks, block j = tokens [j*b, min((j+1)*b, L)).
+     grid_h > 0: 2-D windows on each view's patch grid ("Methodologie" §1: the compression branch
+     downsamples spatially). The sequence is N = L / P views of P = special + grid_h * grid_w
+     tokens: `special` leading tokens (camera, register), then the patches row by row. Each view
+     contributes one block of its special tokens (if special > 0), then the windows of
+     win_h x (b / win_h) patches tiling its grid from the top-left, row by row, cut at the
+     right and bottom edges. Blocks are numbered view by view; query blocks stay 64 consecutive
+     tokens. Requires 1 <= win_h, b % win_h == 0, 0 <= special <= b, L % P == 0. */
+  int32_t grid_h, grid_w, special, win_h;
   uint32_t* dev_status; /* optional device word that receives S3R_DEV_* bits (may be NULL) */
   void* const* stage_events; /* optional: S3R_NUM_STAGES + 1 cudaEvent_t handles that
                                 s3r_sparse_attn_fwd records on `stream` at the stage boundaries
@@ -117,6 +127,9 @@ int s3r_version(void);
 
 /* Number of kernels this process has launched through the library so far (monotonic). */
 uint64_t s3r_kernel_launches(void);
+
+/* Number of key blocks nb of the geometry in params (0 if params are invalid). */
+int64_t s3r_num_key_blocks(const s3r_params* params);
 
 /* Bytes of device workspace s3r_sparse_attn_fwd needs for these sizes (0 if params invalid). */
 size_t s3r_workspace_bytes(const s3r_params* params);
@@ -161,7 +174,9 @@ s3r_status s3r_topk_blocks(const s3r_params* params, const float* scores, int32_
  *   q, k, v [L, H, d] bf16 (read); idx [H, nqb, forced + topk] int32 (read): distinct block
  *           indices in [0, nb) per row (entries outside that range are skipped; with
  *           S3R_FLAG_DEBUG_CHECKS they also raise S3R_DEV_BAD_INDEX)
- *   o_sel   [L, H, d] fp32 (written) */
+ *   o_sel   [L, H, d] fp32 (written)
+ *   With 2-D windows narrower than 8 patches (b / win_h < 8) this entry point returns
+ *   S3R_ERR_UNSUPPORTED; s3r_sparse_attn_fwd takes them. */
 s3r_status s3r_sel_attn(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,
                         const s3r_bf16* v, const int32_t* idx, float* o_sel, s3r_stream stream);
 

@@ -33,6 +33,7 @@ EXPORTS = {
     "s3r_version": (ctypes.c_int, []),
     "s3r_kernel_launches": (ctypes.c_uint64, []),
     "s3r_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "s3r_num_key_blocks": (ctypes.c_int64, [_P]),
     "s3r_read_device_status": (ctypes.c_int, [_P, _P, _P]),
     "s3r_workspace_status_word": (_P, [_P]),
     "s3r_compress_kv": (ctypes.c_int, [_P, _P, _P, _P, _P, _P]),
@@ -58,6 +59,10 @@ class Params(ctypes.Structure):
         ("scale", ctypes.c_float),
         ("flags", ctypes.c_uint32),
         ("forced", ctypes.c_int32),
+        ("grid_h", ctypes.c_int32),
+        ("grid_w", ctypes.c_int32),
+        ("special", ctypes.c_int32),
+        ("win_h", ctypes.c_int32),
         ("dev_status", ctypes.c_void_p),
         ("stage_events", ctypes.c_void_p),
     ]

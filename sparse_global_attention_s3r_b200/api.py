@@ -27,7 +27,10 @@ class Config:
     """Sizes of one call: L tokens (N views x P tokens), H heads, d, block size b, top-k.
 
     forced: leading key blocks kept in every selection list (VGGT's reference frame: with P
-    tokens per view, ceil(P / b)); the top-k then picks topk more among the other blocks."""
+    tokens per view, ceil(P / b)); the top-k then picks topk more among the other blocks.
+    grid_h, grid_w, special, win_h: 2-D windows (grid_h > 0). The sequence is L / P views of
+    P = special + grid_h * grid_w tokens; key blocks are each view's special tokens, then
+    win_h x (block / win_h) windows of its patch grid."""
 
     L: int
     H: int
@@ -38,6 +41,10 @@ class Config:
     debug_checks: bool = False
     test_timeout: bool = False  # testing only: exercise the bounded-wait timeout path
     forced: int = 0
+    grid_h: int = 0
+    grid_w: int = 0
+    special: int = 0
+    win_h: int = 0
 
     @property
     def nsel(self) -> int:
@@ -46,7 +53,8 @@ class Config:
 
     @property
     def nb(self) -> int:
-        return -(-self.L // self.block)
+        """Key blocks, as the library counts them (0 for invalid sizes)."""
+        return int(_lib.load().s3r_num_key_blocks(ctypes.byref(self.params())))
 
     @property
     def nqb(self) -> int:
@@ -57,7 +65,7 @@ class Config:
                            0.0 if self.scale is None else float(self.scale),
                            (_lib.S3R_FLAG_DEBUG_CHECKS if self.debug_checks else 0)
                            | (_lib.S3R_FLAG_TEST_TIMEOUT if self.test_timeout else 0),
-                           self.forced,
+                           self.forced, self.grid_h, self.grid_w, self.special, self.win_h,
                            None if dev_status is None else dev_status.data_ptr(),
                            None if stage_events is None else ctypes.addressof(stage_events))
 
@@ -247,3 +255,61 @@ class SparseAttention:
         self(*self._dev_in)
         out_host.copy_(self.out, non_blocking=True)
         return out_host
+
+
+class HostPipeline:
+    """The fused path over a stream of independent steps whose inputs live in pinned host memory.
+
+    ``submit`` enqueues one step: its inputs are copied in on a copy-in stream, the path runs on
+    the caller's current stream, and the output is copied back on a copy-out stream. Two sets of
+    device inputs and outputs alternate, so the copy-in of step i+1 and the copy-out of step i-1
+    overlap the kernels of step i; each step still moves all of its inputs in and its output out.
+    Everything is asynchronous: ``synchronize`` waits for every submitted step, after which the
+    host outputs may be read. A host output buffer must not be reused before that.
+    """
+
+    def __init__(self, cfg: Config, device=None):
+        self.cfg = cfg
+        self.device = torch.device(device or "cuda")
+        self.workspace = alloc_workspace(cfg, self.device)
+        self.idx = torch.empty((cfg.H, cfg.nqb, cfg.nsel), dtype=torch.int32, device=self.device)
+        lhd = _lhd(cfg)
+        self.ins = [[torch.empty(lhd, dtype=torch.bfloat16, device=self.device) for _ in range(3)]
+                    + [torch.empty((cfg.L, cfg.H, 2), dtype=torch.float32, device=self.device)]
+                    for _ in range(2)]
+        self.outs = [torch.empty(lhd, dtype=torch.bfloat16, device=self.device) for _ in range(2)]
+        self.copy_in = torch.cuda.Stream(self.device)
+        self.copy_out = torch.cuda.Stream(self.device)
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of the slot are on device
+        self.ev_done = [torch.cuda.Event() for _ in range(2)]  # the slot's kernels have finished
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]   # the slot's output is on the host
+        self.steps = 0
+
+    def submit(self, q, k, v, gates, out_host: torch.Tensor, after: torch.cuda.Event = None):
+        """Enqueue one step (q, k, v bf16 and gates fp32, pinned host tensors) writing out_host.
+        ``after``: an event the copy-in of this step waits for (e.g. a timing start)."""
+        i = self.steps % 2
+        compute = torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(self.copy_in):
+            if after is not None:
+                self.copy_in.wait_event(after)
+            if self.steps >= 2:  # step n-2 has finished reading this slot's inputs
+                self.copy_in.wait_event(self.ev_done[i])
+            for dst, src in zip(self.ins[i], (q, k, v, gates)):
+                dst.copy_(src, non_blocking=True)
+            self.ev_in[i].record(self.copy_in)
+        compute.wait_event(self.ev_in[i])
+        if self.steps >= 2:  # step n-2's output has left this slot
+            compute.wait_event(self.ev_out[i])
+        sparse_attn_fwd(self.cfg, *self.ins[i], self.workspace, self.outs[i], self.idx)
+        self.ev_done[i].record(compute)
+        with torch.cuda.stream(self.copy_out):
+            self.copy_out.wait_event(self.ev_done[i])
+            out_host.copy_(self.outs[i], non_blocking=True)
+            self.ev_out[i].record(self.copy_out)
+        self.steps += 1
+        return out_host
+
+    def synchronize(self) -> None:
+        self.copy_out.synchronize()
+        torch.cuda.current_stream(self.device).synchronize()

@@ -35,7 +35,31 @@ s3r_status derive(const s3r_params* prm, Problem* out) {
   p.k = prm->topk;
   p.F = prm->forced;
   p.nsel = p.F + p.k;
-  p.nb = (p.L + p.b - 1) / p.b;
+  BlockGeo& g = p.geo;
+  g.L = p.L;
+  g.b = p.b;
+  if (prm->grid_h == 0) {
+    p.nb = (p.L + p.b - 1) / p.b;
+  } else {  // 2-D windows: check the geometry, count the blocks of a view
+    if (prm->grid_h < 1 || prm->grid_w < 1 || prm->special < 0 || prm->special > p.b ||
+        prm->win_h < 1 || p.b % prm->win_h != 0)
+      return S3R_ERR_INVALID_ARG;
+    g.two_d = 1;
+    g.special = prm->special;
+    g.gh = prm->grid_h;
+    g.gw = prm->grid_w;
+    g.wh = prm->win_h;
+    const int ww = p.b / g.wh;  // a power of 2, as b is
+    while ((1 << g.lww) < ww) ++g.lww;
+    g.P = static_cast<int64_t>(g.special) + static_cast<int64_t>(g.gh) * g.gw;
+    if (p.L % g.P != 0) return S3R_ERR_INVALID_ARG;
+    g.cols = (g.gw + ww - 1) / ww;
+    const int64_t per_view =
+        (g.special > 0 ? 1 : 0) + static_cast<int64_t>((g.gh + g.wh - 1) / g.wh) * g.cols;
+    if (per_view > S3R_MAX_BLOCKS) return S3R_ERR_UNSUPPORTED;
+    g.per_view = static_cast<int>(per_view);
+    p.nb = (p.L / g.P) * per_view;
+  }
   p.nqb = (p.L + p.qb - 1) / p.qb;
   if (p.nb > S3R_MAX_BLOCKS) return S3R_ERR_UNSUPPORTED;
   if (p.F < 0 || p.k > p.nb - p.F) return S3R_ERR_INVALID_ARG;
@@ -169,6 +193,11 @@ uint64_t s3r_kernel_launches(void) { return g_launches.load(std::memory_order_re
 
 size_t s3r_workspace_bytes(const s3r_params* params) { return fused_workspace_bytes(params); }
 
+int64_t s3r_num_key_blocks(const s3r_params* params) {
+  Problem p;
+  return derive(params, &p) == S3R_OK ? p.nb : 0;
+}
+
 uint32_t* s3r_workspace_status_word(void* workspace) {
   return static_cast<uint32_t*>(workspace);  // the status word is the first region
 }
@@ -222,6 +251,10 @@ s3r_status s3r_sel_attn(const s3r_params* params, const s3r_bf16* q, const s3r_b
   if (st != S3R_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(o_sel))
     return S3R_ERR_INVALID_ARG;
+  // gathered straight from K and V, a window row is one TMA box; a 128-byte-swizzled box must
+  // cover whole 8-row (1024-byte) swizzle atoms, so windows narrower than 8 patches are not
+  // gathered this way (the fused call, which gathers from its slot-ordered copies, takes them)
+  if (p.geo.two_d && (1 << p.geo.lww) < 8) return S3R_ERR_UNSUPPORTED;
   return launched(launch_sel_attn(p, q, k, v, false, idx, o_sel, nullptr, nullptr, nullptr, stream));
 }
 

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "geometry.cuh"
 #include "s3r.h"
 
 namespace s3r {
@@ -15,6 +16,7 @@ struct Problem {
   int k;            // top-k (blocks chosen by score)
   int F;            // leading key blocks kept in every selection list (0 = none)
   int nsel;         // selection list length F + k
+  BlockGeo geo;     // which tokens each key block holds
   int64_t nb, nqb;  // key blocks, query blocks
   float scale;      // softmax scale
   float scale_log2; // scale * log2(e): logits in base-2 units

@@ -71,7 +71,9 @@ struct SelArgs {
   const float* gates;  // [L, H, 2]  fp32 (fused combine)
   uint16_t* out;       // [L, H, 64] bf16 (fused combine)
   int64_t L, nb, nqb;
-  int64_t nb_full;  // key blocks that lie wholly below L
+  BlockGeo geo;      // which tokens each key block holds
+  int box;           // K/V rows per TMA box: a run of consecutive tokens (or copy rows)
+  int head_major;    // K/V are the [H, nb*b, 64] copies in slot order
   int kv_xh, kv_yh;  // K/V box of head h, token tok at (h*kv_xh, h*kv_yh + tok): token-major
                      // [L, H, 64] is (64, 0), the head-major [H, nb*b, 64] copy is (0, nb*b)
   int H, b, lb, topk, nsteps;  // lb = log2(b)
@@ -164,7 +166,7 @@ __global__ void __maxnreg__(128)
       int issued = 0;
       mbar_arrive_expect_tx(&bars->q_full, kQBytes);
       tma_load_2d(sbase + kOffQ, &tmQ, h * 64, static_cast<int32_t>(q0), &bars->q_full);
-      const int box = a.b < kStep ? a.b : kStep;  // rows per TMA box: 32 for b = 32, else 64
+      const int box = a.box;
       for (int t = 0; t < ns; ++t) {
         const int stage = t % kStages;
         if (!mbar_wait(&bars->kv_empty[stage], ((t / kStages) & 1) ^ 1, abort, lim)) {
@@ -176,13 +178,21 @@ __global__ void __maxnreg__(128)
         for (int qb = 0; qb < 2; ++qb) {
           const int32_t* list = list_of[qb];
           for (int part = 0; part < kStep / box; ++part) {
-            // position of this box in the query block's token list, and its first token
+            // position of this box in the query block's slot list: block j, slot o
             const int pos = t * kStep + part * box;
             bool valid;
             const int64_t j = sel_block(list, pos >> a.lb, a.topk, a.nb, valid);
-            const int64_t tok = j * a.b + (pos & (a.b - 1));
+            const int o = pos & (a.b - 1);
+            // the copy's slot row, or the 1-D token (past L reads zeros); a 2-D window's run of
+            // box slots lies in one patch row, so it is box consecutive tokens from its first
+            // (a run whose first slot holds no token holds none: any row will do, it is masked)
+            int64_t row = j * a.b + o;
+            if (!a.head_major && a.geo.two_d) {
+              const int64_t tk = slot_token(a.geo, j, o);
+              row = tk >= 0 ? tk : 0;
+            }
             const uint32_t row_off = (qb * kStep + part * box) * 128;
-            const int32_t x = h * a.kv_xh, y = static_cast<int32_t>(h * a.kv_yh + tok);
+            const int32_t x = h * a.kv_xh, y = static_cast<int32_t>(h * a.kv_yh + row);
             tma_load_2d(sk + row_off, &tmK, x, y, &bars->kv_full[stage]);
             tma_load_2d(sk + kTileBytes + row_off, &tmV, x, y, &bars->kv_full[stage]);
           }
@@ -246,7 +256,7 @@ __global__ void __maxnreg__(128)
     // ------------------------------------------------------------------ softmax warps
     const int g = warp & 3;       // TMEM lane quadrant: rows 32g .. 32g+31
     const int qb = g >> 1;        // which of the two query blocks these rows belong to
-    const int tq = lane & 3, tr = lane >> 2;
+    const int tq = lane & 3;
     const uint32_t tl0 = tbase + (static_cast<uint32_t>(g * 32) << 16);
     const uint32_t tl16 = tbase + (static_cast<uint32_t>(g * 32 + 16) << 16);
     const float sl2 = a.scale_log2;
@@ -295,8 +305,8 @@ __global__ void __maxnreg__(128)
             v[2][c] = __uint_as_float(r[2 * hh + 1][4 * rep + e]);
             v[3][c] = __uint_as_float(r[2 * hh + 1][4 * rep + 2 + e]);
           }
-      // columns whose token does not exist: past k*b, an out-of-range index, or past L. A
-      // 64-token step spans at most two selected blocks (b >= 32).
+      // columns whose slot holds no token: past the list, an out-of-range index, past L, or
+      // outside a view's patch grid. A 64-slot step spans at most two selected blocks (b >= 32).
       {
         const int p0 = t * kStep;
         const int s_lo = p0 >> a.lb, s_hi = (p0 + kStep - 1) >> a.lb;
@@ -306,16 +316,18 @@ __global__ void __maxnreg__(128)
         if ((a.flags & S3R_FLAG_DEBUG_CHECKS) && lane == 0 &&
             ((!ok_lo && s_lo < a.topk) || (!ok_hi && s_hi < a.topk)))
           set_status(a.status, S3R_DEV_BAD_INDEX);
-        // the same for the whole warp; false only on a list's last step or at the partial block
-        const bool all_valid = ok_lo && ok_hi && j_lo < a.nb_full && j_hi < a.nb_full;
+        const BlockOrigin bo_lo = block_origin(a.geo, j_lo), bo_hi = block_origin(a.geo, j_hi);
+        // the same for the whole warp; false only on a list's last step or at a cut block
+        const bool all_valid =
+            ok_lo && ok_hi && origin_full(a.geo, bo_lo) && origin_full(a.geo, bo_hi);
         if (!all_valid) {
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int pos = p0 + col_of(c);
             const bool lo = (pos >> a.lb) == s_lo;
             const bool valid = lo ? ok_lo : ok_hi;
-            const int64_t tok = (lo ? j_lo : j_hi) * a.b + (pos & (a.b - 1));
-            if (!valid || tok >= a.L) v[0][c] = v[1][c] = v[2][c] = v[3][c] = -INFINITY;
+            if (!valid || origin_token(a.geo, lo ? bo_lo : bo_hi, pos & (a.b - 1)) < 0)
+              v[0][c] = v[1][c] = v[2][c] = v[3][c] = -INFINITY;
           }
         }
       }
@@ -478,7 +490,11 @@ cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t*
                             const uint16_t* v, bool head_major, const int32_t* idx, float* o_sel,
                             const float* o_cmp, const float* gates, uint16_t* out,
                             cudaStream_t st) {
-  const int box = p.b < kStep ? p.b : kStep;
+  // rows per K/V box: a run of slots that are consecutive rows in memory (32 for b = 32, else
+  // 64; gathers of 2-D windows from K and V themselves: one window row, at most 64)
+  int box = p.b < kStep ? p.b : kStep;
+  if (!head_major && p.geo.two_d && (1 << p.geo.lww) < box) box = 1 << p.geo.lww;
+  if (box < 8) return cudaErrorInvalidValue;  // whole 1024-byte swizzle atoms only
   const int64_t Lp = p.nb * p.b;
   if (head_major && p.H * Lp > INT32_MAX) return cudaErrorInvalidValue;  // TMA coordinates
   CUtensorMap tq, tk, tv;
@@ -497,7 +513,7 @@ cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t*
   if (e != cudaSuccess) return e;
   const int64_t ntok = static_cast<int64_t>(p.nsel) * p.b;
   const int lb = p.b == 32 ? 5 : p.b == 64 ? 6 : 7;
-  SelArgs a{idx, o_sel, o_cmp, gates, out, p.L, p.nb, p.nqb, p.L / p.b,
+  SelArgs a{idx, o_sel, o_cmp, gates, out, p.L, p.nb, p.nqb, p.geo, box, head_major ? 1 : 0,
             head_major ? 0 : 64, head_major ? static_cast<int>(Lp) : 0, p.H, p.b, lb, p.nsel,
             static_cast<int>((ntok + kStep - 1) / kStep), p.scale_log2, p.flags, p.status,
             (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull};

@@ -24,7 +24,7 @@ def declared_functions():
 def test_library_exports_every_declared_function():
     lib = _lib.load()
     names = declared_functions()
-    assert len(names) == 13, names
+    assert len(names) == 14, names
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_lib.EXPORTS)
@@ -62,6 +62,11 @@ A16_NOT256 = ctypes.c_void_p((1 << 20) + 16)
     (dict(topk=17), _lib.S3R_ERR_INVALID_ARG),  # nb = 16
     (dict(topk=4, forced=13), _lib.S3R_ERR_INVALID_ARG),  # forced + topk > nb
     (dict(forced=-1), _lib.S3R_ERR_INVALID_ARG),
+    # 2-D windows: L must be whole views, win_h must divide b, special must fit one block
+    (dict(L=1001, grid_h=3, grid_w=3, special=1, win_h=2), _lib.S3R_ERR_INVALID_ARG),
+    (dict(L=1020, grid_h=10, grid_w=10, special=2, win_h=3), _lib.S3R_ERR_INVALID_ARG),
+    (dict(L=6 * 166, block=32, grid_h=10, grid_w=10, special=66, win_h=4), _lib.S3R_ERR_INVALID_ARG),
+    (dict(L=1020, grid_h=10, grid_w=-1, special=2, win_h=2), _lib.S3R_ERR_INVALID_ARG),
     (dict(scale=float("nan")), _lib.S3R_ERR_INVALID_ARG),
     (dict(scale=float("inf")), _lib.S3R_ERR_INVALID_ARG),
     (dict(L=_lib.S3R_MAX_BLOCKS * 32 + 1, block=32, topk=1), _lib.S3R_ERR_UNSUPPORTED),
@@ -145,3 +150,24 @@ def test_static_entry_point_rejects_oversized_and_bad_sizes_before_any_launch():
     bad = _params(d=128)
     assert lib.s3r_sparse_attn_fwd_static(ctypes.byref(bad), A16, A16, A16, A16, A16, None,
                                           None) == _lib.S3R_ERR_UNSUPPORTED
+
+
+def test_num_key_blocks_of_the_geometries():
+    lib = _lib.load()
+    # 1-D: ceil(L / b)
+    assert lib.s3r_num_key_blocks(ctypes.byref(_params(L=1000, block=64))) == 16
+    # VGGT layout: 4 views of 5 special tokens + 37 x 37 patches, 8 x 8 windows: 1 + 5 * 5 a view
+    vggt = _params(L=4 * 1374, block=64, grid_h=37, grid_w=37, special=5, win_h=8)
+    assert lib.s3r_num_key_blocks(ctypes.byref(vggt)) == 4 * 26
+    # no special tokens, 4 x 8 windows on 10 x 13: 3 x 2 windows a view
+    assert lib.s3r_num_key_blocks(ctypes.byref(
+        _params(L=2 * 130, block=32, grid_h=10, grid_w=13, special=0, win_h=4))) == 2 * 6
+    assert lib.s3r_num_key_blocks(ctypes.byref(_params(L=0))) == 0
+    cfg = api.Config(L=4 * 1374, H=16, block=64, topk=16, grid_h=37, grid_w=37, special=5, win_h=8)
+    assert cfg.nb == 104
+
+
+def test_sel_attn_rejects_windows_narrower_than_8_before_any_launch():
+    lib = _lib.load()
+    narrow = _params(L=2 * 130, block=32, topk=2, grid_h=10, grid_w=13, special=0, win_h=8)  # 8 x 4
+    assert lib.s3r_sel_attn(ctypes.byref(narrow), A16, A16, A16, A16, A16, None) == _lib.S3R_ERR_UNSUPPORTED

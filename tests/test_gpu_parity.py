@@ -308,3 +308,103 @@ def test_forced_sel_attn(dev, name):
     torch.cuda.synchronize()
     ref = O.sel_attn(pb, O.bf16_bits(x.q), O.bf16_bits(x.k), O.bf16_bits(x.v), idx)
     check_close("o_sel", f64(o), ref, 2.0 ** -8 * np.abs(f64(x.v)).max() + 1e-6, rl2=4e-3)
+
+
+# --------------------------------------------------------------------------------------------
+# 2-D windows on each view's patch grid (special tokens as a block of their own)
+# --------------------------------------------------------------------------------------------
+
+WINDOWS = {  # name: (views, special, grid_h, grid_w, b, win_h, H, k, forced_views, seed)
+    "vggt_4_views_8x8": (4, 5, 37, 37, 64, 8, 2, 16, 0, 30),
+    "vggt_ref_view_forced": (4, 5, 37, 37, 64, 8, 2, 12, 1, 31),
+    "odd_grid_4x8_b32": (3, 3, 10, 13, 32, 4, 2, 5, 0, 32),
+    "wide_8x16_b128": (2, 0, 20, 35, 128, 8, 2, 3, 0, 33),
+    "k_above_32_4x8": (6, 5, 16, 16, 32, 4, 2, 40, 0, 34),
+}
+
+
+def window_inputs(name, device):
+    N, special, gh, gw, b, wh, H, k, fv, seed = WINDOWS[name]
+    L = N * (special + gh * gw)
+    geo = dict(grid_h=gh, grid_w=gw, special=special, win_h=wh)
+    per_view = api.Config(L=L, H=H, block=b, topk=1, **geo).nb // N
+    F = fv * per_view
+    x = synth.make_inputs(L, H, 64, b, seed)
+    cfg = api.Config(L=L, H=H, block=b, topk=k, forced=F, **geo)
+    pb = O.Problem(L, H, 64, b, k, forced=F, **geo)
+    assert cfg.nb == pb.nb
+    d = {n: getattr(x, n).to(device) for n in ("q", "k", "v", "gates")}
+    return cfg, pb, x, d
+
+
+@pytest.mark.parametrize("name", list(WINDOWS))
+def test_windows_compress_kv(dev, name):
+    cfg, pb, x, d = window_inputs(name, dev)
+    kc, vc = api.compress_kv(cfg, d["k"], d["v"])
+    torch.cuda.synchronize()
+    for got, src in ((kc, x.k), (vc, x.v)):
+        exact = check_pooled(f64(got), O.pool(pb, O.bf16_bits(src)))
+        assert exact >= 0.99, exact
+
+
+@pytest.mark.parametrize("name", list(WINDOWS))
+def test_windows_sel_attn_gathers_from_k_and_v(dev, name):
+    """The step entry point gathers window rows straight from K, V [L, H, 64]."""
+    cfg, pb, x, d = window_inputs(name, dev)
+    rng = np.random.default_rng(WINDOWS[name][-1])
+    n = cfg.nsel
+    idx = np.stack([np.stack([rng.permutation(cfg.nb)[:n] for _ in range(cfg.nqb)])
+                    for _ in range(cfg.H)]).astype(np.int32)
+    o = api.sel_attn(cfg, d["q"], d["k"], d["v"], torch.from_numpy(idx).to(dev))
+    torch.cuda.synchronize()
+    ref = O.sel_attn(pb, O.bf16_bits(x.q), O.bf16_bits(x.k), O.bf16_bits(x.v), idx)
+    check_close("o_sel", f64(o), ref, 2.0 ** -8 * np.abs(f64(x.v)).max() + 1e-6, rl2=4e-3)
+
+
+@pytest.mark.parametrize("name", list(WINDOWS))
+def test_windows_whole_path(dev, name):
+    cfg, pb, x, d = window_inputs(name, dev)
+    out, idx = _fused(cfg, d)
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    ref = O.sparse_attn(pb, *bits, x.gates.numpy())
+    stats = check_selection(idx, ref.idx, ref.gap, ref.scores, cfg.topk, cfg.forced)
+    cond = O.sparse_attn(pb, *bits, x.gates.numpy(), idx_given=idx, pooled=(ref.kc, ref.vc))
+    check_output(out, cond.out)
+    if stats["sets_equal"] == 1.0:
+        check_output(out, ref.out)
+
+
+def test_windows_one_patch_high_match_1d_blocks_bit_for_bit(dev):
+    """Windows 1 x b on a grid b-multiple wide without special tokens are the 1-D blocks: the
+    fused path must produce identical bits either way."""
+    N, gh, gw, b, k, H = 3, 5, 128, 64, 6, 2
+    L = N * gh * gw
+    x = synth.make_inputs(L, H, 64, b, 35)
+    d = {n: getattr(x, n).to(dev) for n in ("q", "k", "v", "gates")}
+    one = api.Config(L=L, H=H, block=b, topk=k)
+    two = api.Config(L=L, H=H, block=b, topk=k, grid_h=gh, grid_w=gw, special=0, win_h=1)
+    assert one.nb == two.nb
+    o1, i1 = _fused(one, d)
+    o2, i2 = _fused(two, d)
+    np.testing.assert_array_equal(i1, i2)
+    np.testing.assert_array_equal(o1, o2)
+
+
+def test_host_pipeline_matches_device_calls(dev):
+    """Steps submitted from pinned host memory through the overlapped pipeline give the same
+    outputs as device-resident calls, step by step, with every slot reused at least once."""
+    L, H, b, k = 3000, 2, 64, 5
+    cfg = api.Config(L=L, H=H, block=b, topk=k)
+    steps = [synth.make_inputs(L, H, 64, b, 40 + s) for s in range(5)]
+    want = []
+    sa = api.SparseAttention(cfg, dev)
+    for x in steps:
+        want.append(sa(*(getattr(x, n).to(dev) for n in ("q", "k", "v", "gates"))).cpu())
+    pipe = api.HostPipeline(cfg, dev)
+    host_out = [torch.empty((L, H, 64), dtype=torch.bfloat16).pin_memory() for _ in steps]
+    host_in = [[getattr(x, n).pin_memory() for n in ("q", "k", "v", "gates")] for x in steps]
+    for ins, o in zip(host_in, host_out):
+        pipe.submit(*ins, o)
+    pipe.synchronize()
+    for got, ref in zip(host_out, want):
+        assert torch.equal(got, ref)
