@@ -447,17 +447,79 @@ def run_native(args, wl):
     print(json.dumps(line), flush=True)
 
 
+# the pi^3-like sweep at N = 200 views (L = 274,800, H = 16): each (b, top-k) setting is a stack of
+# 24 layers with independent seeded inputs, generated before the timed region
+SWEEP = dict(L=274800, H=16, layers=24, settings=((32, 32), (64, 16), (128, 8)), seed=4000)
+
+
+def run_sweep(args):
+    """One step = the whole path over all 24 layers of every setting; prints one JSON line with
+    the summed attention time and tokens/s of each setting."""
+    import torch
+
+    from sparse_global_attention_s3r_b200 import _lib, api, synth
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", 0)
+    L, H, layers = SWEEP["L"], SWEEP["H"], SWEEP["layers"]
+    result, total_ms, launches = {}, 0.0, 0
+    with ClockSampler(physical_gpu(0)) as clocks:
+        for b, k in SWEEP["settings"]:
+            cfg = api.Config(L=L, H=H, block=b, topk=k)
+            xs = [synth.make_inputs(L, H, 64, b, SWEEP["seed"] + 100 * b + i, device=dev)
+                  for i in range(layers)]
+            sa = api.SparseAttention(cfg, dev)
+            for _ in range(args.warmup):
+                for x in xs:
+                    sa(x.q, x.k, x.v, x.gates)
+            torch.cuda.synchronize()
+            n0 = _lib.kernel_launches()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(args.steps):
+                for x in xs:
+                    sa(x.q, x.k, x.v, x.gates)
+            e1.record()
+            torch.cuda.synchronize()
+            launches += _lib.kernel_launches() - n0
+            ms = e0.elapsed_time(e1) / args.steps  # one pass over the 24-layer stack
+            total_ms += ms
+            result[f"b{b}_k{k}"] = {"ms_24_layers": ms, "ms_per_layer": ms / layers,
+                                    "tokens_per_s": layers * L / (ms / 1e3), "nb": cfg.nb}
+            del xs, sa
+            torch.cuda.empty_cache()
+    n_settings = len(SWEEP["settings"])
+    line = {
+        "metric": "sparse global-attn tokens/s, pi3-like sweep at 200 views (24 layers per setting)",
+        "value": n_settings * layers * L / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "pi3-like sweep: N=200 views, L=274,800, H=16, d=64, "
+                               "(b, top-k) in {(32,32), (64,16), (128,8)}, 24 layers each",
+                   "L": L, "H": H, "layers": layers,
+                   "l2": "each layer's Q/K/V (563 MB each) exceed L2; no flush"},
+        "sweep": result, "gpu_launches": launches, "clocks": clocks.summary(),
+    }
+    print(json.dumps(line))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="n1000")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["pi3_sweep"], default="n1000")
     ap.add_argument("--oracle-blocks", type=int, default=8,
                     help="query blocks in the timed CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.workload == "pi3_sweep":
+        if args.impl == "reference":
+            raise SystemExit("--impl reference times the oracle on the single-layer workloads")
+        return run_sweep(args)
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, wl)
