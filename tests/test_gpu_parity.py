@@ -320,6 +320,9 @@ WINDOWS = {  # name: (views, special, grid_h, grid_w, b, win_h, H, k, forced_vie
     "odd_grid_4x8_b32": (3, 3, 10, 13, 32, 4, 2, 5, 0, 32),
     "wide_8x16_b128": (2, 0, 20, 35, 128, 8, 2, 3, 0, 33),
     "k_above_32_4x8": (6, 5, 16, 16, 32, 4, 2, 40, 0, 34),
+    "one_view_grid_smaller_than_window": (1, 2, 3, 5, 64, 8, 2, 1, 0, 36),
+    "special_fills_a_block": (3, 32, 6, 9, 32, 4, 2, 4, 0, 37),
+    "forced_views_k_above_32": (5, 5, 16, 16, 32, 4, 2, 36, 1, 38),
 }
 
 
