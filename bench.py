@@ -368,6 +368,38 @@ def run_native(args, wl):
     d2h = outs_h[0].numel() * outs_h[0].element_size()
     del host, outs_h, pipe
 
+    # context, not a target: dense attention on the same Q, K, V (torch's SDPA, the library's
+    # flash kernel) for a seeded sample of query rows against all L keys, extrapolated linearly
+    # in the rows (each row's attention is independent of the others)
+    dense = None
+    if rank == 0 and not args.no_dense_context:
+        import torch.nn.functional as F
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+
+        rows = min(cfg.L, args.dense_rows)
+        r0 = int(torch.randint(0, cfg.L - rows + 1, (1,), generator=torch.Generator().manual_seed(5)))
+        qh = q[r0:r0 + rows].permute(1, 0, 2).unsqueeze(0)  # [1, H, rows, d] views
+        kh_, vh_ = k.permute(1, 0, 2).unsqueeze(0), v.permute(1, 0, 2).unsqueeze(0)
+        try:
+            # the flash kernel only: a fallback would materialise rows x L logits
+            with sdpa_kernel(SDPBackend.FLASH_ATTENTION):
+                for _ in range(2):
+                    F.scaled_dot_product_attention(qh, kh_, vh_)
+                torch.cuda.synchronize()
+                d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                d0.record()
+                F.scaled_dot_product_attention(qh, kh_, vh_)
+                d1.record()
+                torch.cuda.synchronize()
+            dense_ms = d0.elapsed_time(d1) * cfg.L / rows
+            dense = {"ms_per_layer": dense_ms, "sparse_speedup": dense_ms / ms_max,
+                     "tflops": 4.0 * cfg.L * cfg.L * cfg.d * cfg.H / (dense_ms / 1e3) / 1e12,
+                     "how": f"torch SDPA (flash) on {rows} seeded query rows x all {cfg.L} keys, "
+                            f"all {cfg.H} heads, extrapolated to {cfg.L} rows"}
+        except RuntimeError as e:
+            dense = {"unavailable": str(e).splitlines()[0][:200]}
+        del qh, kh_, vh_
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import oracle as O
@@ -442,6 +474,7 @@ def run_native(args, wl):
                        "step, overlapped with the neighbouring steps' kernels"},
         "cpu_baseline": cpu,
         "gpu_launches": launches,
+        "dense_context": dense,
         "clocks": clocks.summary(),
     }
     print(json.dumps(line), flush=True)
@@ -515,6 +548,10 @@ def main():
     ap.add_argument("--oracle-blocks", type=int, default=8,
                     help="query blocks in the timed CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense-context", action="store_true",
+                    help="skip timing dense attention (torch SDPA) on a sample of query rows")
+    ap.add_argument("--dense-rows", type=int, default=16384,
+                    help="query rows of the dense-attention context sample")
     args = ap.parse_args()
     if args.workload == "pi3_sweep":
         if args.impl == "reference":

@@ -79,4 +79,33 @@ __host__ __device__ __forceinline__ bool block_full(const BlockGeo& g, int64_t j
   return origin_full(g, block_origin(g, j));
 }
 
+// Bits of the slots o0 .. o0+n-1 (n <= 64) of the block that starts at bo: bit i set when slot
+// o0 + i holds a token. A window contributes, for each of its patch rows that lies in the grid,
+// the run of its first cv slots (cv = columns of the window inside the grid).
+__host__ __device__ __forceinline__ uint64_t range_bits(int lo, int hi) {  // bits lo .. hi-1
+  if (hi <= lo) return 0ull;
+  const uint64_t upto_hi = hi >= 64 ? ~0ull : ((1ull << hi) - 1ull);
+  const uint64_t below_lo = (1ull << lo) - 1ull;
+  return upto_hi & ~below_lo;
+}
+
+__host__ __device__ __forceinline__ uint64_t slot_bits(const BlockGeo& g, const BlockOrigin& bo,
+                                                       int o0, int n) {
+  if (bo.kind == 0) {  // tokens first .. L-1 of the run
+    const int64_t cnt = g.L - bo.first - o0;
+    return range_bits(0, cnt < 0 ? 0 : (cnt > n ? n : static_cast<int>(cnt)));
+  }
+  if (bo.kind == 1) return range_bits(0, g.special - o0 > n ? n : g.special - o0);
+  const int ww = 1 << g.lww;
+  const int rv = g.gh - bo.r0 < g.wh ? g.gh - bo.r0 : g.wh;  // window rows inside the grid
+  const int cv = g.gw - bo.c0 < ww ? g.gw - bo.c0 : ww;      // window columns inside the grid
+  uint64_t bits = 0ull;
+  for (int r = o0 >> g.lww; r < rv && (r << g.lww) < o0 + n; ++r) {
+    const int lo = (r << g.lww) > o0 ? (r << g.lww) : o0;
+    const int hi = (r << g.lww) + cv < o0 + n ? (r << g.lww) + cv : o0 + n;
+    bits |= range_bits(lo - o0, hi - o0);
+  }
+  return bits;
+}
+
 }  // namespace s3r

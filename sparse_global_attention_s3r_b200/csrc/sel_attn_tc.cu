@@ -321,14 +321,18 @@ __global__ void __maxnreg__(128)
         const bool all_valid =
             ok_lo && ok_hi && origin_full(a.geo, bo_lo) && origin_full(a.geo, bo_hi);
         if (!all_valid) {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int pos = p0 + col_of(c);
-            const bool lo = (pos >> a.lb) == s_lo;
-            const bool valid = lo ? ok_lo : ok_hi;
-            if (!valid || origin_token(a.geo, lo ? bo_lo : bo_hi, pos & (a.b - 1)) < 0)
-              v[0][c] = v[1][c] = v[2][c] = v[3][c] = -INFINITY;
+          // bit p: slot p0 + p of the list holds a token (b >= 64: one block covers the step;
+          // b = 32: two blocks, 32 slots each)
+          uint64_t bits;
+          if (a.b >= kStep) {
+            bits = ok_lo ? slot_bits(a.geo, bo_lo, p0 & (a.b - 1), kStep) : 0ull;
+          } else {
+            bits = (ok_lo ? slot_bits(a.geo, bo_lo, 0, 32) : 0ull) |
+                   ((ok_hi ? slot_bits(a.geo, bo_hi, 0, 32) : 0ull) << 32);
           }
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            if (!((bits >> col_of(c)) & 1ull)) v[0][c] = v[1][c] = v[2][c] = v[3][c] = -INFINITY;
         }
       }
       // row maxima of this step (the quad's 4 threads hold the same rows)
