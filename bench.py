@@ -118,17 +118,19 @@ def algorithmic(cfg):
     sel_tokens = k * b
     cmp_flops = 4.0 * L * nb * d * H
     sel_flops = 4.0 * L * sel_tokens * d * H
+    single = getattr(cfg, "single_kernel", False)  # the compressed stage also runs selection
     return {
-        "cmp_exp2": 2.0 * L * nb * H,  # one per (query, summary) pair in each of the two passes
+        # one exp2 per (query, summary) pair in each of the two passes (+ one per selected token)
+        "cmp_exp2": 2.0 * L * nb * H + (L * sel_tokens * H if single else 0.0),
         "cmp_flops": cmp_flops,
         "sel_flops": sel_flops,
         "flops": cmp_flops + sel_flops,
         "stage_work": {
             # K, V read; Kc, Vc and the head-major copies of K, V (nb*b rows) written
             "pool": ("hbm", 2.0 * (L + nb + nb * b) * H * d * 2),              # bytes
-            "cmp": ("tensor", cmp_flops),                                     # flops
+            "cmp": ("tensor", cmp_flops + (sel_flops if single else 0.0)),    # flops
             "topk": ("hbm", H * nqb * (nb * 4.0 + k * 4.0)),                  # bytes
-            "sel_combine": ("tensor", sel_flops),                             # flops
+            "sel_combine": ("tensor", 0.0 if single else sel_flops),          # flops
         },
     }
 
@@ -313,7 +315,8 @@ def run_native(args, wl):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
 
-    cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"], **wl.get("geo", {}))
+    cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"],
+                     single_kernel=args.single_kernel, **wl.get("geo", {}))
     seed = rank_seed(wl["seed"], rank)  # an independent layer per GPU
     x = synth.make_inputs(cfg.L, cfg.H, cfg.d, cfg.block, seed, device=dev)
     q, k, v, gates = x.q, x.k, x.v, x.gates
@@ -459,6 +462,8 @@ def run_native(args, wl):
         "data": "synthetic",
         "config": {"workload": wl["desc"], "L": cfg.L, "H": cfg.H, "d": cfg.d, "block": cfg.block,
                    "topk": cfg.topk, "qblock": 64, "seed": wl["seed"], **wl.get("geo", {}),
+                   "kernels": "pool + one fused kernel" if args.single_kernel else
+                              "pool + compressed/top-k + selection/combine",
                    "parallelism": "independent layer per GPU" if world > 1 else "single GPU",
                    "l2": "inputs exceed L2 (each of Q/K/V is %.2f GB > 126 MB); no flush" %
                          (q.numel() * 2 / 1e9)},
@@ -548,6 +553,8 @@ def main():
     ap.add_argument("--oracle-blocks", type=int, default=8,
                     help="query blocks in the timed CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--single-kernel", action="store_true",
+                    help="run the compressed branch, top-k and selection as one kernel (k <= 32)")
     ap.add_argument("--no-dense-context", action="store_true",
                     help="skip timing dense attention (torch SDPA) on a sample of query rows")
     ap.add_argument("--dense-rows", type=int, default=16384,

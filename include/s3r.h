@@ -74,9 +74,15 @@ typedef enum {
 
 /* params.flags */
 #define S3R_FLAG_DEBUG_CHECKS 0x1u /* validate idx on the device in s3r_sel_attn */
-#define S3R_FLAG_TEST_TIMEOUT 0x2u /* testing only: the compressed-branch kernel waits on a barrier
-                                      that nothing signals, with a 1 ms limit, so the timeout path
-                                      runs: S3R_DEV_TIMEOUT is set and the outputs are invalid */
+#define S3R_FLAG_TEST_TIMEOUT 0x2u /* testing only: the compressed-branch and selection kernels
+                                      wait on a barrier that nothing signals, with a 1 ms limit, so
+                                      their timeout paths run: S3R_DEV_TIMEOUT is set and the
+                                      outputs are invalid */
+#define S3R_FLAG_SINGLE_KERNEL 0x4u /* s3r_sparse_attn_fwd with topk <= 32: after pooling, one
+                                       kernel per (query tile, head) runs the compressed branch,
+                                       the top-k and the selection branch with the gated combine,
+                                       keeping O_cmp (as bf16) and the lists on chip (2 launches);
+                                       its stage S3R_STAGE_CMP then covers selection too */
 
 typedef struct {
   int64_t L;      /* tokens = N views * P tokens per view, >= 1 */

@@ -40,6 +40,7 @@ class Config:
     scale: Optional[float] = None  # None -> 1/sqrt(d)
     debug_checks: bool = False
     test_timeout: bool = False  # testing only: exercise the bounded-wait timeout path
+    single_kernel: bool = False  # topk <= 32: compressed branch, top-k and selection in one kernel
     forced: int = 0
     grid_h: int = 0
     grid_w: int = 0
@@ -64,7 +65,8 @@ class Config:
         return _lib.Params(self.L, self.H, self.d, self.block, QBLOCK, self.topk,
                            0.0 if self.scale is None else float(self.scale),
                            (_lib.S3R_FLAG_DEBUG_CHECKS if self.debug_checks else 0)
-                           | (_lib.S3R_FLAG_TEST_TIMEOUT if self.test_timeout else 0),
+                           | (_lib.S3R_FLAG_TEST_TIMEOUT if self.test_timeout else 0)
+                           | (_lib.S3R_FLAG_SINGLE_KERNEL if self.single_kernel else 0),
                            self.forced, self.grid_h, self.grid_w, self.special, self.win_h,
                            None if dev_status is None else dev_status.data_ptr(),
                            None if stage_events is None else ctypes.addressof(stage_events))

@@ -157,6 +157,13 @@ int fused_forward(const s3r_params* params, const uint16_t* q, const uint16_t* k
   if ((st = launched(launch_pool_kv(p, k, v, kc, vc, kh, vh, stream))) != S3R_OK) return st;
   if (mark(1) != cudaSuccess) return S3R_ERR_CUDA;
   const bool fused_topk = p.k <= kFusedTopkMax;
+  if ((p.flags & S3R_FLAG_SINGLE_KERNEL) && fused_topk && hm) {
+    st = launched(launch_fused_tc(p, q, kc, vc, kh, vh, gate_logits, out, idx_out, stream));
+    if (st != S3R_OK) return st;
+    for (int i = 2; i <= 4; ++i)
+      if (mark(i) != cudaSuccess) return S3R_ERR_CUDA;
+    return S3R_OK;
+  }
   if ((st = launched(launch_cmp_attn_tc(p, q, kc, vc, nullptr, o_cmp, fused_topk ? nullptr : scores,
                                         fused_topk ? idx : nullptr, stream))) != S3R_OK)
     return st;

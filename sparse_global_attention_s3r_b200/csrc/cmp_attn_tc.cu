@@ -30,6 +30,8 @@
 // TMEM columns: S[2] (64 fp32 each) | O (64 fp32) | Q (64 bf16 = 32) | P (64 bf16 = 32).
 // Every wait is an mbarrier wait bounded in time that also watches a CTA abort flag; on expiry
 // the kernel records S3R_DEV_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
+#include <climits>
+
 #include "s3r.h"
 #include "common.cuh"
 #include "internal.h"
@@ -80,14 +82,56 @@ struct __align__(8) Bars {
   uint64_t never;  // never signalled: waited on only under S3R_FLAG_TEST_TIMEOUT
 };
 
+// barriers of the selection phase of the single fused kernel
+struct __align__(8) Bars2 {
+  uint64_t lists_ready;  // both score warps have posted their lists (and read their last sums)
+  uint64_t ocmp_read;    // every softmax warp has read O_cmp out of TMEM
+  uint64_t q2_full;
+  uint64_t kv2_full[2], kv2_empty[2];
+  uint64_t s2_full, s2_empty;
+  uint64_t p2_full, p2_empty;
+  uint64_t o2_full;
+  uint64_t pair[4];  // per lane quadrant: both column halves have posted their row statistics
+};
+
 constexpr uint32_t kOffKV = 0;                                 // stage s: K at +2s*8K, V +8K
 constexpr uint32_t kOffRed = kOffKV + kStages * 2 * kKVBytes;  // [kRed][4 quadrant][64] f32
 constexpr uint32_t kOffStat = kOffRed + kRed * 4 * 64 * 4;     // [2 halves][128 rows] float2
 constexpr uint32_t kOffBars = kOffStat + 2 * 128 * 8;
-constexpr uint32_t kOffMisc = kOffBars + sizeof(Bars);  // tmem base, abort flag
-constexpr uint32_t kSmemUsed = kOffMisc + 16;
+
+// The single fused kernel runs the selection branch in the same CTA once the compressed branch
+// is done. Its gathered K/V ring and Q tile take the Kc/Vc ring's 80 KB; O_cmp (bf16) takes the
+// partial-sum and statistics area; then come the row-statistics exchange, the top-k lists and
+// the barriers. Two CTAs still share an SM.
+constexpr int kSelStep = 64;    // slots of each query block per selection step
+constexpr int kSelStages = 2;   // gathered K/V ring depth
+constexpr uint32_t kSelTileBytes = 2 * kSelStep * 128;  // 128 tokens x 128 B: one K or V tile
+constexpr uint32_t kOffKV2 = 0;  // stage s: K tile at 2s*16K, V tile at +16K
+constexpr uint32_t kOffQ2 = kOffKV2 + kSelStages * 2 * kSelTileBytes;
+constexpr uint32_t kQ2Bytes = kBM * 128;
+static_assert(kOffQ2 + kQ2Bytes <= kOffRed, "the selection ring and Q tile fit the Kc/Vc ring");
+constexpr uint32_t kOffOcmp = kOffRed;  // [128 rows][64] bf16
+constexpr uint32_t kOcmpBytes = kBM * 64 * 2;
+static_assert(kOcmpBytes >= kOffBars - kOffRed, "O_cmp covers the partial sums and statistics");
+constexpr uint32_t kOffXch = kOffOcmp + kOcmpBytes;        // [2 parity][2 half][128 rows] f32
+constexpr uint32_t kOffLists = kOffXch + 2 * 2 * 128 * 4;  // [2 query blocks][32] int32
+constexpr uint32_t kOffBarsF = kOffLists + 2 * 32 * 4;
+constexpr uint32_t kColS2 = 0, kColO2 = 128, kColP2 = 192;  // selection TMEM: S | O_sel | P
+constexpr uint32_t kIdescQK2 = idesc_bf16_f32(kBM, 2 * kSelStep, 0, 0);  // Q smem, K K-major
+constexpr float kMoveRef = 32.f;  // base-2 margin before a selection row's reference max moves
+
+template <bool kFused>
+constexpr uint32_t bars_offset() { return kFused ? kOffBarsF : kOffBars; }
+template <bool kFused>
+constexpr uint32_t misc_offset() {  // tmem base, abort flag
+  return bars_offset<kFused>() + sizeof(Bars) + (kFused ? sizeof(Bars2) : 0);
+}
 // At most two CTAs share an SM (shared memory), so two 256-column TMEM allocations always fit.
-constexpr uint32_t kSmemBytes = (kSmemUsed + 1024 > 80 * 1024 ? kSmemUsed + 1024 : 80 * 1024);
+template <bool kFused>
+constexpr uint32_t smem_bytes() {
+  return misc_offset<kFused>() + 16 + 1024 > 80 * 1024 ? misc_offset<kFused>() + 16 + 1024
+                                                       : 80 * 1024;
+}
 
 struct CmpArgs {
   const uint16_t* q;  // [L, H, 64]
@@ -103,7 +147,26 @@ struct CmpArgs {
   uint32_t* status;
   uint64_t limit_ns;
   uint32_t flags;
+  // the selection phase of the single fused kernel
+  const float* gates;  // [L, H, 2] fp32
+  uint16_t* out;       // [L, H, 64] bf16
+  BlockGeo geo;        // which tokens each key block holds
+  int64_t Lp;          // rows of one head in the head-major K/V copies (nb * b)
+  int b, lb, nsel, nsteps2;  // block size, log2(b), list length forced + topk, 64-slot steps
 };
+
+// Block index of entry s of a query block's selection list in the fused kernel: the forced
+// blocks 0 .. forced-1, then the streamed top-k held in shared memory; past the list, invalid.
+__device__ __forceinline__ int64_t fused_sel_block(const int32_t* topk_list, int s, int forced,
+                                                   int nsel, int64_t nb, bool& ok) {
+  if (s >= nsel) {
+    ok = false;
+    return 0;
+  }
+  const int64_t j = s < forced ? s : topk_list[s - forced];
+  ok = j >= 0 && j < nb;
+  return ok ? j : 0;
+}
 
 // Offer one candidate key c per lane to the warp's sorted list (lane i holds the i-th largest
 // key; lanes 0..k-1 are the current top-k). Keys are unique. Candidates above the k-th key are
@@ -165,18 +228,240 @@ __device__ __forceinline__ float max8(const float (&v)[8]) {
   return fmax3(fmax3(v[0], v[1], v[2]), fmax3(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
 }
 
+// The selection phase of the single fused kernel for one softmax warp. Two warps per TMEM lane
+// quadrant (32 rows of one query block) each take 32 of a step's 64 columns, 4 rows x 8 columns
+// per thread with the 16x256b load shape. The two halves swap their row maxima every step (and
+// their row sums at the end) through shared memory on a bounded per-quadrant mbarrier. A row's
+// reference max is fixed at its first step with a valid column and moves (with O_sel and the row
+// sum rescaled once the previous product has completed) only if a logit exceeds it by 32 in
+// base-2 units, so bf16 P stays below 2^32. Ends with the gated combine of O_cmp (parked in
+// shared memory as bf16) and O_sel, written as bf16. False if a wait gave up.
+__device__ __forceinline__ bool fused_selection(const CmpArgs& a, int h, int64_t q0, int g,
+                                                int half, int lane, uint32_t tbase,
+                                                uint8_t* smem, const int32_t* lists, Bars2* b2,
+                                                volatile int* abort, uint64_t lim) {
+  const int qb = g >> 1;
+  const int tq = lane & 3, tr = lane >> 2;
+  const uint32_t tl0 = tbase + (static_cast<uint32_t>(g * 32) << 16);
+  const uint32_t tl16 = tbase + (static_cast<uint32_t>(g * 32 + 16) << 16);
+  const float sl2 = a.scale_log2;
+  const int32_t* list = lists + qb * 32;
+  float* xch = reinterpret_cast<float*>(smem + kOffXch);  // [parity][half][row]
+
+  {  // the other query block's P columns of these rows stay zero for the whole phase
+    const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    tmem_st32x16(tl0 + kColP2 + (1 - qb) * 32 + half * 16, z);
+    tmem_wait_st_keep16(z);
+  }
+  // value v[i][c]: row tr + 8i of the quadrant, column 32*half + 8*(c/2) + 2*tq + c%2 of the
+  // step's 64 columns of the query block
+  auto col_of = [&](int c) { return half * 32 + 8 * (c >> 1) + 2 * tq + (c & 1); };
+  // post this warp's values for rows tr + 8i (one thread per quad) and return the other half's
+  auto exchange = [&](const float (&mine)[4], float (&theirs)[4], int phase) -> bool {
+    float* buf = xch + (phase & 1) * 256;
+    if (tq == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) buf[half * 128 + g * 32 + tr + 8 * i] = mine[i];
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&b2->pair[g]);
+    if (!mbar_wait(&b2->pair[g], phase & 1, abort, lim)) return false;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) theirs[i] = buf[(1 - half) * 128 + g * 32 + tr + 8 * i];
+    return true;
+  };
+  float mr[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mr[i] = -INFINITY, l[i] = 0.f;
+
+  for (int t = 0; t < a.nsteps2; ++t) {
+    if (!mbar_wait(&b2->s2_full, t & 1, abort, lim)) return false;
+    tc_fence_after();
+    uint32_t r0[16], r1[16];
+    tmem_ld16x256_x4(tl0 + kColS2 + qb * 64 + half * 32, r0);
+    tmem_ld16x256_x4(tl16 + kColS2 + qb * 64 + half * 32, r1);
+    tmem_wait_ld_n<16>(r0);
+    tmem_wait_ld_n<16>(r1);
+    tc_fence_before();
+    __syncwarp();  // one arrival per warp: its lanes' TMEM loads have all completed
+    if (lane == 0) mbar_arrive(&b2->s2_empty);
+    float v[4][8];
+    unpack_rows(r0, r1, v);
+    {  // columns whose slot holds no token (a 64-slot step spans at most two blocks, b >= 32)
+      const int p0 = t * kSelStep;
+      const int s_lo = p0 >> a.lb, s_hi = (p0 + kSelStep - 1) >> a.lb;
+      bool ok_lo, ok_hi;
+      const int64_t j_lo = fused_sel_block(list, s_lo, a.forced, a.nsel, a.nb, ok_lo);
+      const int64_t j_hi = fused_sel_block(list, s_hi, a.forced, a.nsel, a.nb, ok_hi);
+      const BlockOrigin bo_lo = block_origin(a.geo, j_lo), bo_hi = block_origin(a.geo, j_hi);
+      const bool all_valid =
+          ok_lo && ok_hi && origin_full(a.geo, bo_lo) && origin_full(a.geo, bo_hi);
+      if (!all_valid) {
+        uint64_t bits;
+        if (a.b >= kSelStep) {
+          bits = ok_lo ? slot_bits(a.geo, bo_lo, p0 & (a.b - 1), kSelStep) : 0ull;
+        } else {
+          bits = (ok_lo ? slot_bits(a.geo, bo_lo, 0, 32) : 0ull) |
+                 ((ok_hi ? slot_bits(a.geo, bo_hi, 0, 32) : 0ull) << 32);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (!((bits >> col_of(c)) & 1ull)) v[0][c] = v[1][c] = v[2][c] = v[3][c] = -INFINITY;
+      }
+    }
+    // row maxima of this step over both column halves
+    float tmax[4], other[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float m = max8(v[i]);
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      tmax[i] = m;
+    }
+    if (!exchange(tmax, other, t)) return false;
+    bool move = false;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      tmax[i] = fmaxf(tmax[i], other[i]);
+      move |= tmax[i] * sl2 > mr[i] * sl2 + kMoveRef;  // true on the first step with a valid column
+    }
+    // P(t) may overwrite the P buffer (and O_sel be rescaled) once P*V of step t-1 completed
+    if (!mbar_wait(&b2->p2_empty, (t & 1) ^ 1, abort, lim)) return false;
+    if (__any_sync(0xffffffffu, move)) {
+      float f[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float mn = tmax[i] * sl2 > mr[i] * sl2 + kMoveRef ? tmax[i] : mr[i];
+        f[i] = mr[i] == -INFINITY ? 0.f : exp2_approx((mr[i] - mn) * sl2);
+        l[i] *= f[i];
+        mr[i] = mn;
+      }
+      if (t > 0) {  // this half's O_sel columns of the warp's rows (lane = row) times the factor
+        const int src = 4 * (lane & 7);  // a thread of the quad that holds row `lane`
+        const float f0 = __shfl_sync(0xffffffffu, f[0], src);
+        const float f1 = __shfl_sync(0xffffffffu, f[1], src);
+        const float f2 = __shfl_sync(0xffffffffu, f[2], src);
+        const float f3 = __shfl_sync(0xffffffffu, f[3], src);
+        const int which = lane >> 3;
+        const float fr = which == 0 ? f0 : which == 1 ? f1 : which == 2 ? f2 : f3;
+        tc_fence_after();
+#pragma unroll 1
+        for (int q4 = 0; q4 < 2; ++q4) {
+          uint32_t o[16];
+          tmem_ld32x16(tl0 + kColO2 + half * 32 + 16 * q4, o);
+          tmem_wait_ld_n<16>(o);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * fr);
+          tmem_st32x16(tl0 + kColO2 + half * 32 + 16 * q4, o);
+          tmem_wait_st_keep16(o);
+        }
+      }
+    }
+    // P = exp2(v * sl2 - ref * sl2), its row sums, and bf16 P in the 16x128b store layout:
+    // repetition rep covers TMEM columns 4rep..4rep+3 of this half's 16, lane tr -> register
+    // 2rep, lane tr+8 -> 2rep+1; value columns (2rep, 2rep+1) are keys 32half + 8rep + 2tq + {0,1}
+    float off[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) off[i] = mr[i] == -INFINITY ? 0.f : -mr[i] * sl2;
+    uint32_t a0[8], a1[8];
+#pragma unroll
+    for (int rep = 0; rep < 4; ++rep) {
+      const int c = 2 * rep;
+      float e[4][2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 x = __ffma2_rn(make_float2(v[i][c], v[i][c + 1]), make_float2(sl2, sl2),
+                                    make_float2(off[i], off[i]));
+        e[i][0] = exp2_approx(x.x);
+        e[i][1] = exp2_approx(x.y);
+        l[i] += e[i][0] + e[i][1];
+      }
+      a0[2 * rep] = pack_bf16(e[0][0], e[0][1]);
+      a0[2 * rep + 1] = pack_bf16(e[1][0], e[1][1]);
+      a1[2 * rep] = pack_bf16(e[2][0], e[2][1]);
+      a1[2 * rep + 1] = pack_bf16(e[3][0], e[3][1]);
+    }
+    tmem_st16x128_x4(tl0 + kColP2 + qb * 32 + half * 16, a0);
+    tmem_st16x128_x4(tl16 + kColP2 + qb * 32 + half * 16, a1);
+    tmem_wait_st_keep8(a0);
+    tmem_wait_st_keep8(a1);
+    tc_fence_before();
+    __syncwarp();  // one arrival per warp: its lanes' TMEM stores have all completed
+    if (lane == 0) mbar_arrive(&b2->p2_full);
+  }
+
+  // row sums over both halves, then O_sel / l on this half's 32 columns (lane = row), combined
+  float lsum[4], lother[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float s = l[i];
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    lsum[i] = s;
+  }
+  if (!exchange(lsum, lother, a.nsteps2)) return false;
+  if (!mbar_wait(&b2->o2_full, 0, abort, lim)) return false;
+  const int src = 4 * (lane & 7);
+  float tot[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) tot[i] = lsum[i] + lother[i];
+  const float s0 = __shfl_sync(0xffffffffu, tot[0], src);
+  const float s1 = __shfl_sync(0xffffffffu, tot[1], src);
+  const float s2 = __shfl_sync(0xffffffffu, tot[2], src);
+  const float s3 = __shfl_sync(0xffffffffu, tot[3], src);
+  const int which = lane >> 3;
+  const float rs = which == 0 ? s0 : which == 1 ? s1 : which == 2 ? s2 : s3;
+  const float inv = rs > 0.f ? 1.f / rs : 0.f;
+  tc_fence_after();
+  uint32_t o[32];
+  tmem_ld32(tl0 + kColO2 + half * 32, o);
+  tmem_wait_ld_regs(o);
+  const int64_t row = q0 + g * 32 + lane;
+  if (row < a.L) {
+    const int64_t at = (row * a.H + h) * 64 + half * 32;
+    const float2 gl = *reinterpret_cast<const float2*>(a.gates + (row * a.H + h) * 2);
+    const float gc = 1.f / (1.f + expf(-gl.x));
+    const float gs = 1.f / (1.f + expf(-gl.y));
+    const uint4* oc = reinterpret_cast<const uint4*>(smem + kOffOcmp) + (g * 32 + lane) * 8 + half * 4;
+    uint4* dst = reinterpret_cast<uint4*>(a.out + at);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 c = oc[j];
+      const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float c_lo = __uint_as_float(cw[e] << 16), c_hi = __uint_as_float(cw[e] & 0xFFFF0000u);
+        w[e] = pack_bf16(gc * c_lo + gs * (__uint_as_float(o[8 * j + 2 * e]) * inv),
+                         gc * c_hi + gs * (__uint_as_float(o[8 * j + 2 * e + 1]) * inv));
+      }
+      dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  return true;
+}
+
+// kFused: after the compressed branch, the same CTA runs the selection branch for its two query
+// blocks on the streamed top-k lists and writes the gated combine; tmQ2, tmK2, tmV2 (the Q tile,
+// and the head-major K/V copies) are used only then.
+template <bool kFused>
 __global__ void __launch_bounds__(kThreads, 2)
     cmp_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const CmpArgs a) {
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmQ2,
+                       const __grid_constant__ CUtensorMap tmK2,
+                       const __grid_constant__ CUtensorMap tmV2, const CmpArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_addr(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);  // 1024-byte aligned base
   const uint32_t sbase = smem_addr(smem);
-  Bars* bars = reinterpret_cast<Bars*>(smem + kOffBars);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  volatile int* abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  Bars* bars = reinterpret_cast<Bars*>(smem + bars_offset<kFused>());
+  Bars2* b2 = reinterpret_cast<Bars2*>(smem + bars_offset<kFused>() + sizeof(Bars));
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + misc_offset<kFused>());
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + misc_offset<kFused>() + 4);
   float* red = reinterpret_cast<float*>(smem + kOffRed);
   float2* stat = reinterpret_cast<float2*>(smem + kOffStat);
+  int32_t* lists = reinterpret_cast<int32_t*>(smem + kOffLists);  // fused: [2][32] top-k
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
@@ -205,12 +490,32 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->drain, 1);
     mbar_init(&bars->never, 1);
+    if constexpr (kFused) {
+      mbar_init(&b2->lists_ready, 2);
+      mbar_init(&b2->ocmp_read, kSoftmaxWarps);
+      mbar_init(&b2->q2_full, 1);
+      for (int s = 0; s < kSelStages; ++s) {
+        mbar_init(&b2->kv2_full[s], 1);
+        mbar_init(&b2->kv2_empty[s], 1);
+      }
+      mbar_init(&b2->s2_full, 1);
+      mbar_init(&b2->s2_empty, kSoftmaxWarps);
+      mbar_init(&b2->p2_full, kSoftmaxWarps);
+      mbar_init(&b2->p2_empty, 1);
+      mbar_init(&b2->o2_full, 1);
+      for (int g = 0; g < 4; ++g) mbar_init(&b2->pair[g], 2);
+    }
     *abort = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    if constexpr (kFused) {
+      prefetch_tmap(&tmQ2);
+      prefetch_tmap(&tmK2);
+      prefetch_tmap(&tmV2);
+    }
   }
   if (warp == 1) tmem_alloc(tmem_holder, kTmemCols);
   tc_fence_before();
@@ -243,6 +548,51 @@ __global__ void __launch_bounds__(kThreads, 2)
         int dummy = 0;
         for (int u = issued - 1; u >= 0 && u >= issued - kStages; --u)
           mbar_wait(&bars->kv_full[u % kStages], (u / kStages) & 1, &dummy, lim);
+      }
+      if constexpr (kFused) {
+        // selection: once every compressed-branch product has completed (the Kc/Vc ring is
+        // free) and the lists are posted, load the Q tile and gather the selected blocks' K/V
+        // rows from the head-major copies, 64 slots of each query block per step
+        if (ok) ok = mbar_wait(&bars->o_full, 0, abort, lim);
+        if (ok) ok = mbar_wait(&b2->lists_ready, 0, abort, lim);
+        int issued2 = 0;
+        bool q_issued = false;
+        if (ok) {
+          mbar_arrive_expect_tx(&b2->q2_full, kQ2Bytes);
+          tma_load_2d(sbase + kOffQ2, &tmQ2, h * 64, static_cast<int32_t>(q0), &b2->q2_full);
+          q_issued = true;
+          const int box = a.b < kSelStep ? a.b : kSelStep;  // rows per box: one run of slots
+          for (int t = 0; t < a.nsteps2; ++t) {
+            const int stage = t % kSelStages;
+            if (!mbar_wait(&b2->kv2_empty[stage], ((t / kSelStages) & 1) ^ 1, abort, lim)) {
+              ok = false;
+              break;
+            }
+            const uint32_t sk = sbase + kOffKV2 + stage * 2 * kSelTileBytes;
+            mbar_arrive_expect_tx(&b2->kv2_full[stage], 2 * kSelTileBytes);
+            for (int qb = 0; qb < 2; ++qb) {
+              for (int part = 0; part < kSelStep / box; ++part) {
+                const int pos = t * kSelStep + part * box;
+                bool valid;  // an entry past the list loads block 0 and is masked
+                const int64_t j = fused_sel_block(lists + qb * 32, pos >> a.lb, a.forced, a.nsel,
+                                                  a.nb, valid);
+                const int64_t row = j * a.b + (pos & (a.b - 1));  // slot row of the copy
+                const uint32_t row_off = (qb * kSelStep + part * box) * 128;
+                const int32_t y = static_cast<int32_t>(h * a.Lp + row);
+                tma_load_2d(sk + row_off, &tmK2, 0, y, &b2->kv2_full[stage]);
+                tma_load_2d(sk + kSelTileBytes + row_off, &tmV2, 0, y, &b2->kv2_full[stage]);
+              }
+            }
+            issued2 = t + 1;
+          }
+        }
+        if (!ok) {
+          raise_abort(abort, a.status);
+          int dummy = 0;
+          if (q_issued) mbar_wait(&b2->q2_full, 0, &dummy, lim);
+          for (int t = issued2 - 1; t >= 0 && t >= issued2 - kSelStages; --t)
+            mbar_wait(&b2->kv2_full[t % kSelStages], (t / kSelStages) & 1, &dummy, lim);
+        }
       }
     }
   } else if (warp == 1) {
@@ -286,9 +636,48 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (t > 0 && !(ok = pv(t - 1))) break;
       }
       if (ok) ok = pv(nt - 1);
-      if (ok) {
-        tc_commit(&bars->o_full);
-      } else {
+      if (ok) tc_commit(&bars->o_full);
+      if constexpr (kFused) {
+        // selection: S = Q K^T (M=128 x N=128, Q from shared memory: its TMEM columns now hold
+        // P) and O_sel += P V, with O_sel where O_cmp was once the softmax warps have read it
+        if (ok) ok = mbar_wait(&b2->q2_full, 0, abort, lim);
+        if (ok) ok = mbar_wait(&b2->ocmp_read, 0, abort, lim);
+        tc_fence_after();
+        const uint64_t dq = desc_sw128(sbase + kOffQ2);
+        auto qk2 = [&](int t) -> bool {
+          const int stage = t % kSelStages;
+          if (!mbar_wait(&b2->kv2_full[stage], (t / kSelStages) & 1, abort, lim)) return false;
+          if (!mbar_wait(&b2->s2_empty, (t & 1) ^ 1, abort, lim)) return false;
+          tc_fence_after();
+          const uint64_t dk = desc_sw128(sbase + kOffKV2 + stage * 2 * kSelTileBytes);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ss(tbase + kColS2, dq + 2 * ks, dk + 2 * ks, kIdescQK2, ks > 0);
+          tc_commit(&b2->s2_full);
+          return true;
+        };
+        auto pv2 = [&](int t) -> bool {
+          const int stage = t % kSelStages;
+          if (!mbar_wait(&b2->p2_full, t & 1, abort, lim)) return false;
+          tc_fence_after();
+          const uint64_t dv =
+              desc_sw128(sbase + kOffKV2 + stage * 2 * kSelTileBytes + kSelTileBytes);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)  // 128 keys in steps of 16: 16 rows x 128 B = 2048 B
+            mma_ts(tbase + kColO2, tbase + kColP2 + ks * 8, dv + 128 * ks, kIdescPV,
+                   (t > 0 || ks > 0) ? 1u : 0u);
+          tc_commit(&b2->kv2_empty[stage]);
+          tc_commit(&b2->p2_empty);
+          return true;
+        };
+        for (int t = 0; ok && t < a.nsteps2; ++t) {
+          if (!(ok = qk2(t))) break;
+          if (t > 0 && !(ok = pv2(t - 1))) break;
+        }
+        if (ok) ok = pv2(a.nsteps2 - 1);
+        if (ok) tc_commit(&b2->o2_full);
+      }
+      if (!ok) {
         raise_abort(abort, a.status);
         int dummy = 0;
         tc_commit(&bars->drain);  // every MMA issued so far has finished once this arrives
@@ -499,14 +888,36 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t o[32];
       tmem_ld32(tl0 + kColO + half * 32, o);
       tmem_wait_ld_regs(o);
-      const int64_t row = q0 + g * 32 + lane;
-      if (row < a.L) {
-        float4* dst = reinterpret_cast<float4*>(a.o_cmp + (row * a.H + h) * 64 + half * 32);
+      if constexpr (kFused) {
+        // O_cmp has left TMEM (the selection accumulates there next); once the score warps
+        // have read their last partial sums it is parked, in bf16, over that area: this thread
+        // writes and later reads back row g*32 + lane, columns half*32 ..
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b2->ocmp_read);
+        if ((ok = mbar_wait(&b2->lists_ready, 0, abort, lim))) {
+          uint4* dst = reinterpret_cast<uint4*>(smem + kOffOcmp) + (g * 32 + lane) * 8 + half * 4;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          dst[j] = make_float4(__uint_as_float(o[4 * j]), __uint_as_float(o[4 * j + 1]),
-                               __uint_as_float(o[4 * j + 2]), __uint_as_float(o[4 * j + 3]));
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_uint4(
+                pack_bf16(__uint_as_float(o[8 * j]), __uint_as_float(o[8 * j + 1])),
+                pack_bf16(__uint_as_float(o[8 * j + 2]), __uint_as_float(o[8 * j + 3])),
+                pack_bf16(__uint_as_float(o[8 * j + 4]), __uint_as_float(o[8 * j + 5])),
+                pack_bf16(__uint_as_float(o[8 * j + 6]), __uint_as_float(o[8 * j + 7])));
+        }
+      } else {
+        const int64_t row = q0 + g * 32 + lane;
+        if (row < a.L) {
+          float4* dst = reinterpret_cast<float4*>(a.o_cmp + (row * a.H + h) * 64 + half * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(__uint_as_float(o[4 * j]), __uint_as_float(o[4 * j + 1]),
+                                 __uint_as_float(o[4 * j + 2]), __uint_as_float(o[4 * j + 3]));
+        }
       }
+    }
+    if constexpr (kFused) {
+      if (ok) ok = fused_selection(a, h, q0, g, half, lane, tbase, smem, lists, b2, abort, lim);
     }
     if (!ok) raise_abort(abort, a.status);
   } else {
@@ -553,6 +964,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane < a.topk)
         list[a.forced + lane] = static_cast<int32_t>(~static_cast<uint32_t>(best & 0xFFFFFFFFull));
     }
+    if constexpr (kFused) {  // the top-k part of the list, for this CTA's selection phase
+      if (lane < a.topk)
+        lists[qb * 32 + lane] = static_cast<int32_t>(~static_cast<uint32_t>(best & 0xFFFFFFFFull));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b2->lists_ready);  // also after a timeout: waiters stop sooner
+    }
   }
 
   __syncwarp();
@@ -571,13 +988,41 @@ cudaError_t launch_cmp_attn_tc(const Problem& p, const uint16_t* q, const uint16
   CUtensorMap tk, tv;
   if (!make_tmap_head_rows(&tk, kc, p.nb, p.H, kBN) || !make_tmap_head_rows(&tv, vc, p.nb, p.H, kBN))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(cmp_attn_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  constexpr uint32_t smem = smem_bytes<false>();
+  cudaError_t e = cudaFuncSetAttribute(cmp_attn_tc_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   CmpArgs a{q, lse, o_cmp, scores, idx, p.k, p.F, p.L, p.nb, p.nqb, p.H, p.scale_log2, p.status,
             (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull, p.flags};
   dim3 grid(static_cast<unsigned>((p.L + kBM - 1) / kBM), p.H);
-  cmp_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tk, tv, a);
+  cmp_attn_tc_kernel<false><<<grid, kThreads, smem, st>>>(tk, tv, tk, tk, tk, a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fused_tc(const Problem& p, const uint16_t* q, const uint16_t* kc,
+                            const uint16_t* vc, const uint16_t* kh, const uint16_t* vh,
+                            const float* gates, uint16_t* out, int32_t* idx, cudaStream_t st) {
+  const int64_t Lp = p.nb * p.b;
+  if (p.k > kFusedTopkMax || p.H * Lp > INT32_MAX) return cudaErrorInvalidValue;
+  const int box = p.b < kSelStep ? p.b : kSelStep;
+  CUtensorMap tk, tv, tq2, tk2, tv2;
+  if (!make_tmap_head_rows(&tk, kc, p.nb, p.H, kBN) || !make_tmap_head_rows(&tv, vc, p.nb, p.H, kBN) ||
+      !make_tmap_head_rows(&tq2, q, p.L, p.H, kBM) || !make_tmap_rows64(&tk2, kh, p.H * Lp, box) ||
+      !make_tmap_rows64(&tv2, vh, p.H * Lp, box))
+    return cudaErrorInvalidValue;
+  constexpr uint32_t smem = smem_bytes<true>();
+  cudaError_t e = cudaFuncSetAttribute(cmp_attn_tc_kernel<true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int lb = p.b == 32 ? 5 : p.b == 64 ? 6 : 7;
+  const int64_t ntok = static_cast<int64_t>(p.nsel) * p.b;
+  CmpArgs a{q, nullptr, nullptr, nullptr, idx, p.k, p.F, p.L, p.nb, p.nqb, p.H, p.scale_log2,
+            p.status, (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull, p.flags,
+            gates, out, p.geo, Lp, p.b, lb, p.nsel,
+            static_cast<int>((ntok + kSelStep - 1) / kSelStep)};
+  dim3 grid(static_cast<unsigned>((p.L + kBM - 1) / kBM), p.H);
+  cmp_attn_tc_kernel<true><<<grid, kThreads, smem, st>>>(tk, tv, tq2, tk2, tv2, a);
   count_launch();
   return cudaGetLastError();
 }

@@ -36,6 +36,12 @@ constexpr int kFusedTopkMax = 32;
 cudaError_t launch_cmp_attn_tc(const Problem& p, const uint16_t* q, const uint16_t* kc,
                                const uint16_t* vc, float* lse, float* o_cmp, float* scores,
                                int32_t* idx, cudaStream_t st);
+// The single fused kernel (topk <= kFusedTopkMax): the compressed branch with the streamed
+// top-k, then, in the same CTA, the selection branch on the head-major K/V copies kh, vh and the
+// gated combine into out; idx (nullable) receives the selection lists.
+cudaError_t launch_fused_tc(const Problem& p, const uint16_t* q, const uint16_t* kc,
+                            const uint16_t* vc, const uint16_t* kh, const uint16_t* vh,
+                            const float* gates, uint16_t* out, int32_t* idx, cudaStream_t st);
 cudaError_t launch_topk(const Problem& p, const float* scores, int32_t* idx, cudaStream_t st);
 // o_sel != nullptr: write the selection output (fp32). Otherwise fuse the gated combine:
 // read o_cmp and gates and write out (bf16).

@@ -249,6 +249,26 @@ def test_bounded_wait_timeout_is_reported_and_the_context_survives(dev):
     check_close("lse after a timeout", f64(lse), rlse, 2e-5)
 
 
+def test_selection_bounded_wait_timeout_is_reported_and_the_context_survives(dev):
+    """The selection kernel's softmax warps wait on a barrier nothing signals: the MMA issuer and
+    the gather producer give up on their own bounded waits, drain what they issued, the kernel
+    records S3R_DEV_TIMEOUT and frees its TMEM; the next call is correct."""
+    cfg0, pb, x, d = inputs("ragged_b32_odd_k", dev)
+    rng = np.random.default_rng(3)
+    idx = np.stack([np.stack([rng.permutation(cfg0.nb)[:cfg0.topk] for _ in range(cfg0.nqb)])
+                    for _ in range(cfg0.H)]).astype(np.int32)
+    idx_d = torch.from_numpy(idx).to(dev)
+    word = torch.zeros(1, dtype=torch.int32, device=dev)
+    bad = api.Config(L=cfg0.L, H=cfg0.H, block=cfg0.block, topk=cfg0.topk, test_timeout=True)
+    api.sel_attn(bad, d["q"], d["k"], d["v"], idx_d, dev_status=word)
+    assert api.read_device_status(word) & _lib.S3R_DEV_TIMEOUT
+    o = api.sel_attn(cfg0, d["q"], d["k"], d["v"], idx_d, dev_status=word)
+    assert api.read_device_status(word) == 0
+    ref = O.sel_attn(pb, O.bf16_bits(x.q), O.bf16_bits(x.k), O.bf16_bits(x.v), idx)
+    check_close("o_sel after a timeout", f64(o), ref, 2.0 ** -8 * np.abs(f64(x.v)).max() + 1e-6,
+                rl2=4e-3)
+
+
 # --------------------------------------------------------------------------------------------
 # VGGT variant: the reference frame's blocks open every selection list
 # --------------------------------------------------------------------------------------------
@@ -411,3 +431,64 @@ def test_host_pipeline_matches_device_calls(dev):
     pipe.synchronize()
     for got, ref in zip(host_out, want):
         assert torch.equal(got, ref)
+
+
+# --------------------------------------------------------------------------------------------
+# the single fused kernel: compressed branch, streamed top-k and selection in one CTA
+# --------------------------------------------------------------------------------------------
+
+SINGLE = ["tiny", "ragged_b64", "ragged_b32_odd_k", "ragged_b128", "single_partial_block",
+          "one_token", "tail_of_one_row", "dense_selection", "multi_tile_keys"]
+
+
+def _single(cfg):
+    return api.Config(**{**cfg.__dict__, "single_kernel": True})
+
+
+@pytest.mark.parametrize("name", SINGLE)
+def test_single_kernel_whole_path(dev, name):
+    """Two launches (pooling, then one kernel per query tile): the same lists as the three-launch
+    path (the compressed branch is the same arithmetic), and the output against the oracle."""
+    cfg, pb, x, d = inputs(name, dev)
+    n0 = _lib.kernel_launches()
+    out, idx = _fused(_single(cfg), d)
+    assert _lib.kernel_launches() - n0 == 2
+    out3, idx3 = _fused(cfg, d)
+    np.testing.assert_array_equal(idx, idx3)
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    ref = O.sparse_attn(pb, *bits, x.gates.numpy(), idx_given=idx)
+    check_output(out, ref.out)
+    # O_cmp is kept as bf16 on chip: within a bf16 rounding of the three-launch output
+    assert np.abs(out - out3).max() <= 2.0 ** -7 * np.abs(out3).max() + 1e-6
+
+
+@pytest.mark.parametrize("name", ["vggt_4_views", "forced_b32_odd_list", "forced_plus_k_is_nb"])
+def test_single_kernel_forced(dev, name):
+    cfg, pb, x, d = forced_inputs(name, dev)
+    out, idx = _fused(_single(cfg), d)
+    out3, idx3 = _fused(cfg, d)
+    np.testing.assert_array_equal(idx, idx3)
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    check_output(out, O.sparse_attn(pb, *bits, x.gates.numpy(), idx_given=idx).out)
+
+
+@pytest.mark.parametrize("name", ["vggt_4_views_8x8", "vggt_ref_view_forced", "odd_grid_4x8_b32",
+                                  "wide_8x16_b128", "special_fills_a_block"])
+def test_single_kernel_windows(dev, name):
+    cfg, pb, x, d = window_inputs(name, dev)
+    out, idx = _fused(_single(cfg), d)
+    out3, idx3 = _fused(cfg, d)
+    np.testing.assert_array_equal(idx, idx3)
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    check_output(out, O.sparse_attn(pb, *bits, x.gates.numpy(), idx_given=idx).out)
+
+
+def test_single_kernel_timeout_is_reported_and_the_context_survives(dev):
+    cfg, pb, x, d = inputs("ragged_b64", dev)
+    word = torch.zeros(1, dtype=torch.int32, device=dev)
+    bad = api.Config(**{**cfg.__dict__, "single_kernel": True, "test_timeout": True})
+    api.sparse_attn_fwd(bad, d["q"], d["k"], d["v"], d["gates"], dev_status=word)
+    assert api.read_device_status(word) & _lib.S3R_DEV_TIMEOUT
+    out, idx = _fused(_single(cfg), d)
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    check_output(out, O.sparse_attn(pb, *bits, x.gates.numpy(), idx_given=idx).out)
