@@ -28,6 +28,11 @@
 //               winners are inserted by a warp-wide ordered shift, so the score matrix never
 //               exists; blocks below `forced` never compete
 // TMEM columns: S[2] (64 fp32 each) | O (64 fp32) | Q (64 bf16 = 32) | P (64 bf16 = 32).
+// The kernel is a template on kFused. cmp_attn_tc_kernel<false> is the compressed branch alone
+// (O_cmp, lse, scores and/or the top-k to global memory). cmp_attn_tc_kernel<true> is the single
+// fused kernel: after pass B the same warps run the selection branch for the CTA's two query
+// blocks on the streamed top-k (fused_selection) and write the gated combine; O_cmp is parked in
+// shared memory as bf16 and the selection's ring reuses the Kc/Vc ring.
 // Every wait is an mbarrier wait bounded in time that also watches a CTA abort flag; on expiry
 // the kernel records S3R_DEV_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
 #include <climits>
