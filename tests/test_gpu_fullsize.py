@@ -17,7 +17,7 @@ from parity import check_output, check_selection
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
-FULL = {  # name: (L, H, b, k, seed, sampled query blocks)
+FULL = {  # name: (L, H, b, k, seed, sampled query blocks[, 2-D geometry, forced views, single])
     "vggt32": (43968, 16, 64, 16, 1, 64),
     "n100": (137400, 16, 64, 32, 2, 48),
     "n1000": (1374000, 16, 64, 32, 3, 64),
@@ -25,6 +25,11 @@ FULL = {  # name: (L, H, b, k, seed, sampled query blocks)
     "pi3_b64": (274800, 16, 64, 16, 4001, 24),
     "pi3_b128": (274800, 16, 128, 8, 4002, 24),
     "pi3_b64_all_blocks": (274800, 16, 64, 4294, 4003, 3),  # top-k = nb: dense selection
+    # the 1000-view layer with 2-D key windows (5 special tokens + 37 x 37 patches a view, 8 x 8)
+    "n1000_windows": (1374000, 16, 64, 32, 3, 32, dict(grid_h=37, grid_w=37, special=5, win_h=8)),
+    # VGGT-32 with the reference view forced, through the single fused kernel
+    "vggt32_ref_view_single": (43968, 16, 64, 16, 5, 48,
+                               dict(grid_h=37, grid_w=37, special=5, win_h=8), 1, True),
 }
 
 
@@ -32,15 +37,20 @@ FULL = {  # name: (L, H, b, k, seed, sampled query blocks)
 def test_fused_path_at_workload_size(name):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    L, H, b, k, seed, nsample = FULL[name]
+    L, H, b, k, seed, nsample, *more = FULL[name]
+    geo = more[0] if more else {}
+    forced_views = more[1] if len(more) > 1 else 0
+    single = more[2] if len(more) > 2 else False
+    forced = forced_views * (api.Config(L=L, H=H, block=b, topk=1, **geo).nb // (L // (
+        geo["special"] + geo["grid_h"] * geo["grid_w"]))) if forced_views else 0
     dev = torch.device("cuda")
     x = synth.make_inputs(L, H, 64, b, seed, device=dev)
-    cfg = api.Config(L=L, H=H, block=b, topk=k)
+    cfg = api.Config(L=L, H=H, block=b, topk=k, forced=forced, single_kernel=single, **geo)
     sa = api.SparseAttention(cfg, dev)
     out = sa(x.q, x.k, x.v, x.gates)
     torch.cuda.synchronize()
 
-    pb = O.Problem(L, H, 64, b, k)
+    pb = O.Problem(L, H, 64, b, k, forced=forced, **geo)
     rng = np.random.default_rng(seed)
     blocks = sorted(set(rng.choice(cfg.nqb - 1, size=nsample - 1, replace=False).tolist())
                     | {cfg.nqb - 1})
@@ -55,7 +65,7 @@ def test_fused_path_at_workload_size(name):
 
     kc, vc = O.pool(pb, bits[1]), O.pool(pb, bits[2])
     ref = O.sparse_attn(pb, *bits, gates, qblocks=blocks, pooled=(kc, vc))
-    stats = check_selection(got_idx, ref.idx, ref.gap, ref.scores, k)
+    stats = check_selection(got_idx, ref.idx, ref.gap, ref.scores, k, forced)
     # conditional oracle: the oracle's compressed branch, its selection run on the GPU's indices
     o_sel = O.sel_attn(pb, *bits, got_idx, qblocks=blocks)
     cond_out = O.combine(ref.o_cmp, o_sel, np.ascontiguousarray(gates[rows]))
