@@ -492,3 +492,46 @@ def test_single_kernel_timeout_is_reported_and_the_context_survives(dev):
     out, idx = _fused(_single(cfg), d)
     bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
     check_output(out, O.sparse_attn(pb, *bits, x.gates.numpy(), idx_given=idx).out)
+
+
+# --------------------------------------------------------------------------------------------
+# seeded random configurations across every option at once
+# --------------------------------------------------------------------------------------------
+
+def _random_config(seed):
+    """A small configuration drawn from every axis: block size, top-k on both sides of 32,
+    forced blocks, 1-D or 2-D geometry (special tokens, cut windows), single kernel or not."""
+    rng = np.random.default_rng(1000 + seed)
+    b = int(rng.choice([32, 64, 128]))
+    H = int(rng.integers(1, 4))
+    geo = {}
+    if rng.random() < 0.5:
+        wh = int(rng.choice([w for w in (1, 2, 4, 8) if b // w >= 8]))
+        gh, gw = int(rng.integers(1, 24)), int(rng.integers(1, 40))
+        special = int(rng.integers(0, min(b, 6) + 1))
+        views = int(rng.integers(1, 5))
+        geo = dict(grid_h=gh, grid_w=gw, special=special, win_h=wh)
+        L = views * (special + gh * gw)
+    else:
+        L = int(rng.integers(1, 5000))
+    nb = api.Config(L=L, H=H, block=b, topk=1, **geo).nb
+    forced = int(rng.integers(0, min(nb - 1, 8) + 1)) if nb > 1 and rng.random() < 0.4 else 0
+    k = int(rng.integers(1, min(nb - forced, 40) + 1))
+    single = bool(k <= 32 and rng.random() < 0.5)
+    return dict(L=L, H=H, block=b, topk=k, forced=forced, single_kernel=single, **geo)
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_configurations(dev, seed):
+    kw = _random_config(seed)
+    cfg = api.Config(**kw)
+    x = synth.make_inputs(cfg.L, cfg.H, 64, cfg.block, 2000 + seed)
+    d = {n: getattr(x, n).to(dev) for n in ("q", "k", "v", "gates")}
+    out, idx = _fused(cfg, d)
+    pk = {k: v for k, v in kw.items() if k not in ("block", "topk", "single_kernel", "L", "H")}
+    pb = O.Problem(cfg.L, cfg.H, 64, cfg.block, cfg.topk, **pk)
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    ref = O.sparse_attn(pb, *bits, x.gates.numpy())
+    check_selection(idx, ref.idx, ref.gap, ref.scores, cfg.topk, cfg.forced)
+    cond = O.sparse_attn(pb, *bits, x.gates.numpy(), idx_given=idx, pooled=(ref.kc, ref.vc))
+    check_output(out, cond.out)
