@@ -79,11 +79,11 @@ SM_COUNT = 148
 # --no-cpu-baseline), with the SHA-256 of the sources that kernel was built from: once any of them
 # changes, the figure no longer describes the kernel and the roofline reports null.
 TRAFFIC = {
-    "cmp": {"workload": "n1000", "bytes": 2992064768 + 5627342848,
+    "cmp": {"workload": "n1000", "bytes": 3004162304 + 5629871104,
              "sources": ["sparse_global_attention_s3r_b200/csrc/cmp_attn_tc.cu",
                          "sparse_global_attention_s3r_b200/csrc/common.cuh",
                          "sparse_global_attention_s3r_b200/csrc/sm100.cuh"],
-             "sha256": "2897a8c4599c1ccc77cde43ef68e95706e376e7b0ad8941e7c5e4636c4f479c1"},
+             "sha256": "e9f86e53355f80f5358f0ad84a73e3af03ddfb748dd0fffdbb9ed91733994b67"},
 }
 
 
