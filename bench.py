@@ -42,6 +42,16 @@ WORKLOADS = {
                  L=137400, H=16, block=64, topk=32, seed=2),
     "vggt32": dict(desc="VGGT-like layer: N=32 views x P=1374, L=43,968, H=16, d=64, b=64, top-k=16",
                    L=43968, H=16, block=64, topk=16, seed=1),
+    # VGGT's hybrid: the reference view's blocks kept for every query (ceil(1374/64) = 22 leading
+    # blocks; with windows, the view's 26 blocks), top-k = 16 more
+    "vggt32_ref": dict(desc="VGGT-like layer with the reference view kept: N=32 x P=1374, "
+                            "L=43,968, H=16, d=64, b=64, forced=22, top-k=16",
+                       L=43968, H=16, block=64, topk=16, seed=1, forced=22),
+    "vggt32_ref_windows": dict(desc="VGGT-like layer with 2-D key windows and the reference view "
+                                    "kept: N=32 x (5 + 37x37), 8x8 windows, L=43,968, H=16, "
+                                    "d=64, b=64, forced=26, top-k=16",
+                               L=43968, H=16, block=64, topk=16, seed=1, forced=26,
+                               geo=dict(grid_h=37, grid_w=37, special=5, win_h=8)),
     "tiny": dict(desc="tiny: N=4 x P=256, L=1024, H=2, d=64, b=64, top-k=4",
                  L=1024, H=2, block=64, topk=4, seed=0),
     # the same 1000 views with key blocks as 2-D windows: each view's 5 camera/register tokens,
@@ -113,9 +123,9 @@ def algorithmic(cfg):
     """Algorithmic work per call: FLOPs of Q.Kc^T + P.Vc (once) and of the selection's
     Q.K^T + P.V over the tokens actually selected; bytes of each stage's compulsory traffic."""
     L, H, d, b, k, nb, nqb = cfg.L, cfg.H, cfg.d, cfg.block, cfg.topk, cfg.nb, cfg.nqb
-    # tokens selected per query block: k blocks of b (an upper bound: the ragged last 1-D block,
-    # and 2-D windows cut at a grid edge or a view's special-token block, hold fewer)
-    sel_tokens = k * b
+    # tokens selected per query block: forced + k blocks of b (an upper bound: the ragged last
+    # 1-D block, and 2-D windows cut at a grid edge or a view's special-token block, hold fewer)
+    sel_tokens = (getattr(cfg, "forced", 0) + k) * b
     cmp_flops = 4.0 * L * nb * d * H
     sel_flops = 4.0 * L * sel_tokens * d * H
     single = getattr(cfg, "single_kernel", False)  # the compressed stage also runs selection
@@ -260,7 +270,8 @@ def run_reference(args, wl):
     from oracle import oracle as O
     from sparse_global_attention_s3r_b200 import api, synth
 
-    cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"], **wl.get("geo", {}))
+    cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"],
+                     forced=wl.get("forced", 0), **wl.get("geo", {}))
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     x = synth.make_inputs(cfg.L, cfg.H, cfg.d, cfg.block, wl["seed"], device=dev)
     bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
@@ -316,7 +327,8 @@ def run_native(args, wl):
                                 device_id=dev)
 
     cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"],
-                     single_kernel=args.single_kernel, **wl.get("geo", {}))
+                     forced=wl.get("forced", 0), single_kernel=args.single_kernel,
+                     **wl.get("geo", {}))
     seed = rank_seed(wl["seed"], rank)  # an independent layer per GPU
     x = synth.make_inputs(cfg.L, cfg.H, cfg.d, cfg.block, seed, device=dev)
     q, k, v, gates = x.q, x.k, x.v, x.gates
@@ -461,7 +473,8 @@ def run_native(args, wl):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": wl["desc"], "L": cfg.L, "H": cfg.H, "d": cfg.d, "block": cfg.block,
-                   "topk": cfg.topk, "qblock": 64, "seed": wl["seed"], **wl.get("geo", {}),
+                   "topk": cfg.topk, "forced": cfg.forced, "qblock": 64, "seed": wl["seed"],
+                   **wl.get("geo", {}),
                    "kernels": "pool + one fused kernel" if args.single_kernel else
                               "pool + compressed/top-k + selection/combine",
                    "parallelism": "independent layer per GPU" if world > 1 else "single GPU",
