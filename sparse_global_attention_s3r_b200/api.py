@@ -7,7 +7,9 @@ contiguous, with the layouts of include/s3r.h:
     q, k, v      [L, H, 64] bf16          gates  [L, H, 2] fp32
     k_cmp, v_cmp [nb, H, 64] bf16         lse    [H, L] fp32
     o_cmp, o_sel [L, H, 64] fp32          scores [H, nqb, nb] fp32
-    idx          [H, nqb, topk] int32     out    [L, H, 64] bf16
+    idx          [H, nqb, forced + topk] int32
+    out          [L, H, 64] bf16
+nb counts the key blocks of the configured geometry (Config.nb), nqb = ceil(L / 64).
 """
 from __future__ import annotations
 
