@@ -446,18 +446,21 @@ def run_native(args, wl):
         roof = {"bound": "tensor", "achieved": units / dom_s / 1e12,
                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = measured_traffic(dom, args.workload)
-    roof["kernel"] = dom
     roof["peak_source"] = peaks["source"] + (" sustained bf16" if bound == "tensor" else " copy")
     if dom == "cmp":
-        # the compressed branch needs two exponentials per (query, summary) pair; their unit,
-        # not the tensor pipe, is the tighter bound
+        # The compressed branch needs two exponentials per (query, summary) pair. Their unit
+        # (MUFU.EX2, 16 per clock per SM) sets its speed of light, 203 ms at 1000 views, well above
+        # the tensor work's 110-130 ms: the binding roofline is this ALU one; the tensor view
+        # (the algorithmic bf16 FLOPs against the measured GEMM peak) is kept beside it.
         ex2_peak = EX2_PER_CLK_SM * SM_COUNT * peaks.get("sm_max_mhz", 1965.0) * 1e6
         ach = work["cmp_exp2"] / dom_s
-        roof["co_bound"] = {"bound": "alu", "what": "exp2 on the MUFU pipe",
-                            "achieved": ach / 1e12, "peak": ex2_peak / 1e12, "unit": "Texp2/s",
-                            "frac": ach / ex2_peak,
-                            "peak_source": "16 ex2 per clock per SM x 148 SMs x max SM clock"}
+        tensor_view = dict(roof)
+        roof = {"bound": "alu", "what": "exp2 on the MUFU pipe", "achieved": ach / 1e12,
+                "peak": ex2_peak / 1e12, "unit": "Texp2/s", "frac": ach / ex2_peak,
+                "peak_source": "16 ex2 per clock per SM x 148 SMs x max SM clock",
+                "tensor_view": tensor_view}
+    roof["traffic"] = measured_traffic(dom, args.workload)
+    roof["kernel"] = dom
     stages = {}
     for n in _lib.STAGES:
         b_, u_ = work["stage_work"][n]
