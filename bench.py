@@ -9,10 +9,26 @@ in HBM. Default workload: the 1000-view sequence, L = 1,374,000 tokens (N = 1000
 tokens), H = 16, d = 64, b = 64, top-k = 32. Each GPU runs its own independent layer (weak
 scaling, no data-path collective); the step time is the maximum over ranks.
 
-Prints one JSON line (rank 0): tokens/s, algorithmic TFLOP/s and fraction of the measured bf16
-peak, per-stage times from CUDA events recorded inside the fused call, the roofline of the
-dominant kernel, an end-to-end figure through pinned host buffers, the fp64 CPU oracle's timed
-sample, the kernel-launch count and the SM clocks sampled during the timed region.
+Prints one JSON line (rank 0) with:
+
+- tokens/s, algorithmic TFLOP/s and fraction of the measured bf16 peak;
+- per-stage times from CUDA events recorded inside the fused call;
+- the roofline of the dominant kernel (for the compressed branch its exp2 rate against the MUFU
+  peak, with the tensor view beside it) and that kernel's recorded DRAM traffic;
+- an end-to-end figure from pinned host memory through HostPipeline;
+- dense attention (torch SDPA, flash) on the same inputs as context;
+- the fp64 CPU oracle's timed sample;
+- the kernel-launch count;
+- the SM clocks sampled during the timed region.
+
+Other workloads:
+
+- n100, vggt32, tiny;
+- n1000_windows: 2-D key windows;
+- vggt32_ref, vggt32_ref_windows: the reference view kept;
+- pi3_sweep: 24 layers per (b, top-k) setting at 200 views.
+
+--single-kernel runs the compressed branch, top-k and selection as one kernel.
 
 --impl reference times the CPU oracle (the only other implementation of this method) on bounded
 samples of the same workload and prints the same line with "impl": "reference".
