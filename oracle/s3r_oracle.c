@@ -41,6 +41,14 @@
  *   s3r_ref_sel         dense attention (torch SDPA, fp64) when k = nb; brute force per query.
  *   s3r_ref_combine     gate limits and the zero-logit midpoint.
  *   whole pipeline      composition of the pinned steps plus permutation invariances.
+ *   s3r_ref_bwd         torch autograd of the forward restated in torch ops (whose output equals
+ *                       this file's forward); a central finite difference along a random
+ *                       direction; torch SDPA's own backward when the gates switch one branch
+ *                       off (dense selection; attention over torch-pooled means); key gradients
+ *                       summing to zero and value gradients conserving the gated mass; equal
+ *                       values giving no query/key gradient.
+ * The backward (the path is trained end to end, arXiv abstract) holds the selection lists fixed,
+ * since a top-k has no gradient, and passes the bf16 rounding of the pooled K/V straight through.
  */
 #include "s3r_oracle.h"
 
@@ -470,6 +478,157 @@ int s3r_ref_sel(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, c
   sel_ctx c = {p, q, k, v, &rm, idx, o_sel, 0};
   parallel_for((int64_t)p->H * rm.nq, p->threads, sel_task, &c);
   row_map_free(&rm);
+  return c.bad_index ? -3 : 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* backward of the whole path (selection held fixed, pooled rounding passed straight through)  */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+  const s3r_ref_params* p;
+  const uint16_t *q, *k, *v;
+  const double *kc, *vc;
+  const float* gates;
+  const int32_t* idx;
+  const double* dout;
+  double *dq, *dk, *dv, *dgates;
+  int bad_index; /* set when an index is out of range */
+} bwd_ctx;
+
+/* One head: every row's forward again, then its gradients; the pooled summaries' gradients are
+ * gathered over all rows and spread back over their blocks' tokens at the end. */
+static void bwd_task(void* vctx, int64_t h) {
+  bwd_ctx* c = (bwd_ctx*)vctx;
+  const s3r_ref_params* p = c->p;
+  const int64_t nb = s3r_ref_num_blocks(p), nqb = ceil_div(p->L, p->qblock);
+  const int64_t H = p->H, d = p->d, HD = H * d;
+  const int32_t n_list = p->forced + p->topk;
+  double* sc = (double*)malloc(sizeof(double) * (size_t)nb);    /* compressed logits, then P */
+  double* dkc = (double*)calloc((size_t)(nb * d), sizeof(double));
+  double* dvc = (double*)calloc((size_t)(nb * d), sizeof(double));
+  double* qv = (double*)malloc(sizeof(double) * (size_t)d);
+  double* oc = (double*)malloc(sizeof(double) * (size_t)d);
+  double* os = (double*)malloc(sizeof(double) * (size_t)d);
+  double* doc = (double*)malloc(sizeof(double) * (size_t)d);
+  double* dos = (double*)malloc(sizeof(double) * (size_t)d);
+  char* chosen = (char*)malloc((size_t)nb);
+  int64_t* tokens = (int64_t*)malloc(sizeof(int64_t) * (size_t)n_list * (size_t)p->block);
+  double* ss = (double*)malloc(sizeof(double) * (size_t)n_list * (size_t)p->block);
+
+  for (int64_t i = 0; i < nqb; ++i) {
+    /* the query block's token set T, each selected block once */
+    const int32_t* sel = c->idx + (h * nqb + i) * n_list;
+    int64_t nt = 0;
+    for (int64_t j = 0; j < nb; ++j) chosen[j] = 0;
+    for (int32_t s = 0; s < n_list; ++s) {
+      const int64_t j = sel[s];
+      if (j < 0 || j >= nb) {
+        c->bad_index = 1;
+        continue;
+      }
+      if (chosen[j]) continue;
+      chosen[j] = 1;
+      nt += s3r_ref_block_tokens(p, j, tokens + nt);
+    }
+    const int64_t r1 = (i + 1) * p->qblock < p->L ? (i + 1) * p->qblock : p->L;
+    for (int64_t r = i * p->qblock; r < r1; ++r) {
+      for (int64_t e = 0; e < d; ++e) qv[e] = bf16_value(c->q[r * HD + h * d + e]);
+      /* compressed branch: P over all nb summaries and O_cmp */
+      double m = -INFINITY;
+      for (int64_t j = 0; j < nb; ++j) {
+        double dot = 0.0;
+        for (int64_t e = 0; e < d; ++e) dot += qv[e] * c->kc[j * HD + h * d + e];
+        sc[j] = p->scale * dot;
+        if (sc[j] > m) m = sc[j];
+      }
+      double l = 0.0;
+      for (int64_t j = 0; j < nb; ++j) l += exp(sc[j] - m);
+      for (int64_t e = 0; e < d; ++e) oc[e] = 0.0;
+      for (int64_t j = 0; j < nb; ++j) {
+        sc[j] = exp(sc[j] - m) / l;
+        for (int64_t e = 0; e < d; ++e) oc[e] += sc[j] * c->vc[j * HD + h * d + e];
+      }
+      /* selection branch: P over the tokens of T and O_sel */
+      double ms = -INFINITY;
+      for (int64_t a = 0; a < nt; ++a) {
+        double dot = 0.0;
+        for (int64_t e = 0; e < d; ++e) dot += qv[e] * bf16_value(c->k[tokens[a] * HD + h * d + e]);
+        ss[a] = p->scale * dot;
+        if (ss[a] > ms) ms = ss[a];
+      }
+      double ls = 0.0;
+      for (int64_t a = 0; a < nt; ++a) ls += exp(ss[a] - ms);
+      for (int64_t e = 0; e < d; ++e) os[e] = 0.0;
+      for (int64_t a = 0; a < nt; ++a) {
+        ss[a] = exp(ss[a] - ms) / ls;
+        for (int64_t e = 0; e < d; ++e) os[e] += ss[a] * bf16_value(c->v[tokens[a] * HD + h * d + e]);
+      }
+      /* gated aggregation: out = g0 O_cmp + g1 O_sel with g = sigmoid(logit) */
+      const double g0 = sigmoid((double)c->gates[(r * H + h) * 2 + 0]);
+      const double g1 = sigmoid((double)c->gates[(r * H + h) * 2 + 1]);
+      const double* dy = c->dout + r * HD + h * d;
+      double yc = 0.0, ys = 0.0;
+      for (int64_t e = 0; e < d; ++e) {
+        yc += dy[e] * oc[e];
+        ys += dy[e] * os[e];
+        doc[e] = g0 * dy[e];
+        dos[e] = g1 * dy[e];
+      }
+      c->dgates[(r * H + h) * 2 + 0] = g0 * (1.0 - g0) * yc;
+      c->dgates[(r * H + h) * 2 + 1] = g1 * (1.0 - g1) * ys;
+      /* softmax backward: dS = P (dP - <dO, O>), dP = <dO, value>; dq = scale sum dS key,
+       * dkey = scale dS q, dvalue = P dO */
+      double* dqr = c->dq + r * HD + h * d;
+      for (int64_t e = 0; e < d; ++e) dqr[e] = 0.0;
+      double dc = 0.0, ds = 0.0;
+      for (int64_t e = 0; e < d; ++e) dc += doc[e] * oc[e], ds += dos[e] * os[e];
+      for (int64_t j = 0; j < nb; ++j) {
+        double dp = 0.0;
+        for (int64_t e = 0; e < d; ++e) dp += doc[e] * c->vc[j * HD + h * d + e];
+        const double dsj = sc[j] * (dp - dc);
+        for (int64_t e = 0; e < d; ++e) {
+          dqr[e] += p->scale * dsj * c->kc[j * HD + h * d + e];
+          dkc[j * d + e] += p->scale * dsj * qv[e];
+          dvc[j * d + e] += sc[j] * doc[e];
+        }
+      }
+      for (int64_t a = 0; a < nt; ++a) {
+        const int64_t t = tokens[a];
+        double dp = 0.0;
+        for (int64_t e = 0; e < d; ++e) dp += dos[e] * bf16_value(c->v[t * HD + h * d + e]);
+        const double dsa = ss[a] * (dp - ds);
+        for (int64_t e = 0; e < d; ++e) {
+          dqr[e] += p->scale * dsa * bf16_value(c->k[t * HD + h * d + e]);
+          c->dk[t * HD + h * d + e] += p->scale * dsa * qv[e];
+          c->dv[t * HD + h * d + e] += ss[a] * dos[e];
+        }
+      }
+    }
+  }
+  /* pooling backward: each summary is the mean of its block's tokens */
+  for (int64_t j = 0; j < nb; ++j) {
+    const int64_t n = s3r_ref_block_tokens(p, j, tokens);
+    for (int64_t a = 0; a < n; ++a)
+      for (int64_t e = 0; e < d; ++e) {
+        c->dk[tokens[a] * HD + h * d + e] += dkc[j * d + e] / (double)n;
+        c->dv[tokens[a] * HD + h * d + e] += dvc[j * d + e] / (double)n;
+      }
+  }
+  free(sc), free(dkc), free(dvc), free(qv), free(oc), free(os), free(doc), free(dos);
+  free(chosen), free(tokens), free(ss);
+}
+
+int s3r_ref_bwd(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                const double* kc, const double* vc, const float* gates, const int32_t* idx,
+                const double* dout, double* dq, double* dk, double* dv, double* dgates) {
+  if (check_params(p) || !q || !k || !v || !kc || !vc || !gates || !idx || !dout || !dq || !dk ||
+      !dv || !dgates || p->topk < 1 || p->forced < 0)
+    return -1;
+  const int64_t n = p->L * p->H * p->d;
+  for (int64_t e = 0; e < n; ++e) dk[e] = 0.0, dv[e] = 0.0;
+  bwd_ctx c = {p, q, k, v, kc, vc, gates, idx, dout, dq, dk, dv, dgates, 0};
+  parallel_for(p->H, p->threads, bwd_task, &c); /* heads touch disjoint slices of every array */
   return c.bad_index ? -3 : 0;
 }
 

@@ -100,6 +100,17 @@ int s3r_ref_topk(int64_t rows, int64_t n, int32_t k, int32_t forced, const doubl
 int s3r_ref_sel(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                 const int64_t* qblocks, int64_t nq, const int32_t* idx, double* o_sel);
 
+/* Backward of the whole path (Speed3R is trained end to end, arXiv abstract): given dout =
+ * dLoss/dout [L, H, d], the gradients dq, dk, dv [L, H, d] and dgates [L, H, 2] (all double, all
+ * rows). The selection lists idx [H, nqb, F + k] are held fixed (no gradient flows through the
+ * top-k), and the bf16 rounding of the pooled K/V is passed straight through: kc, vc are the
+ * pooled values the forward used (s3r_ref_pool), and dK[t] += dKc[j] / n_j for the n_j tokens t
+ * of block j (the same for V). Returns 0, -1 on bad parameters, -3 when idx holds an index
+ * outside [0, nb). */
+int s3r_ref_bwd(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                const double* kc, const double* vc, const float* gates, const int32_t* idx,
+                const double* dout, double* dq, double* dk, double* dv, double* dgates);
+
 /* Gated aggregation over n rows: out = sigmoid(g[...,0]) * o_cmp + sigmoid(g[...,1]) * o_sel. */
 int s3r_ref_combine(int64_t n, int32_t H, int32_t d, const double* o_cmp, const double* o_sel,
                     const float* gates, double* out);

@@ -39,7 +39,7 @@ MUTANTS = {
         "return (x->index < y->index) - (x->index > y->index);"),
     "topk_gap_from_the_top": (
         "a[c->k - 1].score - a[c->k].score", "a[0].score - a[c->k].score"),
-    "sel_ignores_scale": ("s[a] = p->scale * dot;", "s[a] = dot;"),
+    "sel_ignores_scale": (" s[a] = p->scale * dot;", " s[a] = dot;"),
     "sel_uses_first_query_row": (
         "const int64_t t_q = rm->first[i] + r;", "const int64_t t_q = rm->first[i];"),
     "sel_keys_from_values": (
@@ -65,7 +65,25 @@ MUTANTS = {
     "window_rows_use_grid_width": (
         "const int64_t wr = m / cols, wc = m % cols;", "const int64_t wr = m / p->grid_w, wc = m % cols;"),
     "sel_list_skips_forced_blocks": (
-        "const int32_t n_list = p->forced + p->topk;", "const int32_t n_list = p->topk;"),
+        "const int32_t n_list = p->forced + p->topk; /* always-kept",
+        "const int32_t n_list = p->topk; /* always-kept"),
+    "bwd_sel_drops_softmax_centering": (
+        "const double dsa = ss[a] * (dp - ds);", "const double dsa = ss[a] * dp;"),
+    "bwd_cmp_centres_with_the_other_branch": (
+        "const double dsj = sc[j] * (dp - dc);", "const double dsj = sc[j] * (dp - ds);"),
+    "bwd_pool_spread_without_divisor": (
+        "c->dk[tokens[a] * HD + h * d + e] += dkc[j * d + e] / (double)n;",
+        "c->dk[tokens[a] * HD + h * d + e] += dkc[j * d + e];"),
+    "bwd_gate_derivative_drops_one_minus": (
+        "c->dgates[(r * H + h) * 2 + 0] = g0 * (1.0 - g0) * yc;",
+        "c->dgates[(r * H + h) * 2 + 0] = g0 * yc;"),
+    "bwd_sel_value_grad_ignores_gate": (
+        "c->dv[t * HD + h * d + e] += ss[a] * dos[e];", "c->dv[t * HD + h * d + e] += ss[a] * dy[e];"),
+    "bwd_cmp_key_grad_misses_scale": (
+        "dkc[j * d + e] += p->scale * dsj * qv[e];", "dkc[j * d + e] += dsj * qv[e];"),
+    "bwd_sel_dq_from_values": (
+        "dqr[e] += p->scale * dsa * bf16_value(c->k[t * HD + h * d + e]);",
+        "dqr[e] += p->scale * dsa * bf16_value(c->v[t * HD + h * d + e]);"),
 }
 
 

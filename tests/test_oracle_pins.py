@@ -691,3 +691,182 @@ def test_2d_reference_view_forced_covers_every_token_of_view_zero():
     np.testing.assert_array_equal(np.sort(toks), np.arange(P))
     assert (res.idx[..., :per_view] == np.arange(per_view)).all()
     assert (res.idx[..., per_view:] >= per_view).all()
+
+
+# --------------------------------------------------------------------------------------------
+# backward: gradients of the whole path with the selection held fixed
+# --------------------------------------------------------------------------------------------
+# The path is trained end to end (arXiv abstract of Speed3R), so the oracle also gives the
+# gradients of dQ, dK, dV and the gate logits for an upstream gradient dout. The top-k has no
+# gradient: the lists are fixed; the bf16 rounding of the pooled K/V is passed straight through,
+# so the pins hand the backward the exact fp64 means (pool(..., exact=True)).
+
+def _bwd_inputs(pb, seed, gates=None):
+    q = rand_bits((pb.L, pb.H, pb.d), seed, 1.0)
+    k = rand_bits((pb.L, pb.H, pb.d), seed + 1, 1.0)
+    v = rand_bits((pb.L, pb.H, pb.d), seed + 2, 1.0)
+    g = _gates(pb.L, pb.H, seed + 3) if gates is None else gates
+    dout = torch.randn((pb.L, pb.H, pb.d), generator=torch.Generator().manual_seed(seed + 4),
+                       dtype=torch.float64).numpy()
+    return q, k, v, np.ascontiguousarray(g, np.float32), dout
+
+
+def _bwd(pb, q, k, v, g, idx, dout):
+    kc = O.pool(pb, k, exact=True)
+    vc = O.pool(pb, v, exact=True)
+    return O.backward(pb, q, k, v, g, idx, dout, kc=kc, vc=vc), kc, vc
+
+
+def _torch_path(pb, q, k, v, g, idx):
+    """The forward written with torch ops on fp64 leaves (exact pooling, idx fixed): pooled K/V are
+    means of each block's tokens, the compressed branch attends to all of them, the selection
+    branch to the tokens of the listed blocks, and sigmoid gates mix the two."""
+    blocks = [torch.from_numpy(pb.block_tokens(j)) for j in range(pb.nb)]
+    kc = torch.stack([k[t].mean(0) for t in blocks])
+    vc = torch.stack([v[t].mean(0) for t in blocks])
+    out = []
+    for h in range(pb.H):
+        rows_h = []
+        for i in range(pb.nqb):
+            r = slice(i * pb.qblock, min((i + 1) * pb.qblock, pb.L))
+            qi = q[r, h]
+            oc = torch.softmax(pb.softmax_scale * qi @ kc[:, h].T, -1) @ vc[:, h]
+            toks = torch.cat([blocks[j] for j in sorted(set(idx[h, i].tolist()))])
+            os_ = torch.softmax(pb.softmax_scale * qi @ k[toks, h].T, -1) @ v[toks, h]
+            gi = torch.sigmoid(g[r, h])
+            rows_h.append(gi[:, :1] * oc + gi[:, 1:] * os_)
+        out.append(torch.cat(rows_h))
+    return torch.stack(out, 1)
+
+
+def _leaves(q, k, v, g):
+    return [torch.tensor(values_of(q), requires_grad=True),
+            torch.tensor(values_of(k), requires_grad=True),
+            torch.tensor(values_of(v), requires_grad=True),
+            torch.tensor(g.astype(np.float64), requires_grad=True)]
+
+
+@pytest.mark.parametrize("pb", [
+    O.Problem(200, 2, 16, 32, 3),             # 1-D, ragged tail block and query block
+    O.Problem(300, 2, 16, 32, 2, forced=2),   # reference-frame blocks always kept
+    O.Problem(246, 2, 16, 32, 3, forced=1, grid_h=10, grid_w=12, special=3, win_h=4),  # 2-D
+])
+def test_bwd_equals_autograd_of_the_forward(pb):
+    """Gradients equal torch autograd of the forward restated in torch ops, and that restatement's
+    output equals the oracle's own forward (exact pooling, the oracle's selection lists)."""
+    q, k, v, g, dout = _bwd_inputs(pb, 71)
+    kc = O.pool(pb, k, exact=True)
+    vc = O.pool(pb, v, exact=True)
+    fwd = O.sparse_attn(pb, q, k, v, g, pooled=(kc, vc))
+    leaves = _leaves(q, k, v, g)
+    out = _torch_path(pb, *leaves, fwd.idx)
+    np.testing.assert_allclose(out.detach().numpy(), fwd.out, rtol=0, atol=1e-12)
+    (out * torch.from_numpy(dout)).sum().backward()
+    gr = O.backward(pb, q, k, v, g, fwd.idx, dout, kc=kc, vc=vc)
+    for name, mine, ref in zip(["dq", "dk", "dv", "dgates"], [gr.dq, gr.dk, gr.dv, gr.dgates],
+                               leaves):
+        np.testing.assert_allclose(mine, ref.grad.numpy(), rtol=0, atol=1e-11, err_msg=name)
+
+
+def test_bwd_directional_finite_differences():
+    """<grad, u> equals the central difference of <dout, out> along a random direction u of all
+    four inputs at once (no autograd anywhere)."""
+    pb = O.Problem(246, 2, 16, 32, 3, forced=1, grid_h=10, grid_w=12, special=3, win_h=4)
+    q, k, v, g, dout = _bwd_inputs(pb, 83)
+    fwd = O.sparse_attn(pb, q, k, v, g, pooled=(O.pool(pb, k, exact=True), O.pool(pb, v, True)))
+    gr, _, _ = _bwd(pb, q, k, v, g, fwd.idx, dout)
+    x = [torch.from_numpy(values_of(q)), torch.from_numpy(values_of(k)),
+         torch.from_numpy(values_of(v)), torch.from_numpy(g.astype(np.float64))]
+    gen = torch.Generator().manual_seed(5)
+    u = [torch.randn(a.shape, generator=gen, dtype=torch.float64) for a in x]
+    D = torch.from_numpy(dout)
+    eps = 1e-5
+
+    def f(sign):
+        with torch.no_grad():
+            return float((_torch_path(pb, *[a + sign * eps * b for a, b in zip(x, u)], fwd.idx)
+                          * D).sum())
+
+    fd = (f(1) - f(-1)) / (2 * eps)
+    an = sum(float((torch.from_numpy(m) * b).sum())
+             for m, b in zip([gr.dq, gr.dk, gr.dv, gr.dgates], u))
+    assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (fd, an)
+
+
+def test_bwd_selection_over_every_block_equals_library_attention_backward():
+    """Gate logits (-inf, +inf) switch the compressed branch off; with every key block selected
+    the path is dense attention, so dQ, dK, dV are torch SDPA's own fp64 backward and the gate
+    gradients vanish."""
+    for pb in [O.Problem(200, 2, 16, 32, 7), O.Problem(200, 2, 16, 32, 5, forced=2)]:
+        g = np.zeros((pb.L, pb.H, 2), np.float32)
+        g[..., 0], g[..., 1] = -np.inf, np.inf
+        q, k, v, g, dout = _bwd_inputs(pb, 91, gates=g)
+        idx = np.broadcast_to(np.arange(pb.nb, dtype=np.int32)[::-1], (pb.H, pb.nqb, pb.nb))
+        gr, _, _ = _bwd(pb, q, k, v, g, idx, dout)
+        tq, tk, tv = [torch.tensor(values_of(a)).permute(1, 0, 2)[None].requires_grad_()
+                      for a in (q, k, v)]
+        o = F.scaled_dot_product_attention(tq, tk, tv, scale=pb.softmax_scale)
+        (o[0].permute(1, 0, 2) * torch.from_numpy(dout)).sum().backward()
+        for mine, ref in zip([gr.dq, gr.dk, gr.dv], [tq, tk, tv]):
+            np.testing.assert_allclose(mine, ref.grad[0].permute(1, 0, 2).numpy(), rtol=0,
+                                       atol=1e-11)
+        assert np.all(gr.dgates == 0.0)
+
+
+@pytest.mark.parametrize("L", [256, 200])
+def test_bwd_compressed_branch_equals_library_attention_over_pooled_keys(L):
+    """Gate logits (+inf, -inf) leave the compressed branch alone: dense attention of every query
+    over the block means, whose gradient reaches each token through the mean (torch autograd
+    of SDPA over torch-pooled K/V; a ragged last block is the mean of its own tokens)."""
+    pb = O.Problem(L, 2, 16, 32, 2)
+    g = np.zeros((pb.L, pb.H, 2), np.float32)
+    g[..., 0], g[..., 1] = np.inf, -np.inf
+    q, k, v, g, dout = _bwd_inputs(pb, 97, gates=g)
+    idx = np.zeros((pb.H, pb.nqb, pb.nsel), np.int32) + np.arange(pb.nsel, dtype=np.int32)
+    gr, _, _ = _bwd(pb, q, k, v, g, idx, dout)
+    tq, tk, tv = [torch.tensor(values_of(a), requires_grad=True) for a in (q, k, v)]
+    kc = torch.stack([c.mean(0) for c in torch.split(tk, pb.block)])
+    vc = torch.stack([c.mean(0) for c in torch.split(tv, pb.block)])
+    o = F.scaled_dot_product_attention(tq.permute(1, 0, 2)[None], kc.permute(1, 0, 2)[None],
+                                       vc.permute(1, 0, 2)[None], scale=pb.softmax_scale)
+    (o[0].permute(1, 0, 2) * torch.from_numpy(dout)).sum().backward()
+    for mine, ref in zip([gr.dq, gr.dk, gr.dv], [tq, tk, tv]):
+        np.testing.assert_allclose(mine, ref.grad.numpy(), rtol=0, atol=1e-11)
+
+
+def test_bwd_key_gradients_sum_to_zero_and_value_gradients_conserve_mass():
+    """Softmax weights sum to one in both branches and pooling keeps sums, so per head the key
+    gradients sum to zero over all tokens (a common shift of every key changes nothing) and the
+    value gradients sum to sum_r (sigmoid(g0) + sigmoid(g1)) dout_r."""
+    pb = O.Problem(246, 3, 16, 32, 3, forced=1, grid_h=10, grid_w=12, special=3, win_h=4)
+    q, k, v, g, dout = _bwd_inputs(pb, 101)
+    fwd = O.sparse_attn(pb, q, k, v, g)
+    gr, _, _ = _bwd(pb, q, k, v, g, fwd.idx, dout)
+    assert np.abs(gr.dk.sum(0)).max() < 1e-11
+    s = 1 / (1 + np.exp(-g.astype(np.float64)))
+    np.testing.assert_allclose(gr.dv.sum(0), ((s[..., :1] + s[..., 1:]) * dout).sum(0), rtol=0,
+                               atol=1e-11)
+
+
+def test_bwd_equal_values_leave_no_attention_gradient():
+    """When every value row of a head is the same vector w, both branch outputs are w whatever
+    the weights: dQ = dK = 0 and the gate gradients are sigmoid'(g) <dout, w>."""
+    pb = O.Problem(200, 2, 16, 32, 3, forced=1)
+    q, k, _, g, dout = _bwd_inputs(pb, 107)
+    w = rand_bits((1, pb.H, pb.d), 109, 1.0)
+    v = np.ascontiguousarray(np.broadcast_to(w, (pb.L, pb.H, pb.d)))
+    fwd = O.sparse_attn(pb, q, k, v, g)
+    gr, _, _ = _bwd(pb, q, k, v, g, fwd.idx, dout)
+    assert np.abs(gr.dq).max() < 1e-12 and np.abs(gr.dk).max() < 1e-12
+    s = 1 / (1 + np.exp(-g.astype(np.float64)))
+    yw = (dout * values_of(w)).sum(-1)
+    np.testing.assert_allclose(gr.dgates, s * (1 - s) * yw[..., None], rtol=0, atol=1e-12)
+
+
+def test_bwd_rejects_an_out_of_range_index():
+    pb = O.Problem(200, 1, 16, 32, 2)
+    q, k, v, g, dout = _bwd_inputs(pb, 113)
+    idx = np.zeros((pb.H, pb.nqb, pb.nsel), np.int32)
+    idx[0, 1, 1] = pb.nb
+    with pytest.raises(AssertionError, match="-3"):
+        _bwd(pb, q, k, v, g, idx, dout)
