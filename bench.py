@@ -30,6 +30,10 @@ Other workloads:
 
 --single-kernel runs the compressed branch, top-k and selection as one kernel.
 
+--backward also times s3r_sparse_attn_bwd (the gradients of q, k, v and the gate logits, with the
+forward's selection lists held fixed) on the same inputs, and adds a "backward" object: its
+tokens/s, algorithmic TFLOP/s, per-stage times and the roofline of its dominant kernel.
+
 --impl reference times the CPU oracle (the only other implementation of this method) on bounded
 samples of the same workload and prints the same line with "impl": "reference".
 """
@@ -158,6 +162,77 @@ def algorithmic(cfg):
             "topk": ("hbm", H * nqb * (nb * 4.0 + k * 4.0)),                  # bytes
             "sel_combine": ("tensor", 0.0 if single else sel_flops),          # flops
         },
+    }
+
+
+def algorithmic_bwd(cfg):
+    """Algorithmic work of the backward: the five products of softmax attention's gradient
+    (S, dP, dQ, dK, dV: 10 L n d H FLOPs over n keys) for both branches, and per stage what its
+    kernel computes of them (the dq kernel forms S, dP and dQ; the key-side kernels S, dP, dK and
+    dV); the recompute stage is the forward."""
+    L, H, d = cfg.L, cfg.H, cfg.d
+    n_cmp = cfg.nb
+    n_sel = (getattr(cfg, "forced", 0) + cfg.topk) * cfg.block
+    fwd = algorithmic(cfg)["flops"]
+    return {
+        "flops": 10.0 * L * H * d * (n_cmp + n_sel),
+        "stage_work": {
+            "recompute": ("tensor", fwd),
+            # dout, O_cmp, O_sel read; the statistics and dgates written
+            "prep": ("hbm", L * H * (64 * 2 + 2 * 64 * 4 + 6 * 4 + 2 * 4.0)),
+            "dq": ("tensor", 6.0 * L * H * d * (n_cmp + n_sel)),
+            "dkv_cmp": ("tensor", 8.0 * L * H * d * n_cmp),
+            "dkv_sel": ("tensor", 8.0 * L * H * d * n_sel),
+        },
+    }
+
+
+def time_backward(args, cfg, q, k, v, gates, idx, dev, barrier, peaks):
+    """K timed calls of s3r_sparse_attn_bwd after W warm-up calls (a seeded bf16 dout)."""
+    import torch
+
+    from sparse_global_attention_s3r_b200 import _lib, api
+
+    g = torch.Generator(device=dev).manual_seed(99)
+    dout = torch.randn(q.shape, generator=g, device=dev).to(torch.bfloat16)
+    ws = torch.empty(api.bwd_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    grads = (*(torch.empty(q.shape, dtype=torch.float32, device=dev) for _ in range(3)),
+             torch.empty(gates.shape, dtype=torch.float32, device=dev))
+    for _ in range(args.warmup):
+        api.sparse_attn_bwd(cfg, q, k, v, gates, idx, dout, ws, grads=grads)
+    torch.cuda.synchronize()
+    evs = [api.StageEvents(_lib.BWD_STAGES) for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    n0 = _lib.kernel_launches()
+    e0.record()
+    for s in range(args.steps):
+        api.sparse_attn_bwd(cfg, q, k, v, gates, idx, dout, ws, stage_events=evs[s], grads=grads)
+    e1.record()
+    torch.cuda.synchronize()
+    launches = _lib.kernel_launches() - n0
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    stage_ms = {n: statistics.mean(e.stage_ms()[n] for e in evs) for n in _lib.BWD_STAGES}
+    work = algorithmic_bwd(cfg)
+    stages = {}
+    for n, (b_, u_) in work["stage_work"].items():
+        s_ = stage_ms[n] / 1e3
+        stages[n] = {"ms": stage_ms[n],
+                     ("GB/s" if b_ == "hbm" else "TFLOP/s"): u_ / s_ / (1e9 if b_ == "hbm" else 1e12)}
+    dom = max(("dq", "dkv_cmp", "dkv_sel"), key=stage_ms.get)
+    ach = work["stage_work"][dom][1] / (stage_ms[dom] / 1e3) / 1e12
+    del ws, grads, dout
+    return {
+        "ms_per_step": ms, "tokens_per_s": cfg.L / (ms / 1e3),
+        "tflops": work["flops"] / (ms / 1e3) / 1e12, "stage_ms": stages,
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": ach,
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": ach / peaks["bf16_tflops_sustained"],
+                     "peak_source": peaks["source"] + " sustained bf16", "traffic": None},
+        "gpu_launches": launches,
+        "how": "s3r_sparse_attn_bwd on the forward's own selection lists and a seeded bf16 dout; "
+               "each call recomputes the forward (stage 'recompute')",
     }
 
 
@@ -375,6 +450,8 @@ def run_native(args, wl):
     barrier()
     ms_max = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
     stage_ms = {n: statistics.mean(e.stage_ms()[n] for e in stage_ev) for n in _lib.STAGES}
+    bwd = (time_backward(args, cfg, q, k, v, gates, sa.idx, dev, barrier, load_peaks())
+           if args.backward else None)
 
     # end to end through the public API from pinned host memory: every step copies all of its
     # inputs in and its output out. HostPipeline overlaps the copy-in of step i+1 and the
@@ -514,6 +591,8 @@ def run_native(args, wl):
         "dense_context": dense,
         "clocks": clocks.summary(),
     }
+    if bwd is not None:
+        line["backward"] = bwd
     print(json.dumps(line), flush=True)
 
 
@@ -587,6 +666,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--single-kernel", action="store_true",
                     help="run the compressed branch, top-k and selection as one kernel (k <= 32)")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward (s3r_sparse_attn_bwd) on the same inputs")
     ap.add_argument("--no-dense-context", action="store_true",
                     help="skip timing dense attention (torch SDPA) on a sample of query rows")
     ap.add_argument("--dense-rows", type=int, default=16384,

@@ -111,7 +111,9 @@ typedef struct {
   void* const* stage_events; /* optional: S3R_NUM_STAGES + 1 cudaEvent_t handles that
                                 s3r_sparse_attn_fwd records on `stream` at the stage boundaries
                                 (before stage 0, after each stage), for per-stage timing with
-                                cudaEventElapsedTime; ignored by the single-step entry points */
+                                cudaEventElapsedTime; s3r_sparse_attn_bwd records
+                                S3R_NUM_BWD_STAGES + 1 of them the same way; ignored by the
+                                single-step entry points */
 } s3r_params;
 
 /* Stages of s3r_sparse_attn_fwd, in launch order (one kernel each). */
@@ -121,6 +123,14 @@ typedef struct {
                                    where the compressed stage selects the blocks on the fly */
 #define S3R_STAGE_SEL_COMBINE 3 /* selection attention fused with the gated combine */
 #define S3R_NUM_STAGES 4
+
+/* Stages of s3r_sparse_attn_bwd, in launch order. */
+#define S3R_BWD_STAGE_RECOMPUTE 0 /* the forward again: pooling, both branches with their lse */
+#define S3R_BWD_STAGE_PREP 1      /* D and gate gradients; the inverse of the selection lists */
+#define S3R_BWD_STAGE_DQ 2        /* dq of both branches (one kernel) */
+#define S3R_BWD_STAGE_DKV_CMP 3   /* dKc, dVc of the block summaries */
+#define S3R_BWD_STAGE_DKV_SEL 4   /* dk, dv of the selected tokens, plus dKc / n_j, dVc / n_j */
+#define S3R_NUM_BWD_STAGES 5
 
 /* Largest nb (key blocks) this build accepts; beyond it calls return S3R_ERR_UNSUPPORTED. */
 #define S3R_MAX_BLOCKS 49152
@@ -206,6 +216,32 @@ s3r_status s3r_gate_combine(const s3r_params* params, const float* o_cmp, const 
 s3r_status s3r_sparse_attn_fwd(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,
                                const s3r_bf16* v, const float* gate_logits, s3r_bf16* out,
                                int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                               s3r_stream stream);
+
+/* Backward of the whole path (Speed3R is trained end to end: arXiv abstract). Given the upstream
+ * gradient dout of s3r_sparse_attn_fwd's output, the gradients of q, k, v and of the gate logits.
+ * The selection lists are held fixed: a top-k passes no gradient, so idx is an input (the lists
+ * the forward call wrote to idx_out for the same q, k, v). The bf16 rounding of the pooled K/V
+ * passes the gradient unchanged: every token of key block j receives dKc[j] / n_j (n_j = its
+ * token count), and likewise for V. Per head, with P = softmax(scale q K^T) of each branch and
+ * dO = sigmoid(gate) dout:
+ *   dS = P (dO V^T - <dO, O>),  dq = scale dS K,  dK = scale dS^T q,  dV = P^T dO
+ * summed over both branches;  dgates[..., c] = sigmoid'(logit c) <dout, O_branch c>.
+ * The call recomputes the forward (pooling, both branches with their softmax normalisers) in
+ * the workspace, then runs the backward kernels; nothing is kept between calls.
+ *   q, k, v     [L, H, d] bf16; gate_logits [L, H, 2] fp32; dout [L, H, d] bf16 (read)
+ *   idx         [H, nqb, forced + topk] int32 (read): entries distinct within a list; entries
+ *               outside [0, nb) contribute nothing
+ *   dq, dk, dv  [L, H, d] fp32 (written); dgates [L, H, 2] fp32 (written)
+ *   workspace   device buffer of at least s3r_bwd_workspace_bytes(params) bytes, 256-byte aligned.
+ * Returns S3R_ERR_UNSUPPORTED when H * nb * block exceeds 2^31 - 1 (row coordinates of the
+ * slot-order K/V copies). The order in which query blocks add into one key block's dK, dV
+ * follows an atomic fill and may differ between calls (fp32 rounding only). */
+size_t s3r_bwd_workspace_bytes(const s3r_params* params);
+s3r_status s3r_sparse_attn_bwd(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,
+                               const s3r_bf16* v, const float* gate_logits, const int32_t* idx,
+                               const s3r_bf16* dout, float* dq, float* dk, float* dv,
+                               float* dgates, void* workspace, size_t workspace_bytes,
                                s3r_stream stream);
 
 /* Size of the scratch array built into the library for s3r_sparse_attn_fwd_static (32 MiB). */

@@ -26,6 +26,7 @@ S3R_FLAG_SINGLE_KERNEL = 0x4
 S3R_MAX_BLOCKS = 49152
 S3R_STATIC_WORKSPACE_BYTES = 32 << 20
 STAGES = ("pool", "cmp", "topk", "sel_combine")  # S3R_STAGE_* order
+BWD_STAGES = ("recompute", "prep", "dq", "dkv_cmp", "dkv_sel")  # S3R_BWD_STAGE_* order
 
 # every function the header declares, with its ctypes signature
 _P = ctypes.c_void_p
@@ -44,6 +45,8 @@ EXPORTS = {
     "s3r_gate_combine": (ctypes.c_int, [_P, _P, _P, _P, _P, _P]),
     "s3r_sparse_attn_fwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "s3r_sparse_attn_fwd_static": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "s3r_bwd_workspace_bytes": (ctypes.c_size_t, [_P]),
+    "s3r_sparse_attn_bwd": (ctypes.c_int, [_P] * 12 + [ctypes.c_size_t, _P]),
 }
 
 

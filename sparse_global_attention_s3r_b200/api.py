@@ -8,7 +8,8 @@ contiguous, with the layouts of include/s3r.h:
     k_cmp, v_cmp [nb, H, 64] bf16         lse    [H, L] fp32
     o_cmp, o_sel [L, H, 64] fp32          scores [H, nqb, nb] fp32
     idx          [H, nqb, forced + topk] int32
-    out          [L, H, 64] bf16
+    out, dout    [L, H, 64] bf16
+    dq, dk, dv   [L, H, 64] fp32          dgates [L, H, 2] fp32
 nb counts the key blocks of the configured geometry (Config.nb), nqb = ceil(L / 64).
 """
 from __future__ import annotations
@@ -168,10 +169,13 @@ def alloc_workspace(cfg: Config, device=None) -> torch.Tensor:
 
 
 class StageEvents:
-    """S3R_NUM_STAGES + 1 CUDA events that s3r_sparse_attn_fwd records at its stage boundaries."""
+    """CUDA events that s3r_sparse_attn_fwd (S3R_NUM_STAGES + 1) or, with stages=
+    _lib.BWD_STAGES, s3r_sparse_attn_bwd (S3R_NUM_BWD_STAGES + 1) records at its stage
+    boundaries."""
 
-    def __init__(self):
-        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(_lib.STAGES) + 1)]
+    def __init__(self, stages=_lib.STAGES):
+        self.stages = stages
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
         for e in self.events:  # torch creates the underlying event on first record
             e.record()
         self.handles = (ctypes.c_void_p * len(self.events))(
@@ -180,7 +184,7 @@ class StageEvents:
     def stage_ms(self) -> dict:
         """Milliseconds of each stage of the last recorded call (events must have completed)."""
         return {n: self.events[i].elapsed_time(self.events[i + 1])
-                for i, n in enumerate(_lib.STAGES)}
+                for i, n in enumerate(self.stages)}
 
 
 def sparse_attn_fwd(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
@@ -222,6 +226,67 @@ def sparse_attn_fwd_static(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: tor
     _lib.call("s3r_sparse_attn_fwd_static", ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
               _ptr(gates), _ptr(out), _ptr(idx_out), _stream())
     return out
+
+
+def bwd_workspace_bytes(cfg: Config) -> int:
+    p = cfg.params()
+    n = int(_lib.load().s3r_bwd_workspace_bytes(ctypes.byref(p)))
+    if n == 0:
+        raise _lib.S3RError("s3r_bwd_workspace_bytes", _lib.S3R_ERR_INVALID_ARG)
+    return n
+
+
+def sparse_attn_bwd(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                    gates: torch.Tensor, idx: torch.Tensor, dout: torch.Tensor,
+                    workspace: Optional[torch.Tensor] = None,
+                    dev_status: Optional[torch.Tensor] = None,
+                    stage_events: Optional[StageEvents] = None, grads=None):
+    """Gradients of the whole path for the upstream gradient dout, with the selection lists idx
+    (the forward's idx_out) held fixed: returns dq, dk, dv [L,H,d] fp32 and dgates [L,H,2] fp32.
+
+    grads: optional preallocated (dq, dk, dv, dgates) to write into; stage_events: a
+    StageEvents(_lib.BWD_STAGES) that the call records at its stage boundaries."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
+        _need(t, n, _lhd(cfg), torch.bfloat16)
+    _need(gates, "gates", (cfg.L, cfg.H, 2), torch.float32)
+    _need(idx, "idx", (cfg.H, cfg.nqb, cfg.nsel), torch.int32)
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_bytes(cfg), dtype=torch.uint8, device=q.device)
+    if grads is None:
+        grads = (*(torch.empty(_lhd(cfg), dtype=torch.float32, device=q.device) for _ in range(3)),
+                 torch.empty((cfg.L, cfg.H, 2), dtype=torch.float32, device=q.device))
+    dq, dk, dv, dgates = grads
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, n, _lhd(cfg), torch.float32)
+    _need(dgates, "dgates", (cfg.L, cfg.H, 2), torch.float32)
+    p = cfg.params(dev_status, None if stage_events is None else stage_events.handles)
+    _lib.call("s3r_sparse_attn_bwd", ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(gates),
+              _ptr(idx), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgates), _ptr(workspace),
+              workspace.numel(), _stream())
+    return dq, dk, dv, dgates
+
+
+class SparseAttentionFunction(torch.autograd.Function):
+    """autograd wrapper: forward = sparse_attn_fwd (bf16 out), backward = sparse_attn_bwd.
+
+    Gradients are returned in the inputs' dtypes (bf16 for q, k, v; fp32 for the gate logits).
+    The top-k selection passes no gradient."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, gates, cfg: Config):
+        idx = torch.empty((cfg.H, cfg.nqb, cfg.nsel), dtype=torch.int32, device=q.device)
+        out = sparse_attn_fwd(cfg, q, k, v, gates, idx_out=idx)
+        ctx.cfg = cfg
+        ctx.save_for_backward(q, k, v, gates, idx)
+        ctx.mark_non_differentiable(idx)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, gates, idx = ctx.saved_tensors
+        dq, dk, dv, dg = sparse_attn_bwd(ctx.cfg, q, k, v, gates, idx,
+                                         dout.to(torch.bfloat16).contiguous())
+        return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), dg, None
 
 
 def read_device_status(word: torch.Tensor) -> int:

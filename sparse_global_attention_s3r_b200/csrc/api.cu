@@ -115,6 +115,46 @@ Workspace layout(const Problem& p) {
   return w;
 }
 
+// Workspace of the backward call, every region 256-byte aligned:
+//   status | Kc | Vc | Kh | Vh (as the forward) | O_cmp, O_sel [L,H,d] f32 | lse_c, lse_s [H,L]
+//   | statistics [6][H][Lp] f32 | dKc, dVc [nb,H,d] f32 | cnt, cursor [H,nb] | off [H,nb+1]
+//   | ent [H,nqb*nsel] i32
+struct BwdWorkspace {
+  size_t status, kc, vc, kh, vh, o_cmp, o_sel, lse_c, lse_s, stats, dkc, dvc, cnt, cursor, off,
+      ent, total;
+};
+
+BwdWorkspace bwd_ws_layout(const Problem& p) {
+  BwdWorkspace w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += round256(bytes);
+    return at;
+  };
+  const BwdLayout bl = bwd_layout(p);
+  const size_t HD = static_cast<size_t>(p.H) * p.d;
+  const size_t H = static_cast<size_t>(p.H);
+  w.status = take(4);
+  w.kc = take(static_cast<size_t>(p.nb) * HD * 2);
+  w.vc = take(static_cast<size_t>(p.nb) * HD * 2);
+  w.kh = take(static_cast<size_t>(p.nb) * p.b * HD * 2);
+  w.vh = take(static_cast<size_t>(p.nb) * p.b * HD * 2);
+  w.o_cmp = take(static_cast<size_t>(p.L) * HD * 4);
+  w.o_sel = take(static_cast<size_t>(p.L) * HD * 4);
+  w.lse_c = take(H * p.L * 4);
+  w.lse_s = take(H * p.L * 4);
+  w.stats = take(6 * H * bl.Lp * 4);
+  w.dkc = take(static_cast<size_t>(p.nb) * HD * 4);
+  w.dvc = take(static_cast<size_t>(p.nb) * HD * 4);
+  w.cnt = take(H * p.nb * 4);
+  w.cursor = take(H * p.nb * 4);
+  w.off = take(H * (p.nb + 1) * 4);
+  w.ent = take(H * bl.per_head * 4);
+  w.total = off;
+  return w;
+}
+
 }  // namespace
 
 size_t fused_workspace_bytes(const s3r_params* params) {
@@ -273,6 +313,56 @@ s3r_status s3r_gate_combine(const s3r_params* params, const float* o_cmp, const 
   if (!aligned16(o_cmp) || !aligned16(o_sel) || !aligned16(gate_logits) || !aligned16(out))
     return S3R_ERR_INVALID_ARG;
   return launched(launch_gate_combine(p, o_cmp, o_sel, gate_logits, out, stream));
+}
+
+size_t s3r_bwd_workspace_bytes(const s3r_params* params) {
+  Problem p;
+  if (derive(params, &p) != S3R_OK) return 0;
+  return bwd_ws_layout(p).total;
+}
+
+s3r_status s3r_sparse_attn_bwd(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,
+                               const s3r_bf16* v, const float* gate_logits, const int32_t* idx,
+                               const s3r_bf16* dout, float* dq, float* dk, float* dv,
+                               float* dgates, void* workspace, size_t workspace_bytes,
+                               s3r_stream stream) {
+  Problem p;
+  s3r_status st = derive(params, &p);
+  if (st != S3R_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate_logits) ||
+      !aligned16(idx) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv) || !aligned16(dgates))
+    return S3R_ERR_INVALID_ARG;
+  if (!use_head_major(p)) return S3R_ERR_UNSUPPORTED;
+  const BwdWorkspace w = bwd_ws_layout(p);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < w.total)
+    return S3R_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  auto f32 = [&](size_t at) { return reinterpret_cast<float*>(base + at); };
+  auto i32 = [&](size_t at) { return reinterpret_cast<int32_t*>(base + at); };
+  auto b16 = [&](size_t at) { return reinterpret_cast<uint16_t*>(base + at); };
+  uint32_t* status = reinterpret_cast<uint32_t*>(base + w.status);
+  if (!p.status) p.status = status;
+  void* const* ev = params->stage_events;
+  if (cudaMemsetAsync(status, 0, 4, stream) != cudaSuccess) return S3R_ERR_CUDA;
+  if (ev && cudaEventRecord(static_cast<cudaEvent_t>(ev[0]), stream) != cudaSuccess)
+    return S3R_ERR_CUDA;
+  // the forward again, keeping what the backward needs
+  if ((st = launched(launch_pool_kv(p, k, v, b16(w.kc), b16(w.vc), b16(w.kh), b16(w.vh),
+                                    stream))) != S3R_OK)
+    return st;
+  if ((st = launched(launch_cmp_attn_tc(p, q, b16(w.kc), b16(w.vc), f32(w.lse_c), f32(w.o_cmp),
+                                        nullptr, nullptr, stream))) != S3R_OK)
+    return st;
+  if ((st = launched(launch_sel_attn(p, q, b16(w.kh), b16(w.vh), true, idx, f32(w.o_sel), nullptr,
+                                     nullptr, nullptr, stream, f32(w.lse_s)))) != S3R_OK)
+    return st;
+  if (ev && cudaEventRecord(static_cast<cudaEvent_t>(ev[1]), stream) != cudaSuccess)
+    return S3R_ERR_CUDA;
+  BwdBuffers b{q, dout, b16(w.kc), b16(w.vc), b16(w.kh), b16(w.vh), gate_logits, f32(w.o_cmp),
+               f32(w.o_sel), f32(w.lse_c), f32(w.lse_s), idx, f32(w.stats), f32(w.dkc),
+               f32(w.dvc), i32(w.cnt), i32(w.cursor), i32(w.off), i32(w.ent), dq, dk, dv, dgates};
+  return launched(launch_bwd(p, b, stream, ev));
 }
 
 s3r_status s3r_sparse_attn_fwd(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,

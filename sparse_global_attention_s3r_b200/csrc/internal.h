@@ -44,14 +44,38 @@ cudaError_t launch_fused_tc(const Problem& p, const uint16_t* q, const uint16_t*
                             const float* gates, uint16_t* out, int32_t* idx, cudaStream_t st);
 cudaError_t launch_topk(const Problem& p, const float* scores, int32_t* idx, cudaStream_t st);
 // o_sel != nullptr: write the selection output (fp32). Otherwise fuse the gated combine:
-// read o_cmp and gates and write out (bf16).
+// read o_cmp and gates and write out (bf16). lse (nullable): [H, L] natural log of each row's
+// softmax normaliser over its selected tokens.
 // k, v: [L, H, 64] token-major, or (head_major) the [H, nb*b, 64] copies of launch_pool_kv.
 cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t* k,
                             const uint16_t* v, bool head_major, const int32_t* idx, float* o_sel,
                             const float* o_cmp, const float* gates, uint16_t* out,
-                            cudaStream_t st);
+                            cudaStream_t st, float* lse = nullptr);
 cudaError_t launch_gate_combine(const Problem& p, const float* o_cmp, const float* o_sel,
                                 const float* gates, uint16_t* out, cudaStream_t st);
+
+// Backward of the whole path (bwd.cu). The caller has run the pooling (kc, vc and the slot-order
+// copies kh, vh), the compressed branch (o_cmp, lse_c) and the selection branch (o_sel, lse_s)
+// on the same inputs and selection lists idx.
+struct BwdLayout {
+  int64_t Lp;        // rows of the statistics planes: L rounded up to whole 128-row tiles
+  int64_t per_head;  // entries of one head's selection lists: nqb * nsel
+};
+BwdLayout bwd_layout(const Problem& p);
+struct BwdBuffers {
+  const uint16_t *q, *dout, *kc, *vc, *kh, *vh;  // bf16
+  const float *gates, *o_cmp, *o_sel, *lse_c, *lse_s;
+  const int32_t* idx;     // [H, nqb, nsel]
+  float* stats;           // [6][H][Lp] scratch
+  float *dkc, *dvc;       // [nb, H, 64] scratch
+  int32_t *cnt, *cursor;  // [H, nb] scratch
+  int32_t* off;           // [H, nb + 1] scratch
+  int32_t* ent;           // [H, per_head] scratch
+  float *dq, *dk, *dv;    // [L, H, 64] outputs
+  float* dgates;          // [L, H, 2] output
+};
+// ev (nullable): the call's stage events; records events 2..5 (see S3R_BWD_STAGE_*).
+cudaError_t launch_bwd(const Problem& p, const BwdBuffers& b, cudaStream_t st, void* const* ev);
 
 void count_launch();
 

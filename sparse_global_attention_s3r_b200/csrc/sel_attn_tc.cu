@@ -82,6 +82,7 @@ struct SelArgs {
   uint32_t flags;
   uint32_t* status;
   uint64_t limit_ns;
+  float* lse;  // [H, L] natural log of each row's softmax normaliser, or null
 };
 
 __device__ __forceinline__ void raise_abort(volatile int* abort, uint32_t* status) {
@@ -440,6 +441,17 @@ __global__ void __maxnreg__(128)
       const int which = lane >> 3;
       const float rs = which == 0 ? s0 : which == 1 ? s1 : which == 2 ? s2 : s3;
       const float inv = rs > 0.f ? 1.f / rs : 0.f;
+      if (a.lse) {  // lse = (reference max * scale * log2 e + log2 of the row sum) * ln 2
+        const float m0 = __shfl_sync(0xffffffffu, mr[0], src);
+        const float m1 = __shfl_sync(0xffffffffu, mr[1], src);
+        const float m2 = __shfl_sync(0xffffffffu, mr[2], src);
+        const float m3 = __shfl_sync(0xffffffffu, mr[3], src);
+        const float mrow = which == 0 ? m0 : which == 1 ? m1 : which == 2 ? m2 : m3;
+        const int64_t lrow = q0 + g * 32 + lane;
+        if (lrow < a.L)
+          a.lse[static_cast<int64_t>(h) * a.L + lrow] =
+              rs > 0.f ? (mrow * sl2 + log2f(rs)) * kLn2 : -INFINITY;
+      }
       tc_fence_after();
       uint32_t o[2][32];
       tmem_ld32(tl0 + kColO, o[0]);
@@ -496,7 +508,7 @@ __global__ void __maxnreg__(128)
 cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t* k,
                             const uint16_t* v, bool head_major, const int32_t* idx, float* o_sel,
                             const float* o_cmp, const float* gates, uint16_t* out,
-                            cudaStream_t st) {
+                            cudaStream_t st, float* lse) {
   // rows per K/V box: a run of slots that are consecutive rows in memory (32 for b = 32, else
   // 64; gathers of 2-D windows from K and V themselves: one window row, at most 64)
   int box = p.b < kStep ? p.b : kStep;
@@ -523,7 +535,7 @@ cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t*
   SelArgs a{idx, o_sel, o_cmp, gates, out, p.L, p.nb, p.nqb, p.geo, box, head_major ? 1 : 0,
             head_major ? 0 : 64, head_major ? static_cast<int>(Lp) : 0, p.H, p.b, lb, p.nsel,
             static_cast<int>((ntok + kStep - 1) / kStep), p.scale_log2, p.flags, p.status,
-            (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull};
+            (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull, lse};
   dim3 grid(static_cast<unsigned>((p.L + kBM - 1) / kBM), p.H);
   sel_attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
   count_launch();

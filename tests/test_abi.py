@@ -24,7 +24,7 @@ def declared_functions():
 def test_library_exports_every_declared_function():
     lib = _lib.load()
     names = declared_functions()
-    assert len(names) == 14, names
+    assert len(names) == 16, names
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_lib.EXPORTS)
@@ -81,7 +81,9 @@ def test_bad_sizes_are_rejected_by_every_entry_point(kw, want):
     assert lib.s3r_sel_attn(p, A16, A16, A16, A16, A16, s) == want
     assert lib.s3r_gate_combine(p, A16, A16, A16, A16, s) == want
     assert lib.s3r_sparse_attn_fwd(p, A16, A16, A16, A16, A16, None, A256, 1 << 40, s) == want
+    assert lib.s3r_sparse_attn_bwd(p, *[A16] * 10, A256, 1 << 40, s) == want
     assert lib.s3r_workspace_bytes(p) == 0
+    assert lib.s3r_bwd_workspace_bytes(p) == 0
 
 
 def test_null_and_misaligned_pointers_are_rejected():
@@ -95,6 +97,11 @@ def test_null_and_misaligned_pointers_are_rejected():
         assert lib.s3r_sel_attn(p, A16, A16, A16, bad, A16, None) == _lib.S3R_ERR_INVALID_ARG
         assert lib.s3r_gate_combine(p, A16, A16, bad, A16, None) == _lib.S3R_ERR_INVALID_ARG
         assert lib.s3r_sparse_attn_fwd(p, A16, bad, A16, A16, A16, None, A256, 1 << 40, None) == _lib.S3R_ERR_INVALID_ARG
+    for i in range(10):  # every array of the backward is required and 16-byte aligned
+        for bad in (None, A8):
+            args = [A16] * 10
+            args[i] = bad
+            assert lib.s3r_sparse_attn_bwd(p, *args, A256, 1 << 40, None) == _lib.S3R_ERR_INVALID_ARG
     # idx_out is optional but must be aligned when given
     assert lib.s3r_sparse_attn_fwd(p, A16, A16, A16, A16, A16, A8, A256, 1 << 40, None) == _lib.S3R_ERR_INVALID_ARG
     # a misaligned status word
@@ -113,6 +120,29 @@ def test_workspace_checks():
     assert lib.s3r_sparse_attn_fwd(p, A16, A16, A16, A16, A16, None, A256, need - 1, None) == _lib.S3R_ERR_WORKSPACE
     assert lib.s3r_sparse_attn_fwd(p, A16, A16, A16, A16, A16, None, A16_NOT256, need, None) == _lib.S3R_ERR_WORKSPACE
     assert lib.s3r_workspace_status_word(A256) == A256.value
+    need = lib.s3r_bwd_workspace_bytes(ctypes.byref(prm))
+    for ws, n in ((None, need), (A256, need - 1), (A16_NOT256, need)):
+        assert lib.s3r_sparse_attn_bwd(p, *[A16] * 10, ws, n, None) == _lib.S3R_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("L,H,b,k,F", [(1024, 2, 64, 4, 0), (1374000, 16, 64, 32, 0),
+                                       (43968, 16, 64, 16, 22), (1, 1, 128, 1, 0)])
+def test_bwd_workspace_size_matches_layout(L, H, b, k, F):
+    cfg = api.Config(L=L, H=H, block=b, topk=k, forced=F)
+    nb, nqb, d = cfg.nb, cfg.nqb, 64
+    Lp = (L + 127) // 128 * 128
+    want = (r256(4) + 2 * r256(nb * H * d * 2) + 2 * r256(nb * b * H * d * 2)
+            + 2 * r256(L * H * d * 4) + 2 * r256(H * L * 4) + r256(6 * H * Lp * 4)
+            + 2 * r256(nb * H * d * 4) + 2 * r256(H * nb * 4) + r256(H * (nb + 1) * 4)
+            + r256(H * nqb * (F + k) * 4))
+    assert api.bwd_workspace_bytes(cfg) == want
+
+
+def test_bwd_rejects_slot_copies_beyond_32_bit_rows():
+    lib = _lib.load()
+    big = _params(L=65536, H=65535, block=64, topk=1)  # H * nb * b = 65535 * 65536 > 2^31 - 1
+    assert lib.s3r_sparse_attn_bwd(ctypes.byref(big), *[A16] * 10, A256, 1 << 62,
+                                   None) == _lib.S3R_ERR_UNSUPPORTED
 
 
 def r256(x):

@@ -1,0 +1,162 @@
+"""GPU parity of the backward (s3r_sparse_attn_bwd) against the fp64 oracle's gradients.
+
+The selection lists are the forward call's own (idx_out), handed to both sides; the oracle gets
+the pooled K/V rounded to bf16 as the forward used them (its gradient passes that rounding
+straight through, like the library's).
+
+Tolerance (bf16 operands, fp32 accumulation): the kernels round g*P and dS to bf16 before the
+tensor-core products (relative error 2^-9 per element) and take D = g <dout, O> from the fp32
+forward outputs, whose own error is about 2^-8 of |V| (bf16 P in the forward products). Both
+enter every gradient at about 2^-8 relative, so each of dq, dk, dv, dgates must satisfy
+rel-L2 <= 1e-2 and max-abs <= 2e-2 * max|reference| + 1e-6 (a wrong index, sign or dropped term
+gives errors of order 1). The absolute 1e-6 covers gradients that are exactly zero: with a single
+key a branch's P is 1 and dS = P (g dP' - D) vanishes, but in fp32 the difference g dP' - D keeps
+a rounding residue of about 2^-24 |dP| (measured: 4.5e-9 in dq at L = 1).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from sparse_global_attention_s3r_b200 import api, synth
+
+from parity import f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 1e-2
+MAX_REL = 2e-2
+ABS_FLOOR = 1e-6
+
+CASES = {  # name: (L, H, b, k, forced, seed)
+    "ragged_b64": (1000, 2, 64, 5, 0, 41),
+    "ragged_b32_odd_k": (1000, 2, 32, 7, 0, 42),
+    "ragged_b128": (1300, 3, 128, 3, 0, 43),
+    "multi_tile_keys": (9000, 2, 32, 9, 0, 44),   # nb = 282: several key tiles of both kernels
+    "dense_selection": (1000, 2, 64, 16, 0, 45),  # k = nb
+    "single_partial_block": (17, 1, 64, 1, 0, 46),
+    "one_token": (1, 2, 32, 1, 0, 47),
+    "tail_of_one_row": (65, 1, 32, 3, 0, 48),
+    "forced_b32": (2000, 2, 32, 5, 6, 49),        # reference-frame blocks in every list
+    "vggt_4_views": (4 * 1374, 2, 64, 16, 22, 50),
+}
+
+WINDOWS = {  # name: (views, special, grid_h, grid_w, b, win_h, H, k, forced_views, seed)
+    "vggt_8x8_ref_view": (4, 5, 37, 37, 64, 8, 2, 12, 1, 51),
+    "odd_grid_4x8_b32": (3, 3, 10, 13, 32, 4, 2, 5, 0, 52),
+    "wide_8x16_b128": (2, 0, 20, 35, 128, 8, 2, 3, 0, 53),
+    "narrow_8x4_b32": (2, 2, 10, 13, 32, 8, 2, 3, 0, 54),  # windows narrower than 8 patches
+}
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda")
+
+
+def _dout(L, H, seed):
+    g = torch.Generator().manual_seed(1000 + seed)
+    return torch.randn((L, H, 64), generator=g).to(torch.bfloat16)
+
+
+def _check(name, got, ref):
+    got = f64(got)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    scale = float(np.abs(ref).max())
+    err = float(np.abs(got - ref).max())
+    bound = MAX_REL * scale + ABS_FLOOR
+    assert err <= bound, f"{name}: max-abs {err:.3e} > {bound:.3e}"
+    if scale > 0:
+        r = rel_l2(got, ref)
+        assert r <= REL_L2, f"{name}: rel-L2 {r:.3e}"
+
+
+def _run(dev, cfg, pb, x, seed):
+    d = {n: getattr(x, n).to(dev) for n in ("q", "k", "v", "gates")}
+    idx = torch.empty((cfg.H, cfg.nqb, cfg.nsel), dtype=torch.int32, device=dev)
+    api.sparse_attn_fwd(cfg, d["q"], d["k"], d["v"], d["gates"], idx_out=idx)
+    dout = _dout(cfg.L, cfg.H, seed)
+    dq, dk, dv, dg = api.sparse_attn_bwd(cfg, d["q"], d["k"], d["v"], d["gates"], idx,
+                                         dout.to(dev))
+    torch.cuda.synchronize()
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    ref = O.backward(pb, *bits, x.gates.numpy(), idx.cpu().numpy(), dout.double().numpy())
+    for n, got, want in (("dq", dq, ref.dq), ("dk", dk, ref.dk), ("dv", dv, ref.dv),
+                         ("dgates", dg, ref.dgates)):
+        _check(n, got, want)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_bwd_matches_oracle(dev, name):
+    L, H, b, k, F, seed = CASES[name]
+    x = synth.make_inputs(L, H, 64, b, seed)
+    _run(dev, api.Config(L=L, H=H, block=b, topk=k, forced=F),
+         O.Problem(L, H, 64, b, k, forced=F), x, seed)
+
+
+@pytest.mark.parametrize("name", list(WINDOWS))
+def test_bwd_windows_match_oracle(dev, name):
+    N, special, gh, gw, b, wh, H, k, fv, seed = WINDOWS[name]
+    L = N * (special + gh * gw)
+    geo = dict(grid_h=gh, grid_w=gw, special=special, win_h=wh)
+    F = fv * (api.Config(L=L, H=H, block=b, topk=1, **geo).nb // N)
+    x = synth.make_inputs(L, H, 64, b, seed)
+    _run(dev, api.Config(L=L, H=H, block=b, topk=k, forced=F, **geo),
+         O.Problem(L, H, 64, b, k, forced=F, **geo), x, seed)
+
+
+def test_bwd_unselected_blocks_get_only_the_pooled_gradient(dev):
+    """Selection lists naming only block 0: every other key block's tokens receive exactly their
+    share of the compressed branch's dKc / n_j (the selection branch adds nothing there)."""
+    L, H, b, k = 640, 1, 64, 1
+    x = synth.make_inputs(L, H, 64, b, 55)
+    cfg = api.Config(L=L, H=H, block=b, topk=k)
+    pb = O.Problem(L, H, 64, b, k)
+    idx = torch.zeros((H, cfg.nqb, 1), dtype=torch.int32)
+    dout = _dout(L, H, 55)
+    d = {n: getattr(x, n).to(dev) for n in ("q", "k", "v", "gates")}
+    dq, dk, dv, dg = api.sparse_attn_bwd(cfg, d["q"], d["k"], d["v"], d["gates"], idx.to(dev),
+                                         dout.to(dev))
+    torch.cuda.synchronize()
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    ref = O.backward(pb, *bits, x.gates.numpy(), idx.numpy(), dout.double().numpy())
+    for n, got, want in (("dq", dq, ref.dq), ("dk", dk, ref.dk), ("dv", dv, ref.dv)):
+        _check(n, got, want)
+    # tokens of blocks 1.. get the pooled gradient only: equal within each block
+    g = f64(dk)[b:].reshape(L // b - 1, b, H, 64)
+    assert np.abs(g - g[:, :1]).max() <= 1e-6 * max(1.0, np.abs(g).max())
+
+
+def test_bwd_autograd_function(dev):
+    """SparseAttentionFunction: forward = the fused path, backward = s3r_sparse_attn_bwd."""
+    L, H, b, k = 1000, 2, 64, 4
+    x = synth.make_inputs(L, H, 64, b, 56)
+    cfg = api.Config(L=L, H=H, block=b, topk=k)
+    leaves = [getattr(x, n).to(dev).requires_grad_() for n in ("q", "k", "v", "gates")]
+    out = api.SparseAttentionFunction.apply(*leaves, cfg)
+    dout = _dout(L, H, 56).to(dev)
+    out.backward(dout)
+    idx = torch.empty((H, cfg.nqb, cfg.nsel), dtype=torch.int32, device=dev)
+    ref_out = api.sparse_attn_fwd(cfg, *[t.detach() for t in leaves], idx_out=idx)
+    assert torch.equal(out.detach(), ref_out)
+    dq, dk, dv, dg = api.sparse_attn_bwd(cfg, *[t.detach() for t in leaves], idx, dout)
+    # two backward calls may add query blocks into a key block in different orders (atomic
+    # fill), so the bf16 casts may differ by one rounding step
+    for leaf, want in zip(leaves, (dq, dk, dv, dg)):
+        assert leaf.grad.dtype == leaf.dtype
+        torch.testing.assert_close(leaf.grad.float(), want.float(), rtol=8e-3, atol=1e-6)
+
+
+def test_bwd_status_word_stays_clear(dev):
+    L, H, b, k = 1000, 2, 64, 4
+    x = synth.make_inputs(L, H, 64, b, 57)
+    cfg = api.Config(L=L, H=H, block=b, topk=k)
+    d = {n: getattr(x, n).to(dev) for n in ("q", "k", "v", "gates")}
+    idx = torch.empty((H, cfg.nqb, cfg.nsel), dtype=torch.int32, device=dev)
+    api.sparse_attn_fwd(cfg, d["q"], d["k"], d["v"], d["gates"], idx_out=idx)
+    word = torch.zeros(1, dtype=torch.int32, device=dev)
+    api.sparse_attn_bwd(cfg, d["q"], d["k"], d["v"], d["gates"], idx,
+                        _dout(L, H, 57).to(dev), dev_status=word)
+    assert api.read_device_status(word) == 0
