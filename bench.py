@@ -30,9 +30,10 @@ Other workloads:
 
 --single-kernel runs the compressed branch, top-k and selection as one kernel.
 
---backward also times s3r_sparse_attn_bwd (the gradients of q, k, v and the gate logits, with the
-forward's selection lists held fixed) on the same inputs, and adds a "backward" object: its
-tokens/s, algorithmic TFLOP/s, per-stage times and the roofline of its dominant kernel.
+The line also carries a "backward" object: s3r_sparse_attn_bwd (the gradients of q, k, v and the
+gate logits, with the forward's selection lists held fixed) timed on the same inputs, with its
+tokens/s, algorithmic TFLOP/s, per-stage times and the roofline of its dominant kernel
+(--no-backward skips it).
 
 --impl reference times the CPU oracle (the only other implementation of this method) on bounded
 samples of the same workload and prints the same line with "impl": "reference".
@@ -451,7 +452,7 @@ def run_native(args, wl):
     ms_max = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
     stage_ms = {n: statistics.mean(e.stage_ms()[n] for e in stage_ev) for n in _lib.STAGES}
     bwd = (time_backward(args, cfg, q, k, v, gates, sa.idx, dev, barrier, load_peaks())
-           if args.backward else None)
+           if not args.no_backward else None)
 
     # end to end through the public API from pinned host memory: every step copies all of its
     # inputs in and its output out. HostPipeline overlaps the copy-in of step i+1 and the
@@ -666,8 +667,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--single-kernel", action="store_true",
                     help="run the compressed branch, top-k and selection as one kernel (k <= 32)")
-    ap.add_argument("--backward", action="store_true",
-                    help="also time the backward (s3r_sparse_attn_bwd) on the same inputs")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip timing the backward (s3r_sparse_attn_bwd) on the same inputs")
     ap.add_argument("--no-dense-context", action="store_true",
                     help="skip timing dense attention (torch SDPA) on a sample of query rows")
     ap.add_argument("--dense-rows", type=int, default=16384,
