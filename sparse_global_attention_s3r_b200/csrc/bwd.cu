@@ -212,6 +212,31 @@ __global__ void csr_fill_kernel(const int32_t* __restrict__ idx, int32_t* __rest
   }
 }
 
+// The token-side items (head, 64-slot group) in order of decreasing list length: a counting sort
+// on bin nqb - min(len, nqb), so that a CTA pairs two groups of about equal length and the long
+// lists start first.
+__device__ __forceinline__ int64_t item_bin(const int32_t* off, int64_t item, int64_t G,
+                                            int64_t nb, int cpb, int64_t nqb) {
+  const int64_t h = item / G, j = (item - h * G) / cpb;
+  const int64_t len = off[h * (nb + 1) + j + 1] - off[h * (nb + 1) + j];
+  return nqb - (len < nqb ? len : nqb);
+}
+
+__global__ void order_count_kernel(const int32_t* __restrict__ off, int32_t* __restrict__ hist,
+                                   int64_t n_items, int64_t G, int64_t nb, int cpb, int64_t nqb) {
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < n_items;
+       it += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    atomicAdd(hist + item_bin(off, it, G, nb, cpb, nqb), 1);
+}
+
+__global__ void order_fill_kernel(const int32_t* __restrict__ off, int32_t* __restrict__ cursor,
+                                  int32_t* __restrict__ order, int64_t n_items, int64_t G,
+                                  int64_t nb, int cpb, int64_t nqb) {
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < n_items;
+       it += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    order[atomicAdd(cursor + item_bin(off, it, G, nb, cpb, nqb), 1)] = static_cast<int32_t>(it);
+}
+
 // ------------------------------------------------------------------------------------------
 // Q-outer: dq of both branches
 // ------------------------------------------------------------------------------------------
@@ -528,11 +553,12 @@ struct BwdKVArgs {
   const float* stats;   // [6][H][Lp]
   const int32_t* off;   // kSel: [H][nb+1] list offsets
   const int32_t* ent;   // kSel: [H][per_head] query blocks
+  const int32_t* order; // kSel: the H*G (head, group) items, longest list first
   const float* dkc;     // kSel: pooled gradients [nb, H, 64] (already scaled)
   const float* dvc;
   float* out_k;         // !kSel: dKc [nb, H, 64]; kSel: dk [L, H, 64]
   float* out_v;
-  int64_t L, Lp, nb, nqb, kv_rows, per_head, G;
+  int64_t L, Lp, nb, nqb, kv_rows, per_head, G;  // kSel: G groups per head
   BlockGeo geo;
   int H, b, cpb;        // cpb: 64-slot groups per key block
   float scale, scale_log2;
@@ -558,19 +584,25 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int h = blockIdx.y;
   const uint64_t lim = a.limit_ns;
   const int64_t plane = static_cast<int64_t>(a.H) * a.Lp;
-  // kSel: the CTA's two 64-slot groups, their key blocks and query-block lists
+  // kSel: the CTA's two 64-slot groups (items 2x, 2x+1 of the longest-first order, each of its
+  // own head), their key blocks and query-block lists
   int64_t gj[2] = {0, 0};
-  int go[2] = {0, 0}, glen[2] = {0, 0};
+  int go[2] = {0, 0}, glen[2] = {0, 0}, hg[2] = {h, h};
+  bool gvalid[2] = {false, false};
   int64_t gbase[2] = {0, 0};
   int nsteps;
   if constexpr (kSel) {
+    const int64_t n_items = a.G * a.H;
     for (int grp = 0; grp < 2; ++grp) {
-      const int64_t g = 2 * static_cast<int64_t>(blockIdx.x) + grp;
-      const int64_t gg = g < a.G ? g : 2 * static_cast<int64_t>(blockIdx.x);
-      gj[grp] = gg / a.cpb;
-      go[grp] = static_cast<int>(gg - gj[grp] * a.cpb) * 64;
-      if (g < a.G) {
-        const int32_t* o = a.off + static_cast<int64_t>(h) * (a.nb + 1) + gj[grp];
+      const int64_t item = 2 * static_cast<int64_t>(blockIdx.x) + grp;
+      gvalid[grp] = item < n_items;
+      const int64_t it = a.order[gvalid[grp] ? item : 2 * static_cast<int64_t>(blockIdx.x)];
+      hg[grp] = static_cast<int>(it / a.G);
+      const int64_t g = it - static_cast<int64_t>(hg[grp]) * a.G;
+      gj[grp] = g / a.cpb;
+      go[grp] = static_cast<int>(g - gj[grp] * a.cpb) * 64;
+      if (gvalid[grp]) {
+        const int32_t* o = a.off + static_cast<int64_t>(hg[grp]) * (a.nb + 1) + gj[grp];
         gbase[grp] = o[0];
         glen[grp] = o[1] - o[0];
       }
@@ -614,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_arrive_expect_tx(&bars->kv_full, 2 * kKBytes);
       if constexpr (kSel) {  // 64 slots of each group from the slot-order copies
         for (int grp = 0; grp < 2; ++grp) {
-          const int32_t y = static_cast<int32_t>(h * a.kv_rows + gj[grp] * a.b + go[grp]);
+          const int32_t y = static_cast<int32_t>(hg[grp] * a.kv_rows + gj[grp] * a.b + go[grp]);
           tma_load_2d(sbase + kOffK + grp * (kKBytes / 2), &tmK, 0, y, &bars->kv_full);
           tma_load_2d(sbase + kOffV + grp * (kKBytes / 2), &tmV, 0, y, &bars->kv_full);
         }
@@ -635,14 +667,15 @@ __global__ void __launch_bounds__(kThreads, 2)
         if constexpr (kSel) {  // rows (t%2)*32 .. +32 of the (t/2)-th query block of each list
           const int u = t >> 1;
           for (int grp = 0; grp < 2; ++grp) {
+            const int hh = hg[grp];
             const int64_t i = u < glen[grp]
-                                  ? a.ent[static_cast<int64_t>(h) * a.per_head + gbase[grp] + u]
+                                  ? a.ent[static_cast<int64_t>(hh) * a.per_head + gbase[grp] + u]
                                   : 0;
             const int64_t row0 = i * 64 + (t & 1) * 32;
-            tma_load_2d(sq + grp * (kQTile / 2), &tmQ, h * 64, static_cast<int32_t>(row0), full);
-            tma_load_2d(sq + kQTile + grp * (kQTile / 2), &tmO, h * 64,
+            tma_load_2d(sq + grp * (kQTile / 2), &tmQ, hh * 64, static_cast<int32_t>(row0), full);
+            tma_load_2d(sq + kQTile + grp * (kQTile / 2), &tmO, hh * 64,
                         static_cast<int32_t>(row0), full);
-            const float* s0 = a.stats + static_cast<int64_t>(h) * a.Lp + row0;
+            const float* s0 = a.stats + static_cast<int64_t>(hh) * a.Lp + row0;
             const uint32_t sd = sq + 2 * kQTile + grp * 384;
             bulk_load(sd, s0 + kLse2S * plane, 128, full);
             bulk_load(sd + 128, s0 + kGS * plane, 128, full);
@@ -793,15 +826,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       auto kval = [&](int c) { return __uint_as_float(c < 16 ? rk0[c] : rk1[c - 16]) * sc; };
       auto vval = [&](int c) { return __uint_as_float(c < 16 ? rv0[c] : rv1[c - 16]); };
       if constexpr (kSel) {
-        const int64_t g = 2 * static_cast<int64_t>(blockIdx.x) + grp;
         const int o = go[grp] + (row & 63);
-        if (g < a.G && (row & 63) < a.b && o < a.b) {
+        if (gvalid[grp] && (row & 63) < a.b && o < a.b) {
           const int64_t j = gj[grp];
           const int64_t tok = slot_token(a.geo, j, o);
           if (tok >= 0) {
             const float inv = 1.f / static_cast<float>(block_count(a.geo, j));
-            const int64_t src = (j * a.H + h) * 64 + 32 * half;
-            const int64_t dst = (tok * a.H + h) * 64 + 32 * half;
+            const int64_t src = (j * a.H + hg[grp]) * 64 + 32 * half;
+            const int64_t dst = (tok * a.H + hg[grp]) * 64 + 32 * half;
             const float4* pk4 = reinterpret_cast<const float4*>(a.dkc + src);
             const float4* pv4 = reinterpret_cast<const float4*>(a.dvc + src);
             float4* k4 = reinterpret_cast<float4*>(a.out_k + dst);
@@ -854,6 +886,8 @@ BwdLayout bwd_layout(const Problem& p) {
   BwdLayout w{};
   w.Lp = (p.L + 127) / 128 * 128;
   w.per_head = p.nqb * p.nsel;
+  w.cpb = p.b > 64 ? p.b / 64 : 1;
+  w.G = p.nb * w.cpb;
   return w;
 }
 
@@ -889,6 +923,18 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& B, cudaStream_t st,
                                             p.nsel);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // the token-side items, longest list first
+    const int64_t n_items = w.G * p.H;
+    const unsigned ob = static_cast<unsigned>((n_items + 255) / 256 < 4096 ? (n_items + 255) / 256 : 4096);
+    if ((e = cudaMemsetAsync(B.hist, 0, sizeof(int32_t) * (p.nqb + 1), st)) != cudaSuccess) return e;
+    order_count_kernel<<<ob, 256, 0, st>>>(B.off, B.hist, n_items, w.G, p.nb, w.cpb, p.nqb);
+    count_launch();
+    csr_scan_kernel<<<1, 1024, 0, st>>>(B.hist, B.hoff, B.hcur, p.nqb + 1);
+    count_launch();
+    order_fill_kernel<<<ob, 256, 0, st>>>(B.off, B.hcur, B.order, n_items, w.G, p.nb, w.cpb,
+                                          p.nqb);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = mark(2)) != cudaSuccess) return e;
   // dq
@@ -921,7 +967,7 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& B, cudaStream_t st,
         !make_tmap_head_rows(&to, B.dout, p.L, p.H, 64))
       return cudaErrorInvalidValue;
     if ((e = prepare(bwd_kv_kernel<false>, kv_outer::kSmemBytes)) != cudaSuccess) return e;
-    BwdKVArgs a{B.stats, nullptr, nullptr, nullptr, nullptr, B.dkc, B.dvc, p.L, w.Lp, p.nb,
+    BwdKVArgs a{B.stats, nullptr, nullptr, nullptr, nullptr, nullptr, B.dkc, B.dvc, p.L, w.Lp, p.nb,
                 p.nqb, kv_rows, w.per_head, 0, p.geo, p.H, p.b, 1, p.scale, p.scale_log2,
                 p.status, lim};
     dim3 grid(static_cast<unsigned>((p.nb + 127) / 128), p.H);
@@ -938,12 +984,10 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& B, cudaStream_t st,
         !make_tmap_head_rows(&to, B.dout, p.L, p.H, 32))
       return cudaErrorInvalidValue;
     if ((e = prepare(bwd_kv_kernel<true>, kv_outer::kSmemBytes)) != cudaSuccess) return e;
-    const int cpb = p.b > 64 ? p.b / 64 : 1;
-    const int64_t G = p.nb * cpb;
-    BwdKVArgs a{B.stats, B.off, B.ent, B.dkc, B.dvc, B.dk, B.dv, p.L, w.Lp, p.nb, p.nqb,
-                kv_rows, w.per_head, G, p.geo, p.H, p.b, cpb, p.scale, p.scale_log2, p.status,
-                lim};
-    dim3 grid(static_cast<unsigned>((G + 1) / 2), p.H);
+    BwdKVArgs a{B.stats, B.off, B.ent, B.order, B.dkc, B.dvc, B.dk, B.dv, p.L, w.Lp, p.nb,
+                p.nqb, kv_rows, w.per_head, w.G, p.geo, p.H, p.b, w.cpb, p.scale, p.scale_log2,
+                p.status, lim};
+    dim3 grid(static_cast<unsigned>((w.G * p.H + 1) / 2), 1);
     bwd_kv_kernel<true><<<grid, kThreads, kv_outer::kSmemBytes, st>>>(tkh, tvh, tq, to, a);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -60,6 +60,8 @@ cudaError_t launch_gate_combine(const Problem& p, const float* o_cmp, const floa
 struct BwdLayout {
   int64_t Lp;        // rows of the statistics planes: L rounded up to whole 128-row tiles
   int64_t per_head;  // entries of one head's selection lists: nqb * nsel
+  int cpb;           // 64-slot groups per key block (token-side kernel)
+  int64_t G;         // groups per head: nb * cpb
 };
 BwdLayout bwd_layout(const Problem& p);
 struct BwdBuffers {
@@ -71,6 +73,9 @@ struct BwdBuffers {
   int32_t *cnt, *cursor;  // [H, nb] scratch
   int32_t* off;           // [H, nb + 1] scratch
   int32_t* ent;           // [H, per_head] scratch
+  int32_t* order;         // [H * G] scratch: token-side items, longest list first
+  int32_t *hist, *hcur;   // [nqb + 1] scratch
+  int32_t* hoff;          // [nqb + 2] scratch
   float *dq, *dk, *dv;    // [L, H, 64] outputs
   float* dgates;          // [L, H, 2] output
 };

@@ -134,7 +134,8 @@ def test_bwd_workspace_size_matches_layout(L, H, b, k, F):
     want = (r256(4) + 2 * r256(nb * H * d * 2) + 2 * r256(nb * b * H * d * 2)
             + 2 * r256(L * H * d * 4) + 2 * r256(H * L * 4) + r256(6 * H * Lp * 4)
             + 2 * r256(nb * H * d * 4) + 2 * r256(H * nb * 4) + r256(H * (nb + 1) * 4)
-            + r256(H * nqb * (F + k) * 4))
+            + r256(H * nqb * (F + k) * 4) + r256(H * nb * max(1, b // 64) * 4)
+            + 2 * r256((nqb + 1) * 4) + r256((nqb + 2) * 4))
     assert api.bwd_workspace_bytes(cfg) == want
 
 
