@@ -41,6 +41,7 @@ samples of the same workload and prints the same line with "impl": "reference".
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import math
@@ -196,7 +197,22 @@ def time_backward(args, cfg, q, k, v, gates, idx, dev, barrier, peaks):
 
     g = torch.Generator(device=dev).manual_seed(99)
     dout = torch.randn(q.shape, generator=g, device=dev).to(torch.bfloat16)
+    # training use: the forward keeps what the backward needs (save_for_backward), and the
+    # backward reads it from the same workspace instead of recomputing the forward
+    cfg = dataclasses.replace(cfg, save_for_backward=True, single_kernel=False)
     ws = torch.empty(api.bwd_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty_like(idx)
+    for _ in range(args.warmup):
+        api.sparse_attn_fwd(cfg, q, k, v, gates, ws, out, idx)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(args.steps):
+        api.sparse_attn_fwd(cfg, q, k, v, gates, ws, out, idx)
+    f1.record()
+    torch.cuda.synchronize()
+    fwd_save_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps, dev)
     grads = (*(torch.empty(q.shape, dtype=torch.float32, device=dev) for _ in range(3)),
              torch.empty(gates.shape, dtype=torch.float32, device=dev))
     for _ in range(args.warmup):
@@ -219,21 +235,28 @@ def time_backward(args, cfg, q, k, v, gates, idx, dev, barrier, peaks):
     stages = {}
     for n, (b_, u_) in work["stage_work"].items():
         s_ = stage_ms[n] / 1e3
+        if s_ < 1e-5:  # no launch in this stage (the recompute, after a saving forward)
+            stages[n] = {"ms": stage_ms[n], "launched": False}
+            continue
         stages[n] = {"ms": stage_ms[n],
                      ("GB/s" if b_ == "hbm" else "TFLOP/s"): u_ / s_ / (1e9 if b_ == "hbm" else 1e12)}
     dom = max(("dq", "dkv_cmp", "dkv_sel"), key=stage_ms.get)
     ach = work["stage_work"][dom][1] / (stage_ms[dom] / 1e3) / 1e12
-    del ws, grads, dout
+    del ws, grads, dout, out
     return {
         "ms_per_step": ms, "tokens_per_s": cfg.L / (ms / 1e3),
+        "forward_save_ms": fwd_save_ms,
+        "train_step_ms": fwd_save_ms + ms,
         "tflops": work["flops"] / (ms / 1e3) / 1e12, "stage_ms": stages,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": ach,
                      "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                      "frac": ach / peaks["bf16_tflops_sustained"],
                      "peak_source": peaks["source"] + " sustained bf16", "traffic": None},
         "gpu_launches": launches,
-        "how": "s3r_sparse_attn_bwd on the forward's own selection lists and a seeded bf16 dout; "
-               "each call recomputes the forward (stage 'recompute')",
+        "how": "s3r_sparse_attn_bwd on the forward's own selection lists and a seeded bf16 dout, "
+               "reading what a save_for_backward forward kept in the same workspace (the "
+               "recompute stage is empty); forward_save_ms times that forward, train_step_ms "
+               "is forward + backward",
     }
 
 

@@ -83,6 +83,13 @@ typedef enum {
                                        the top-k and the selection branch with the gated combine,
                                        keeping O_cmp (as bf16) and the lists on chip (2 launches);
                                        its stage S3R_STAGE_CMP then covers selection too */
+#define S3R_FLAG_SAVE_FOR_BWD 0x8u  /* s3r_sparse_attn_fwd also keeps, in its workspace, what
+                                       s3r_sparse_attn_bwd needs (O_cmp, O_sel, both branches'
+                                       lse, the pooled K/V and their slot-order copies), so that
+                                       a backward call given the same flag and the same workspace
+                                       skips recomputing the forward. The workspace then grows
+                                       (s3r_workspace_bytes reports it); S3R_FLAG_SINGLE_KERNEL
+                                       is ignored (the 3-kernel path runs) */
 
 typedef struct {
   int64_t L;      /* tokens = N views * P tokens per view, >= 1 */
@@ -237,6 +244,11 @@ s3r_status s3r_sparse_attn_fwd(const s3r_params* params, const s3r_bf16* q, cons
  * Returns S3R_ERR_UNSUPPORTED when H * nb * block exceeds 2^31 - 1 (row coordinates of the
  * slot-order K/V copies). The order in which query blocks add into one key block's dK, dV
  * follows an atomic fill and may differ between calls (fp32 rounding only). */
+/* With S3R_FLAG_SAVE_FOR_BWD in params->flags, the backward reads the forward's saved tensors:
+ * the workspace must be the one the forward call used, of at least s3r_bwd_workspace_bytes
+ * bytes (its first s3r_workspace_bytes bytes are the forward's; pass the same buffer to both
+ * calls), with the same q, k, v, gates and the idx the forward wrote. The call then starts at
+ * S3R_BWD_STAGE_PREP (the recompute stage is empty). */
 size_t s3r_bwd_workspace_bytes(const s3r_params* params);
 s3r_status s3r_sparse_attn_bwd(const s3r_params* params, const s3r_bf16* q, const s3r_bf16* k,
                                const s3r_bf16* v, const float* gate_logits, const int32_t* idx,

@@ -23,6 +23,7 @@ S3R_DEV_BAD_INDEX = 0x2
 S3R_FLAG_DEBUG_CHECKS = 0x1
 S3R_FLAG_TEST_TIMEOUT = 0x2
 S3R_FLAG_SINGLE_KERNEL = 0x4
+S3R_FLAG_SAVE_FOR_BWD = 0x8
 S3R_MAX_BLOCKS = 49152
 S3R_STATIC_WORKSPACE_BYTES = 32 << 20
 STAGES = ("pool", "cmp", "topk", "sel_combine")  # S3R_STAGE_* order

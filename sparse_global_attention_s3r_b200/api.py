@@ -15,6 +15,7 @@ nb counts the key blocks of the configured geometry (Config.nb), nqb = ceil(L / 
 from __future__ import annotations
 
 import ctypes
+import dataclasses
 from dataclasses import dataclass
 from typing import Optional, Tuple
 
@@ -33,7 +34,9 @@ class Config:
     tokens per view, ceil(P / b)); the top-k then picks topk more among the other blocks.
     grid_h, grid_w, special, win_h: 2-D windows (grid_h > 0). The sequence is L / P views of
     P = special + grid_h * grid_w tokens; key blocks are each view's special tokens, then
-    win_h x (block / win_h) windows of its patch grid."""
+    win_h x (block / win_h) windows of its patch grid.
+    save_for_backward: the forward keeps in its workspace what the backward needs, and a backward
+    call with the same config and workspace skips recomputing the forward."""
 
     L: int
     H: int
@@ -49,6 +52,7 @@ class Config:
     grid_w: int = 0
     special: int = 0
     win_h: int = 0
+    save_for_backward: bool = False
 
     @property
     def nsel(self) -> int:
@@ -69,7 +73,8 @@ class Config:
                            0.0 if self.scale is None else float(self.scale),
                            (_lib.S3R_FLAG_DEBUG_CHECKS if self.debug_checks else 0)
                            | (_lib.S3R_FLAG_TEST_TIMEOUT if self.test_timeout else 0)
-                           | (_lib.S3R_FLAG_SINGLE_KERNEL if self.single_kernel else 0),
+                           | (_lib.S3R_FLAG_SINGLE_KERNEL if self.single_kernel else 0)
+                           | (_lib.S3R_FLAG_SAVE_FOR_BWD if self.save_for_backward else 0),
                            self.forced, self.grid_h, self.grid_w, self.special, self.win_h,
                            None if dev_status is None else dev_status.data_ptr(),
                            None if stage_events is None else ctypes.addressof(stage_events))
@@ -245,12 +250,16 @@ def sparse_attn_bwd(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tens
     (the forward's idx_out) held fixed: returns dq, dk, dv [L,H,d] fp32 and dgates [L,H,2] fp32.
 
     grads: optional preallocated (dq, dk, dv, dgates) to write into; stage_events: a
-    StageEvents(_lib.BWD_STAGES) that the call records at its stage boundaries."""
+    StageEvents(_lib.BWD_STAGES) that the call records at its stage boundaries. With
+    cfg.save_for_backward, workspace must be the one the forward call used (allocate
+    bwd_workspace_bytes(cfg) bytes and pass it to both)."""
     for n, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
         _need(t, n, _lhd(cfg), torch.bfloat16)
     _need(gates, "gates", (cfg.L, cfg.H, 2), torch.float32)
     _need(idx, "idx", (cfg.H, cfg.nqb, cfg.nsel), torch.int32)
     if workspace is None:
+        if cfg.save_for_backward:
+            raise ValueError("save_for_backward: pass the forward call's workspace")
         workspace = torch.empty(bwd_workspace_bytes(cfg), dtype=torch.uint8, device=q.device)
     if grads is None:
         grads = (*(torch.empty(_lhd(cfg), dtype=torch.float32, device=q.device) for _ in range(3)),
@@ -270,13 +279,17 @@ class SparseAttentionFunction(torch.autograd.Function):
     """autograd wrapper: forward = sparse_attn_fwd (bf16 out), backward = sparse_attn_bwd.
 
     Gradients are returned in the inputs' dtypes (bf16 for q, k, v; fp32 for the gate logits).
-    The top-k selection passes no gradient."""
+    The top-k selection passes no gradient. The forward runs with save_for_backward and keeps
+    its workspace, so the backward does not recompute the forward."""
 
     @staticmethod
     def forward(ctx, q, k, v, gates, cfg: Config):
+        cfg = dataclasses.replace(cfg, save_for_backward=True, single_kernel=False)
         idx = torch.empty((cfg.H, cfg.nqb, cfg.nsel), dtype=torch.int32, device=q.device)
-        out = sparse_attn_fwd(cfg, q, k, v, gates, idx_out=idx)
+        ws = torch.empty(bwd_workspace_bytes(cfg), dtype=torch.uint8, device=q.device)
+        out = sparse_attn_fwd(cfg, q, k, v, gates, workspace=ws, idx_out=idx)
         ctx.cfg = cfg
+        ctx.ws = ws
         ctx.save_for_backward(q, k, v, gates, idx)
         ctx.mark_non_differentiable(idx)
         return out
@@ -285,7 +298,8 @@ class SparseAttentionFunction(torch.autograd.Function):
     def backward(ctx, dout):
         q, k, v, gates, idx = ctx.saved_tensors
         dq, dk, dv, dg = sparse_attn_bwd(ctx.cfg, q, k, v, gates, idx,
-                                         dout.to(torch.bfloat16).contiguous())
+                                         dout.to(torch.bfloat16).contiguous(), workspace=ctx.ws)
+        ctx.ws = None
         return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype), dg, None
 
 

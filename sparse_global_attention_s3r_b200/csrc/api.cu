@@ -77,12 +77,13 @@ s3r_status launched(cudaError_t e) { return e == cudaSuccess ? S3R_OK : S3R_ERR_
 // Workspace of the fused call, every region 256-byte aligned:
 //   status word | Kc [nb,H,d] bf16 | Vc | Kh [H,nb*b,d] bf16 | Vh | O_cmp [L,H,d] f32
 //   | scores [H,nqb,nb] f32 | idx [H,nqb,forced+k] i32
+//   [with S3R_FLAG_SAVE_FOR_BWD: | O_sel [L,H,d] f32 | lse_c, lse_s [H,L] f32]
 // Kh, Vh are head-major copies of K and V written by the pooling pass, from which the selection
 // branch gathers each selected block as contiguous rows.
 // The score matrix is only materialised when k > kFusedTopkMax; otherwise the compressed-branch
 // kernel selects the top-k on the fly and the scores region is empty.
 struct Workspace {
-  size_t status, kc, vc, kh, vh, o_cmp, scores, idx, total;
+  size_t status, kc, vc, kh, vh, o_cmp, scores, idx, o_sel, lse_c, lse_s, total;
 };
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -111,6 +112,11 @@ Workspace layout(const Problem& p) {
   w.o_cmp = take(static_cast<size_t>(p.L) * HD * 4);
   w.scores = take(p.k > kFusedTopkMax ? static_cast<size_t>(p.H) * p.nqb * p.nb * 4 : 0);
   w.idx = take(static_cast<size_t>(p.H) * p.nqb * p.nsel * 4);
+  if (p.flags & S3R_FLAG_SAVE_FOR_BWD) {  // what the backward reads instead of recomputing
+    w.o_sel = take(static_cast<size_t>(p.L) * HD * 4);
+    w.lse_c = take(static_cast<size_t>(p.H) * p.L * 4);
+    w.lse_s = take(static_cast<size_t>(p.H) * p.L * 4);
+  }
   w.total = off;
   return w;
 }
@@ -135,15 +141,22 @@ BwdWorkspace bwd_ws_layout(const Problem& p) {
   const BwdLayout bl = bwd_layout(p);
   const size_t HD = static_cast<size_t>(p.H) * p.d;
   const size_t H = static_cast<size_t>(p.H);
-  w.status = take(4);
-  w.kc = take(static_cast<size_t>(p.nb) * HD * 2);
-  w.vc = take(static_cast<size_t>(p.nb) * HD * 2);
-  w.kh = take(static_cast<size_t>(p.nb) * p.b * HD * 2);
-  w.vh = take(static_cast<size_t>(p.nb) * p.b * HD * 2);
-  w.o_cmp = take(static_cast<size_t>(p.L) * HD * 4);
-  w.o_sel = take(static_cast<size_t>(p.L) * HD * 4);
-  w.lse_c = take(H * p.L * 4);
-  w.lse_s = take(H * p.L * 4);
+  if (p.flags & S3R_FLAG_SAVE_FOR_BWD) {  // the forward's workspace, with its saved tensors, first
+    const Workspace f = layout(p);
+    w.status = f.status, w.kc = f.kc, w.vc = f.vc, w.kh = f.kh, w.vh = f.vh;
+    w.o_cmp = f.o_cmp, w.o_sel = f.o_sel, w.lse_c = f.lse_c, w.lse_s = f.lse_s;
+    off = f.total;
+  } else {
+    w.status = take(4);
+    w.kc = take(static_cast<size_t>(p.nb) * HD * 2);
+    w.vc = take(static_cast<size_t>(p.nb) * HD * 2);
+    w.kh = take(static_cast<size_t>(p.nb) * p.b * HD * 2);
+    w.vh = take(static_cast<size_t>(p.nb) * p.b * HD * 2);
+    w.o_cmp = take(static_cast<size_t>(p.L) * HD * 4);
+    w.o_sel = take(static_cast<size_t>(p.L) * HD * 4);
+    w.lse_c = take(H * p.L * 4);
+    w.lse_s = take(H * p.L * 4);
+  }
   w.stats = take(6 * H * bl.Lp * 4);
   w.dkc = take(static_cast<size_t>(p.nb) * HD * 4);
   w.dvc = take(static_cast<size_t>(p.nb) * HD * 4);
@@ -177,11 +190,16 @@ int fused_forward(const s3r_params* params, const uint16_t* q, const uint16_t* k
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate_logits) ||
       !aligned16(out) || (idx_out && !aligned16(idx_out)))
     return S3R_ERR_INVALID_ARG;
+  const bool save = (p.flags & S3R_FLAG_SAVE_FOR_BWD) != 0;
+  if (save && !use_head_major(p)) return S3R_ERR_UNSUPPORTED;
   const Workspace w = layout(p);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < w.total)
     return S3R_ERR_WORKSPACE;
   uint8_t* base = static_cast<uint8_t*>(workspace);
   uint32_t* status = reinterpret_cast<uint32_t*>(base + w.status);
+  float* o_sel = save ? reinterpret_cast<float*>(base + w.o_sel) : nullptr;
+  float* lse_c = save ? reinterpret_cast<float*>(base + w.lse_c) : nullptr;
+  float* lse_s = save ? reinterpret_cast<float*>(base + w.lse_s) : nullptr;
   if (!p.status) p.status = status;
   uint16_t* kc = reinterpret_cast<uint16_t*>(base + w.kc);
   uint16_t* vc = reinterpret_cast<uint16_t*>(base + w.vc);
@@ -201,21 +219,21 @@ int fused_forward(const s3r_params* params, const uint16_t* q, const uint16_t* k
   if ((st = launched(launch_pool_kv(p, k, v, kc, vc, kh, vh, stream))) != S3R_OK) return st;
   if (mark(1) != cudaSuccess) return S3R_ERR_CUDA;
   const bool fused_topk = p.k <= kFusedTopkMax;
-  if ((p.flags & S3R_FLAG_SINGLE_KERNEL) && fused_topk && hm) {
+  if ((p.flags & S3R_FLAG_SINGLE_KERNEL) && fused_topk && hm && !save) {
     st = launched(launch_fused_tc(p, q, kc, vc, kh, vh, gate_logits, out, idx_out, stream));
     if (st != S3R_OK) return st;
     for (int i = 2; i <= 4; ++i)
       if (mark(i) != cudaSuccess) return S3R_ERR_CUDA;
     return S3R_OK;
   }
-  if ((st = launched(launch_cmp_attn_tc(p, q, kc, vc, nullptr, o_cmp, fused_topk ? nullptr : scores,
+  if ((st = launched(launch_cmp_attn_tc(p, q, kc, vc, lse_c, o_cmp, fused_topk ? nullptr : scores,
                                         fused_topk ? idx : nullptr, stream))) != S3R_OK)
     return st;
   if (mark(2) != cudaSuccess) return S3R_ERR_CUDA;
   if (!fused_topk && (st = launched(launch_topk(p, scores, idx, stream))) != S3R_OK) return st;
   if (mark(3) != cudaSuccess) return S3R_ERR_CUDA;
-  st = launched(launch_sel_attn(p, q, hm ? kh : k, hm ? vh : v, hm, idx, nullptr, o_cmp, gate_logits,
-                                out, stream));
+  st = launched(launch_sel_attn(p, q, hm ? kh : k, hm ? vh : v, hm, idx, o_sel, o_cmp, gate_logits,
+                                out, stream, lse_s));
   if (st != S3R_OK) return st;
   return mark(4) == cudaSuccess ? S3R_OK : S3R_ERR_CUDA;
 }
@@ -351,16 +369,18 @@ s3r_status s3r_sparse_attn_bwd(const s3r_params* params, const s3r_bf16* q, cons
   if (cudaMemsetAsync(status, 0, 4, stream) != cudaSuccess) return S3R_ERR_CUDA;
   if (ev && cudaEventRecord(static_cast<cudaEvent_t>(ev[0]), stream) != cudaSuccess)
     return S3R_ERR_CUDA;
-  // the forward again, keeping what the backward needs
-  if ((st = launched(launch_pool_kv(p, k, v, b16(w.kc), b16(w.vc), b16(w.kh), b16(w.vh),
-                                    stream))) != S3R_OK)
-    return st;
-  if ((st = launched(launch_cmp_attn_tc(p, q, b16(w.kc), b16(w.vc), f32(w.lse_c), f32(w.o_cmp),
-                                        nullptr, nullptr, stream))) != S3R_OK)
-    return st;
-  if ((st = launched(launch_sel_attn(p, q, b16(w.kh), b16(w.vh), true, idx, f32(w.o_sel), nullptr,
-                                     nullptr, nullptr, stream, f32(w.lse_s)))) != S3R_OK)
-    return st;
+  // the forward again, keeping what the backward needs (unless the forward call saved it)
+  if (!(p.flags & S3R_FLAG_SAVE_FOR_BWD)) {
+    if ((st = launched(launch_pool_kv(p, k, v, b16(w.kc), b16(w.vc), b16(w.kh), b16(w.vh),
+                                      stream))) != S3R_OK)
+      return st;
+    if ((st = launched(launch_cmp_attn_tc(p, q, b16(w.kc), b16(w.vc), f32(w.lse_c), f32(w.o_cmp),
+                                          nullptr, nullptr, stream))) != S3R_OK)
+      return st;
+    if ((st = launched(launch_sel_attn(p, q, b16(w.kh), b16(w.vh), true, idx, f32(w.o_sel),
+                                       nullptr, nullptr, nullptr, stream, f32(w.lse_s)))) != S3R_OK)
+      return st;
+  }
   if (ev && cudaEventRecord(static_cast<cudaEvent_t>(ev[1]), stream) != cudaSuccess)
     return S3R_ERR_CUDA;
   BwdBuffers b{q, dout, b16(w.kc), b16(w.vc), b16(w.kh), b16(w.vh), gate_logits, f32(w.o_cmp),

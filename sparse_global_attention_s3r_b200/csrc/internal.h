@@ -43,8 +43,8 @@ cudaError_t launch_fused_tc(const Problem& p, const uint16_t* q, const uint16_t*
                             const uint16_t* vc, const uint16_t* kh, const uint16_t* vh,
                             const float* gates, uint16_t* out, int32_t* idx, cudaStream_t st);
 cudaError_t launch_topk(const Problem& p, const float* scores, int32_t* idx, cudaStream_t st);
-// o_sel != nullptr: write the selection output (fp32). Otherwise fuse the gated combine:
-// read o_cmp and gates and write out (bf16). lse (nullable): [H, L] natural log of each row's
+// o_sel != nullptr: write the selection output (fp32). out != nullptr: fuse the gated combine,
+// reading o_cmp and gates and writing out (bf16). Either or both. lse (nullable): [H, L] natural log of each row's
 // softmax normaliser over its selected tokens.
 // k, v: [L, H, 64] token-major, or (head_major) the [H, nb*b, 64] copies of launch_pool_kv.
 cudaError_t launch_sel_attn(const Problem& p, const uint16_t* q, const uint16_t* k,

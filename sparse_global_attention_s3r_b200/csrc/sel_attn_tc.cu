@@ -469,7 +469,8 @@ __global__ void __maxnreg__(128)
                                  __uint_as_float(o[j >> 3][(4 * j + 1) & 31]) * inv,
                                  __uint_as_float(o[j >> 3][(4 * j + 2) & 31]) * inv,
                                  __uint_as_float(o[j >> 3][(4 * j + 3) & 31]) * inv);
-        } else {
+        }
+        if (a.out) {
           const float2 gl = *reinterpret_cast<const float2*>(a.gates + (row * a.H + h) * 2);
           const float gc = 1.f / (1.f + expf(-gl.x));
           const float gs = 1.f / (1.f + expf(-gl.y));

@@ -139,6 +139,27 @@ def test_bwd_workspace_size_matches_layout(L, H, b, k, F):
     assert api.bwd_workspace_bytes(cfg) == want
 
 
+@pytest.mark.parametrize("L,H,b,k", [(1024, 2, 64, 4), (1374000, 16, 64, 32), (3000, 2, 32, 40)])
+def test_save_for_backward_workspaces(L, H, b, k):
+    """With S3R_FLAG_SAVE_FOR_BWD the forward's workspace adds O_sel and both lse, and the
+    backward's workspace is the forward's followed by the backward's own scratch."""
+    import dataclasses
+
+    cfg = api.Config(L=L, H=H, block=b, topk=k)
+    save = dataclasses.replace(cfg, save_for_backward=True)
+    fwd, fwd_s = api.workspace_bytes(cfg), api.workspace_bytes(save)
+    assert fwd_s == fwd + r256(L * H * 64 * 4) + 2 * r256(H * L * 4)
+    nb, nqb = cfg.nb, cfg.nqb
+    Lp = (L + 127) // 128 * 128
+    scratch = (r256(6 * H * Lp * 4) + 2 * r256(nb * H * 64 * 4) + 2 * r256(H * nb * 4)
+               + r256(H * (nb + 1) * 4) + r256(H * nqb * k * 4) + r256(H * nb * max(1, b // 64) * 4)
+               + 2 * r256((nqb + 1) * 4) + r256((nqb + 2) * 4))
+    assert api.bwd_workspace_bytes(save) == fwd_s + scratch
+    lib = _lib.load()
+    p = ctypes.byref(save.params())
+    assert lib.s3r_sparse_attn_bwd(p, *[A16] * 10, A256, fwd_s, None) == _lib.S3R_ERR_WORKSPACE
+
+
 def test_bwd_rejects_slot_copies_beyond_32_bit_rows():
     lib = _lib.load()
     big = _params(L=65536, H=65535, block=64, topk=1)  # H * nb * b = 65535 * 65536 > 2^31 - 1
