@@ -1,14 +1,19 @@
 """Comparison helpers shared by the GPU parity tests (no method arithmetic here).
 
-Tolerances (bf16 inputs, fp32 accumulation; derivations in DESIGN.md "Parity bars"):
-  pooled K/V    within 1 bf16 ulp of the correctly rounded mean, >= 99.9 % bit-identical
-  lse           |d| <= 2e-5 absolute (natural-log units)
-  scores        |d| <= 1e-5 * (largest score of the row) + 1e-9
-  o_cmp, o_sel  |d| <= 2^-8 * max|V| + 1e-6 elementwise, relative L2 <= 4e-3
-  combine       |d| <= 1 bf16 ulp of the exact value + 1e-7
-  whole path    indices equal where the oracle's k-th/(k+1)-th score gap > 1e-4; every selected
-                block within tau = 1e-6 * max(1, S_(k)) of the k-th best oracle score; output
-                against the oracle run on the GPU's indices: max-abs <= 2e-2, rel-L2 <= 5e-3
+Tolerances (bf16 inputs, fp32 accumulation), each set by the arithmetic of what it checks:
+  pooled K/V    an fp32 sum then one rounding to bf16, so within 1 bf16 ulp of the correctly
+                rounded mean (the fp32 sum may move a value across a rounding boundary),
+                >= 99.9 % bit-identical
+  lse           fp32 exp2 sums and one log: |d| <= 2e-5 absolute (natural-log units)
+  scores        fp32 sums of fp32 probabilities: |d| <= 1e-5 * (largest score of the row) + 1e-9
+  o_cmp, o_sel  P is rounded to bf16 for the P V product (2^-9 relative per term):
+                |d| <= 2^-8 * max|V| + 1e-6 elementwise, relative L2 <= 4e-3
+  combine       one rounding of the fp32 result to bf16: |d| <= 1 bf16 ulp + 1e-7
+  whole path    indices equal where the oracle's k-th/(k+1)-th score gap > 1e-4 (fp32 scores
+                cannot order closer ties the way fp64 does); every selected block within
+                tau = 1e-6 * max(1, S_(k)) of the k-th best oracle score; output against the
+                oracle run on the GPU's indices: max-abs <= 2e-2, rel-L2 <= 5e-3 (the bf16 output
+                rounding plus the branch errors above)
 """
 from __future__ import annotations
 
