@@ -133,7 +133,8 @@ typedef struct {
 
 /* Stages of s3r_sparse_attn_bwd, in launch order. */
 #define S3R_BWD_STAGE_RECOMPUTE 0 /* the forward again: pooling, both branches with their lse */
-#define S3R_BWD_STAGE_PREP 1      /* D and gate gradients; the inverse of the selection lists */
+#define S3R_BWD_STAGE_PREP 1      /* D and gate gradients; the inverse of the selection lists and
+                                     the token-side work order */
 #define S3R_BWD_STAGE_DQ 2        /* dq of both branches (one kernel) */
 #define S3R_BWD_STAGE_DKV_CMP 3   /* dKc, dVc of the block summaries */
 #define S3R_BWD_STAGE_DKV_SEL 4   /* dk, dv of the selected tokens, plus dKc / n_j, dVc / n_j */

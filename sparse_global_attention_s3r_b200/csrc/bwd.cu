@@ -17,6 +17,8 @@
 //   csr_*_kernel       the inverse of the selection lists: for each (head, key block) the query
 //                      blocks that selected it (counts, per-head prefix sums, atomic fill; the
 //                      order inside a list follows the fill)
+//   order_*_kernel     the token-side items (head, 64-slot group) by decreasing list length, a
+//                      counting sort on the length
 //   bwd_q_kernel       Q-outer, one CTA per 128 query rows (two query blocks) and head: walks
 //                      the nb summaries in 64-column steps, then the selected tokens in steps of
 //                      32 slots per query block (block-diagonal 128 x 64, like the forward
@@ -26,8 +28,9 @@
 //                      S^T = K Q^T, dP'^T = V dout^T, then (g P)^T and dS^T are written in place
 //                      over S^T and dP'^T as bf16 and dV += (gP)^T dout, dK += dS^T Q.
 //                      <false>: the 128 rows are block summaries, every query is a column
-//                      (writes dKc, dVc); <true>: rows are two 64-slot groups of key blocks, each
-//                      walking the query blocks that selected its block, 32 rows of one per step
+//                      (writes dKc, dVc); <true>: rows are two 64-slot groups of key blocks
+//                      (neighbours in the longest-first order, of any heads), each walking the
+//                      query blocks that selected its block, 32 rows of one per step
 //                      (block-diagonal); writes dk, dv per token and adds the pooled gradients
 //                      dKc[j] / n_j.
 // Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-9 softmax
