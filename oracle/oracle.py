@@ -67,7 +67,7 @@ def lib():
             "s3r_ref_sel": [p, p, p, p, p, ctypes.c_int64, p, p],
             "s3r_ref_combine": [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, p, p, p, p],
             "s3r_ref_block_tokens": [p, ctypes.c_int64, p],
-            "s3r_ref_bwd": [p, p, p, p, p, p, p, p, p, p, p, p, p],
+            "s3r_ref_bwd": [p, p, p, p, p, p, p, p, p, ctypes.c_int64, p, p, p, p, p],
         }.items():
             fn = getattr(L, name)
             fn.restype = ctypes.c_int
@@ -244,19 +244,21 @@ def combine(o_cmp, o_sel, gates) -> np.ndarray:
 
 @dataclass
 class Grads:
-    dq: np.ndarray      # [L, H, d]
-    dk: np.ndarray      # [L, H, d]
-    dv: np.ndarray      # [L, H, d]
-    dgates: np.ndarray  # [L, H, 2] gradient of the gate logits
+    dq: np.ndarray      # [R, H, d] (R = L, or the rows of the chosen query blocks)
+    dk: Optional[np.ndarray]  # [L, H, d]; None for a sample of query blocks
+    dv: Optional[np.ndarray]  # [L, H, d]; None for a sample of query blocks
+    dgates: np.ndarray  # [R, H, 2] gradient of the gate logits
 
 
 def backward(pb: Problem, q_bits, k_bits, v_bits, gates, idx, dout, kc=None, vc=None,
-             threads: int = 0) -> Grads:
-    """Gradients of the whole path for the upstream gradient dout [L, H, d] (float64).
+             threads: int = 0, qblocks=None) -> Grads:
+    """Gradients of the whole path for the upstream gradient dout (float64).
 
-    The selection lists idx [H, nqb, forced + topk] are held fixed, and the bf16 rounding of the
-    pooled K/V is passed straight through (each token of block j gets dKc[j] / n_j). kc, vc are
-    the pooled values the forward ran on (default: ``pool`` of k, v).
+    The selection lists idx are held fixed, and the bf16 rounding of the pooled K/V is passed
+    straight through (each token of block j gets dKc[j] / n_j). kc, vc are the pooled values the
+    forward ran on (default: ``pool`` of k, v). With qblocks, only the rows of those query blocks
+    are differentiated: idx is [H, len(qblocks), forced + topk] for them, dout [R, H, d] their
+    rows in list order, and only dq and dgates (row-local) are returned.
     """
     q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
     k_bits = np.ascontiguousarray(k_bits, dtype=np.uint16)
@@ -271,12 +273,21 @@ def backward(pb: Problem, q_bits, k_bits, v_bits, gates, idx, dout, kc=None, vc=
     idx = np.ascontiguousarray(idx, dtype=np.int32)
     dout = np.ascontiguousarray(dout, dtype=np.float64)
     shape = (pb.L, pb.H, pb.d)
-    assert q_bits.shape == shape and dout.shape == shape and gates.shape == (pb.L, pb.H, 2)
-    assert kc.shape == (pb.nb, pb.H, pb.d) and idx.shape == (pb.H, pb.nqb, pb.nsel), idx.shape
-    g = Grads(np.empty(shape), np.empty(shape), np.empty(shape), np.empty((pb.L, pb.H, 2)))
+    qa, nq = _qb_array(qblocks)
+    if qa is None:
+        nq = pb.nqb
+    R = pb.rows_of(qblocks).size
+    assert q_bits.shape == shape and dout.shape == (R, pb.H, pb.d)
+    assert gates.shape == (pb.L, pb.H, 2) and kc.shape == (pb.nb, pb.H, pb.d)
+    assert idx.shape == (pb.H, nq, pb.nsel), idx.shape
+    full = qa is None
+    g = Grads(np.empty((R, pb.H, pb.d)), np.empty(shape) if full else None,
+              np.empty(shape) if full else None, np.empty((R, pb.H, 2)))
     rc = lib().s3r_ref_bwd(ctypes.byref(_params(pb, threads=threads)), _ptr(q_bits), _ptr(k_bits),
-                           _ptr(v_bits), _ptr(kc), _ptr(vc), _ptr(gates), _ptr(idx), _ptr(dout),
-                           _ptr(g.dq), _ptr(g.dk), _ptr(g.dv), _ptr(g.dgates))
+                           _ptr(v_bits), _ptr(kc), _ptr(vc), _ptr(gates), _ptr(idx),
+                           None if full else _ptr(qa), nq, _ptr(dout), _ptr(g.dq),
+                           _ptr(g.dk) if full else None, _ptr(g.dv) if full else None,
+                           _ptr(g.dgates))
     assert rc == 0, rc
     return g
 

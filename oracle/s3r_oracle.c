@@ -491,17 +491,19 @@ typedef struct {
   const double *kc, *vc;
   const float* gates;
   const int32_t* idx;
+  const row_map* rm; /* the query blocks whose rows are differentiated */
   const double* dout;
-  double *dq, *dk, *dv, *dgates;
-  int bad_index; /* set when an index is out of range */
+  double *dq, *dk, *dv, *dgates; /* dk, dv NULL: row-local gradients only */
+  int bad_index;                 /* set when an index is out of range */
 } bwd_ctx;
 
-/* One head: every row's forward again, then its gradients; the pooled summaries' gradients are
- * gathered over all rows and spread back over their blocks' tokens at the end. */
+/* One head: every chosen row's forward again, then its gradients; the pooled summaries'
+ * gradients are gathered over the rows and spread back over their blocks' tokens at the end. */
 static void bwd_task(void* vctx, int64_t h) {
   bwd_ctx* c = (bwd_ctx*)vctx;
   const s3r_ref_params* p = c->p;
-  const int64_t nb = s3r_ref_num_blocks(p), nqb = ceil_div(p->L, p->qblock);
+  const row_map* rm = c->rm;
+  const int64_t nb = s3r_ref_num_blocks(p);
   const int64_t H = p->H, d = p->d, HD = H * d;
   const int32_t n_list = p->forced + p->topk;
   double* sc = (double*)malloc(sizeof(double) * (size_t)nb);    /* compressed logits, then P */
@@ -516,9 +518,9 @@ static void bwd_task(void* vctx, int64_t h) {
   int64_t* tokens = (int64_t*)malloc(sizeof(int64_t) * (size_t)n_list * (size_t)p->block);
   double* ss = (double*)malloc(sizeof(double) * (size_t)n_list * (size_t)p->block);
 
-  for (int64_t i = 0; i < nqb; ++i) {
+  for (int64_t i = 0; i < rm->nq; ++i) {
     /* the query block's token set T, each selected block once */
-    const int32_t* sel = c->idx + (h * nqb + i) * n_list;
+    const int32_t* sel = c->idx + (h * rm->nq + i) * n_list;
     int64_t nt = 0;
     for (int64_t j = 0; j < nb; ++j) chosen[j] = 0;
     for (int32_t s = 0; s < n_list; ++s) {
@@ -531,8 +533,8 @@ static void bwd_task(void* vctx, int64_t h) {
       chosen[j] = 1;
       nt += s3r_ref_block_tokens(p, j, tokens + nt);
     }
-    const int64_t r1 = (i + 1) * p->qblock < p->L ? (i + 1) * p->qblock : p->L;
-    for (int64_t r = i * p->qblock; r < r1; ++r) {
+    for (int64_t rr = 0; rr < rm->count[i]; ++rr) {
+      const int64_t r = rm->first[i] + rr, o = rm->offset[i] + rr; /* sequence row, output row */
       for (int64_t e = 0; e < d; ++e) qv[e] = bf16_value(c->q[r * HD + h * d + e]);
       /* compressed branch: P over all nb summaries and O_cmp */
       double m = -INFINITY;
@@ -567,7 +569,7 @@ static void bwd_task(void* vctx, int64_t h) {
       /* gated aggregation: out = g0 O_cmp + g1 O_sel with g = sigmoid(logit) */
       const double g0 = sigmoid((double)c->gates[(r * H + h) * 2 + 0]);
       const double g1 = sigmoid((double)c->gates[(r * H + h) * 2 + 1]);
-      const double* dy = c->dout + r * HD + h * d;
+      const double* dy = c->dout + o * HD + h * d;
       double yc = 0.0, ys = 0.0;
       for (int64_t e = 0; e < d; ++e) {
         yc += dy[e] * oc[e];
@@ -575,11 +577,11 @@ static void bwd_task(void* vctx, int64_t h) {
         doc[e] = g0 * dy[e];
         dos[e] = g1 * dy[e];
       }
-      c->dgates[(r * H + h) * 2 + 0] = g0 * (1.0 - g0) * yc;
-      c->dgates[(r * H + h) * 2 + 1] = g1 * (1.0 - g1) * ys;
+      c->dgates[(o * H + h) * 2 + 0] = g0 * (1.0 - g0) * yc;
+      c->dgates[(o * H + h) * 2 + 1] = g1 * (1.0 - g1) * ys;
       /* softmax backward: dS = P (dP - <dO, O>), dP = <dO, value>; dq = scale sum dS key,
        * dkey = scale dS q, dvalue = P dO */
-      double* dqr = c->dq + r * HD + h * d;
+      double* dqr = c->dq + o * HD + h * d;
       for (int64_t e = 0; e < d; ++e) dqr[e] = 0.0;
       double dc = 0.0, ds = 0.0;
       for (int64_t e = 0; e < d; ++e) dc += doc[e] * oc[e], ds += dos[e] * os[e];
@@ -598,16 +600,18 @@ static void bwd_task(void* vctx, int64_t h) {
         double dp = 0.0;
         for (int64_t e = 0; e < d; ++e) dp += dos[e] * bf16_value(c->v[t * HD + h * d + e]);
         const double dsa = ss[a] * (dp - ds);
-        for (int64_t e = 0; e < d; ++e) {
+        for (int64_t e = 0; e < d; ++e)
           dqr[e] += p->scale * dsa * bf16_value(c->k[t * HD + h * d + e]);
-          c->dk[t * HD + h * d + e] += p->scale * dsa * qv[e];
-          c->dv[t * HD + h * d + e] += ss[a] * dos[e];
-        }
+        if (c->dk)
+          for (int64_t e = 0; e < d; ++e) {
+            c->dk[t * HD + h * d + e] += p->scale * dsa * qv[e];
+            c->dv[t * HD + h * d + e] += ss[a] * dos[e];
+          }
       }
     }
   }
   /* pooling backward: each summary is the mean of its block's tokens */
-  for (int64_t j = 0; j < nb; ++j) {
+  for (int64_t j = 0; c->dk && j < nb; ++j) {
     const int64_t n = s3r_ref_block_tokens(p, j, tokens);
     for (int64_t a = 0; a < n; ++a)
       for (int64_t e = 0; e < d; ++e) {
@@ -621,14 +625,23 @@ static void bwd_task(void* vctx, int64_t h) {
 
 int s3r_ref_bwd(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                 const double* kc, const double* vc, const float* gates, const int32_t* idx,
-                const double* dout, double* dq, double* dk, double* dv, double* dgates) {
-  if (check_params(p) || !q || !k || !v || !kc || !vc || !gates || !idx || !dout || !dq || !dk ||
-      !dv || !dgates || p->topk < 1 || p->forced < 0)
+                const int64_t* qblocks, int64_t nq, const double* dout, double* dq, double* dk,
+                double* dv, double* dgates) {
+  if (check_params(p) || !q || !k || !v || !kc || !vc || !gates || !idx || !dout || !dq ||
+      !dgates || p->topk < 1 || p->forced < 0)
     return -1;
-  const int64_t n = p->L * p->H * p->d;
-  for (int64_t e = 0; e < n; ++e) dk[e] = 0.0, dv[e] = 0.0;
-  bwd_ctx c = {p, q, k, v, kc, vc, gates, idx, dout, dq, dk, dv, dgates, 0};
+  /* dk, dv sum over every query: all blocks and both arrays, or a sample and neither */
+  if ((!dk) != (!dv) || (qblocks && dk) || (!qblocks && !dk)) return -1;
+  row_map rm;
+  int rc = row_map_make(p, qblocks, nq, &rm);
+  if (rc) return rc;
+  if (dk) {
+    const int64_t n = p->L * p->H * p->d;
+    for (int64_t e = 0; e < n; ++e) dk[e] = 0.0, dv[e] = 0.0;
+  }
+  bwd_ctx c = {p, q, k, v, kc, vc, gates, idx, &rm, dout, dq, dk, dv, dgates, 0};
   parallel_for(p->H, p->threads, bwd_task, &c); /* heads touch disjoint slices of every array */
+  row_map_free(&rm);
   return c.bad_index ? -3 : 0;
 }
 

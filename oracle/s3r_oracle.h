@@ -106,10 +106,15 @@ int s3r_ref_sel(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, c
  * top-k), and the bf16 rounding of the pooled K/V is passed straight through: kc, vc are the
  * pooled values the forward used (s3r_ref_pool), and dK[t] += dKc[j] / n_j for the n_j tokens t
  * of block j (the same for V). Returns 0, -1 on bad parameters, -3 when idx holds an index
- * outside [0, nb). */
+ * outside [0, nb).
+ * qblocks (nullable): differentiate only the rows of these nq query blocks. idx is then
+ * [H, nq, F + k] for them, dout, dq [R, H, d] and dgates [R, H, 2] hold their R rows
+ * concatenated in list order, and dk, dv must be NULL: they sum over every query. With
+ * qblocks NULL every array covers all L rows and dk, dv are required. */
 int s3r_ref_bwd(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                 const double* kc, const double* vc, const float* gates, const int32_t* idx,
-                const double* dout, double* dq, double* dk, double* dv, double* dgates);
+                const int64_t* qblocks, int64_t nq, const double* dout, double* dq, double* dk,
+                double* dv, double* dgates);
 
 /* Gated aggregation over n rows: out = sigmoid(g[...,0]) * o_cmp + sigmoid(g[...,1]) * o_sel. */
 int s3r_ref_combine(int64_t n, int32_t H, int32_t d, const double* o_cmp, const double* o_sel,

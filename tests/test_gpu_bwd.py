@@ -20,13 +20,10 @@ import torch
 from oracle import oracle as O
 from sparse_global_attention_s3r_b200 import api, synth
 
-from parity import f64, rel_l2
+from parity import check_grad, f64
 
 pytestmark = pytest.mark.gpu
 
-REL_L2 = 1e-2
-MAX_REL = 2e-2
-ABS_FLOOR = 1e-6
 
 CASES = {  # name: (L, H, b, k, forced, seed)
     "ragged_b64": (1000, 2, 64, 5, 0, 41),
@@ -61,16 +58,7 @@ def _dout(L, H, seed):
     return torch.randn((L, H, 64), generator=g).to(torch.bfloat16)
 
 
-def _check(name, got, ref):
-    got = f64(got)
-    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
-    scale = float(np.abs(ref).max())
-    err = float(np.abs(got - ref).max())
-    bound = MAX_REL * scale + ABS_FLOOR
-    assert err <= bound, f"{name}: max-abs {err:.3e} > {bound:.3e}"
-    if scale > 0:
-        r = rel_l2(got, ref)
-        assert r <= REL_L2, f"{name}: rel-L2 {r:.3e}"
+_check = check_grad
 
 
 def _run(dev, cfg, pb, x, seed):

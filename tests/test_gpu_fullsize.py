@@ -13,7 +13,7 @@ import torch
 from oracle import oracle as O
 from sparse_global_attention_s3r_b200 import api, synth
 
-from parity import check_output, check_selection
+from parity import check_grad, check_output, check_selection
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -71,3 +71,67 @@ def test_fused_path_at_workload_size(name):
     cond_out = O.combine(ref.o_cmp, o_sel, np.ascontiguousarray(gates[rows]))
     err = check_output(got_out, cond_out)
     print(f"{name}: {stats} {err}")
+
+
+BWD_FULL = {  # name: (L, H, b, k, seed, sampled query blocks[, 2-D geometry, forced views])
+    "n100": (137400, 16, 64, 32, 2, 16),
+    "n1000": (1374000, 16, 64, 32, 3, 8),
+    "vggt32_ref_windows": (43968, 16, 64, 16, 1, 16,
+                           dict(grid_h=37, grid_w=37, special=5, win_h=8), 1),
+}
+
+
+@pytest.mark.parametrize("name", list(BWD_FULL))
+def test_backward_at_workload_size(name):
+    """The backward at the workload sizes, after a save-for-backward forward as bench.py runs it.
+    dq and dgates of a row depend only on that row: on a seeded sample of query blocks (the
+    ragged last one included) they are compared with the oracle's, on the GPU's own lists, under
+    the backward bar. dk and dv sum over every query, so at these sizes they are checked by
+    properties that hold at any size: per head the key gradients sum to zero, and the value
+    gradients sum to sum_r (sigmoid(g0) + sigmoid(g1)) dout_r."""
+    import dataclasses
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    L, H, b, k, seed, nsample, *more = BWD_FULL[name]
+    geo = more[0] if more else {}
+    forced = more[1] * (api.Config(L=L, H=H, block=b, topk=1, **geo).nb // (L // (
+        geo["special"] + geo["grid_h"] * geo["grid_w"]))) if len(more) > 1 else 0
+    dev = torch.device("cuda")
+    x = synth.make_inputs(L, H, 64, b, seed, device=dev)
+    cfg = dataclasses.replace(api.Config(L=L, H=H, block=b, topk=k, forced=forced, **geo),
+                              save_for_backward=True)
+    ws = torch.empty(api.bwd_workspace_bytes(cfg), dtype=torch.uint8, device=dev)
+    idx = torch.empty((H, cfg.nqb, cfg.nsel), dtype=torch.int32, device=dev)
+    api.sparse_attn_fwd(cfg, x.q, x.k, x.v, x.gates, workspace=ws, idx_out=idx)
+    g = torch.Generator(device=dev).manual_seed(seed + 7)
+    dout = torch.randn(x.q.shape, generator=g, device=dev).to(torch.bfloat16)
+    dq, dk, dv, dg = api.sparse_attn_bwd(cfg, x.q, x.k, x.v, x.gates, idx, dout, workspace=ws)
+    torch.cuda.synchronize()
+    del ws
+
+    # invariants of dk, dv over the whole layer (fp64 sums on the GPU)
+    s_dk = dk.double().sum(0)
+    scale_k = dk.double().abs().sum(0)
+    assert float((s_dk.abs() / scale_k.clamp_min(1e-30)).max()) <= 1e-3
+    sg = torch.sigmoid(x.gates.double())
+    want_v = ((sg[..., :1] + sg[..., 1:]) * dout.double()).sum(0)
+    err_v = (dv.double().sum(0) - want_v).abs().max()
+    assert float(err_v) <= 1e-3 * float(dv.double().abs().sum(0).max()), float(err_v)
+
+    pb = O.Problem(L, H, 64, b, k, forced=forced, **geo)
+    rng = np.random.default_rng(seed)
+    blocks = sorted(set(rng.choice(cfg.nqb - 1, size=nsample - 1, replace=False).tolist())
+                    | {cfg.nqb - 1})
+    rows_t = torch.from_numpy(pb.rows_of(blocks)).to(dev)
+    got_dq = dq.index_select(0, rows_t)
+    got_dg = dg.index_select(0, rows_t)
+    dout_rows = dout.index_select(0, rows_t).double().cpu().numpy()
+    got_idx = np.ascontiguousarray(idx[:, blocks].cpu().numpy())
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    gates = x.gates.cpu().numpy()
+    del x, dq, dk, dv, dg, dout
+    torch.cuda.empty_cache()
+    ref = O.backward(pb, *bits, gates, got_idx, dout_rows, qblocks=blocks)
+    check_grad("dq", got_dq, ref.dq)
+    check_grad("dgates", got_dg, ref.dgates)

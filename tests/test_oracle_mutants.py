@@ -75,10 +75,14 @@ MUTANTS = {
         "c->dk[tokens[a] * HD + h * d + e] += dkc[j * d + e] / (double)n;",
         "c->dk[tokens[a] * HD + h * d + e] += dkc[j * d + e];"),
     "bwd_gate_derivative_drops_one_minus": (
-        "c->dgates[(r * H + h) * 2 + 0] = g0 * (1.0 - g0) * yc;",
-        "c->dgates[(r * H + h) * 2 + 0] = g0 * yc;"),
+        "c->dgates[(o * H + h) * 2 + 0] = g0 * (1.0 - g0) * yc;",
+        "c->dgates[(o * H + h) * 2 + 0] = g0 * yc;"),
     "bwd_sel_value_grad_ignores_gate": (
-        "c->dv[t * HD + h * d + e] += ss[a] * dos[e];", "c->dv[t * HD + h * d + e] += ss[a] * dy[e];"),
+        "c->dv[t * HD + h * d + e] += ss[a] * dos[e];",
+        "c->dv[t * HD + h * d + e] += ss[a] * dy[e];"),
+    "bwd_rows_use_the_first_query_row": (
+        "const int64_t r = rm->first[i] + rr, o = rm->offset[i] + rr;",
+        "const int64_t r = rm->first[i], o = rm->offset[i] + rr;"),
     "bwd_cmp_key_grad_misses_scale": (
         "dkc[j * d + e] += p->scale * dsj * qv[e];", "dkc[j * d + e] += dsj * qv[e];"),
     "bwd_sel_dq_from_values": (

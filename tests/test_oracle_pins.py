@@ -870,3 +870,19 @@ def test_bwd_rejects_an_out_of_range_index():
     idx[0, 1, 1] = pb.nb
     with pytest.raises(AssertionError, match="-3"):
         _bwd(pb, q, k, v, g, idx, dout)
+
+
+def test_bwd_sampled_query_blocks_equal_full_run():
+    """dq and dgates of a row depend only on that row: the backward of a sample of query blocks
+    (in any order, the partial last one included) gives exactly the full run's rows."""
+    pb = O.Problem(246, 2, 16, 32, 3, forced=1, grid_h=10, grid_w=12, special=3, win_h=4)
+    q, k, v, g, dout = _bwd_inputs(pb, 117)
+    fwd = O.sparse_attn(pb, q, k, v, g)
+    full, kc, vc = _bwd(pb, q, k, v, g, fwd.idx, dout)
+    qb = [3, 0, 2]  # nqb = 4; block 3 holds the last 54 rows
+    rows = pb.rows_of(qb)
+    part = O.backward(pb, q, k, v, g, np.ascontiguousarray(fwd.idx[:, qb]), dout[rows], kc=kc,
+                      vc=vc, qblocks=qb)
+    assert part.dk is None and part.dv is None
+    np.testing.assert_array_equal(part.dq, full.dq[rows])
+    np.testing.assert_array_equal(part.dgates, full.dgates[rows])
