@@ -160,6 +160,15 @@ def test_save_for_backward_workspaces(L, H, b, k):
     assert lib.s3r_sparse_attn_bwd(p, *[A16] * 10, A256, fwd_s, None) == _lib.S3R_ERR_WORKSPACE
 
 
+def test_save_for_backward_needs_the_slot_copies():
+    """The saving forward keeps the slot-order K/V copies for the backward: sizes whose copies
+    exceed 32-bit row coordinates are rejected before any launch."""
+    lib = _lib.load()
+    big = _params(L=65536, H=65535, block=64, topk=1, flags=_lib.S3R_FLAG_SAVE_FOR_BWD)
+    assert lib.s3r_sparse_attn_fwd(ctypes.byref(big), A16, A16, A16, A16, A16, None, A256,
+                                   1 << 62, None) == _lib.S3R_ERR_UNSUPPORTED
+
+
 def test_bwd_rejects_slot_copies_beyond_32_bit_rows():
     lib = _lib.load()
     big = _params(L=65536, H=65535, block=64, topk=1)  # H * nb * b = 65535 * 65536 > 2^31 - 1
