@@ -280,7 +280,9 @@ class SparseAttentionFunction(torch.autograd.Function):
 
     Gradients are returned in the inputs' dtypes (bf16 for q, k, v; fp32 for the gate logits).
     The top-k selection passes no gradient. The forward runs with save_for_backward and keeps
-    its workspace, so the backward does not recompute the forward."""
+    its workspace until the backward, which then does not recompute the forward. That is
+    bwd_workspace_bytes(cfg) bytes, about 816 per (token, head): O_cmp and O_sel in fp32, the
+    slot-order K/V copies, the lse and the backward's scratch."""
 
     @staticmethod
     def forward(ctx, q, k, v, gates, cfg: Config):
