@@ -886,3 +886,42 @@ def test_bwd_sampled_query_blocks_equal_full_run():
     assert part.dk is None and part.dv is None
     np.testing.assert_array_equal(part.dq, full.dq[rows])
     np.testing.assert_array_equal(part.dgates, full.dgates[rows])
+
+
+def test_bwd_random_configurations_equal_autograd():
+    """Seeded small configurations across every axis at once (block size, top-k, forced blocks,
+    1-D or 2-D geometry with special tokens and cut windows, ragged tails, scale): the oracle's
+    gradients equal torch autograd of the torch restatement of the forward."""
+    rng = np.random.default_rng(2024)
+    for trial in range(8):
+        b = int(rng.choice([8, 16, 32]))
+        if trial % 2:  # 2-D windows
+            wh = int(rng.choice([w for w in (1, 2, 4, 8) if b % w == 0]))
+            gh, gw = int(rng.integers(2, 9)), int(rng.integers(2, 12))
+            special = int(rng.integers(0, min(b, 6) + 1))
+            N = int(rng.integers(1, 4))
+            geo = dict(grid_h=gh, grid_w=gw, special=special, win_h=wh)
+            L = N * (special + gh * gw)
+        else:
+            geo = {}
+            L = int(rng.integers(20, 200))
+        nb = O.Problem(L, 1, 16, b, 1, **geo).nb
+        forced = int(rng.integers(0, min(3, nb - 1) + 1)) if nb > 1 else 0
+        k = int(rng.integers(1, nb - forced + 1))
+        H = int(rng.integers(1, 3))
+        scale = None if trial % 3 else float(rng.uniform(0.05, 0.4))
+        pb = O.Problem(L, H, 16, b, k, qblock=int(rng.choice([16, 32, 64])), scale=scale,
+                       forced=forced, **geo)
+        q, kk, v, g, dout = _bwd_inputs(pb, 300 + trial)
+        kc = O.pool(pb, kk, exact=True)
+        vc = O.pool(pb, v, exact=True)
+        fwd = O.sparse_attn(pb, q, kk, v, g, pooled=(kc, vc))
+        leaves = _leaves(q, kk, v, g)
+        out = _torch_path(pb, *leaves, fwd.idx)
+        np.testing.assert_allclose(out.detach().numpy(), fwd.out, rtol=0, atol=1e-12)
+        (out * torch.from_numpy(dout)).sum().backward()
+        gr = O.backward(pb, q, kk, v, g, fwd.idx, dout, kc=kc, vc=vc)
+        for name, mine, ref in zip(["dq", "dk", "dv", "dgates"],
+                                   [gr.dq, gr.dk, gr.dv, gr.dgates], leaves):
+            np.testing.assert_allclose(mine, ref.grad.numpy(), rtol=0, atol=1e-11,
+                                       err_msg=f"trial {trial}: {name} {pb}")
