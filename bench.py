@@ -13,8 +13,9 @@ Prints one JSON line (rank 0) with:
 
 - tokens/s, algorithmic TFLOP/s and fraction of the measured bf16 peak;
 - per-stage times from CUDA events recorded inside the fused call;
-- the roofline of the dominant kernel (for the compressed branch its exp2 rate against the MUFU
-  peak, with the tensor view beside it) and that kernel's recorded DRAM traffic;
+- the roofline of the dominant kernel (algorithmic bf16 FLOPs against the measured sustained
+  tensor peak; for the compressed branch also its exp2 rate), both attention branches' fraction
+  of that peak next to the 0.5 target, and the dominant kernel's recorded DRAM traffic;
 - an end-to-end figure from pinned host memory through HostPipeline;
 - dense attention (torch SDPA, flash) on the same inputs as context;
 - the fp64 CPU oracle's timed sample;
@@ -24,6 +25,8 @@ Prints one JSON line (rank 0) with:
 Other workloads:
 
 - n100, vggt32, tiny;
+- n1000_k40, n100_k40: top-k = 40, which writes the score matrix and runs the stand-alone top-k
+  kernel;
 - n1000_windows: 2-D key windows;
 - vggt32_ref, vggt32_ref_windows: the reference view kept;
 - pi3_sweep: 24 layers per (b, top-k) setting at 200 views.
@@ -60,8 +63,16 @@ WORKLOADS = {
     "n1000": dict(desc="1000-view sequence: N=1000 views x P=1374 tokens (37x37 patches + 5), "
                        "L=1,374,000, H=16, d=64, b=64, top-k=32, 1 layer",
                   L=1374000, H=16, block=64, topk=32, seed=3),
+    # the same layer with top-k = 40: above the 32 the compressed branch selects on the fly, so
+    # the [H, nqb, nb] score matrix (29.5 GB) is written and the stand-alone top-k kernel reads it
+    "n1000_k40": dict(desc="1000-view sequence, top-k=40 (score matrix + stand-alone top-k): "
+                           "L=1,374,000, H=16, d=64, b=64, 1 layer",
+                      L=1374000, H=16, block=64, topk=40, seed=3),
     "n100": dict(desc="100-view layer: L=137,400, H=16, d=64, b=64, top-k=32",
                  L=137400, H=16, block=64, topk=32, seed=2),
+    "n100_k40": dict(desc="100-view layer, top-k=40 (score matrix + stand-alone top-k): "
+                          "L=137,400, H=16, d=64, b=64",
+                     L=137400, H=16, block=64, topk=40, seed=2),
     "vggt32": dict(desc="VGGT-like layer: N=32 views x P=1374, L=43,968, H=16, d=64, b=64, top-k=16",
                    L=43968, H=16, block=64, topk=16, seed=1),
     # VGGT's hybrid: the reference view's blocks kept for every query (ceil(1374/64) = 22 leading
@@ -101,8 +112,8 @@ def load_peaks():
     return p
 
 
-# MUFU.EX2 issue rate of one SM per clock (4 sub-partitions x 4 lanes; 15.8 measured with a
-# dependent-free ex2.approx loop over all 148 SMs at 1965 MHz) and the SM count of a B200.
+# MUFU.EX2 rate of one SM per clock (4 sub-partitions x 4 lanes), as tests/test_gpu_exp2_rate.py
+# measures it in SM clock cycles, and the SM count of a B200.
 EX2_PER_CLK_SM = 16
 SM_COUNT = 148
 
@@ -347,35 +358,83 @@ class ClockSampler:
 # the CPU oracle, timed on a bounded sample of the workload
 # ---------------------------------------------------------------------------------------------
 
-def oracle_sample(cfg, host_bits, gates_np, n_blocks: int, seed: int):
-    """Time the oracle: pooling of all K/V plus the whole path for n_blocks query blocks (all
-    heads). Returns (tokens/s extrapolated to the full layer, seconds, description, threads)."""
+def sample_blocks(nqb: int, n_blocks: int, seed: int):
+    """A seeded sample of whole query blocks, the ragged last one always included."""
     import numpy as np
 
+    rng = np.random.default_rng(seed)
+    return sorted(set(rng.choice(nqb - 1, size=max(0, min(n_blocks, nqb) - 1),
+                                 replace=False).tolist() if nqb > 1 else []) | {nqb - 1})
+
+
+def oracle_sample(cfg, host_bits, gates_np, n_blocks: int, seed: int, result=None):
+    """Time the oracle: pooling of all K/V plus the whole path for n_blocks query blocks (all
+    heads). Returns (tokens/s extrapolated to the full layer, seconds, description, threads);
+    `result`, a dict, receives the sampled blocks and the oracle's outputs for them."""
     from oracle import oracle as O
 
     pb = O.Problem(cfg.L, cfg.H, cfg.d, cfg.block, cfg.topk, forced=cfg.forced, grid_h=cfg.grid_h,
                    grid_w=cfg.grid_w, special=cfg.special, win_h=cfg.win_h)
-    rng = np.random.default_rng(seed)
-    blocks = sorted(set(rng.choice(cfg.nqb - 1, size=max(0, min(n_blocks, cfg.nqb) - 1),
-                                   replace=False).tolist()
-                        if cfg.nqb > 1 else []) | {cfg.nqb - 1})
+    blocks = sample_blocks(cfg.nqb, n_blocks, seed)
     q, k, v = host_bits
     t0 = time.perf_counter()
     kc = O.pool(pb, k)
     vc = O.pool(pb, v)
     t1 = time.perf_counter()
-    O.sparse_attn(pb, q, k, v, gates_np, qblocks=blocks, pooled=(kc, vc))
+    ref = O.sparse_attn(pb, q, k, v, gates_np, qblocks=blocks, pooled=(kc, vc))
     t2 = time.perf_counter()
     rows = int(pb.rows_of(blocks).size)
     t_full = (t1 - t0) + (t2 - t1) * cfg.L / rows
     desc = (f"pooling of all {cfg.nb} K/V blocks + the whole path for {len(blocks)} seeded query "
             f"blocks ({rows} rows, all {cfg.H} heads); extrapolated to L={cfg.L}")
+    if result is not None:
+        result.update(blocks=blocks, rows=pb.rows_of(blocks), ref=ref)
     return cfg.L / t_full, t2 - t0, desc, O.hardware_threads()
 
 
+def parity_stats(got_idx, got_out, ref, forced: int) -> dict:
+    """The GPU's lists and output on the oracle's sampled query blocks, against the oracle run on
+    its own lists: the fraction of query blocks with the same selected set, the fraction whose
+    k-th/(k+1)-th score gap exceeds 1e-4 (where the sets must agree), and the output's max-abs
+    and relative-L2 error over the query blocks whose sets agree."""
+    import numpy as np
+
+    g = np.sort(got_idx[..., forced:], -1)
+    r = np.sort(ref.idx[..., forced:], -1)
+    same = (g == r).all(-1)                       # [H, nq]
+    out, want = np.asarray(got_out, np.float64), np.asarray(ref.out, np.float64)
+    # a row of a query block, head h, counts where that block's set agrees for head h
+    qb_of_row = ref.rows // 64
+    pos = np.searchsorted(np.unique(qb_of_row), qb_of_row)
+    mask = same[:, pos].T[..., None]              # [R, H, 1]
+    diff = np.where(mask, out - want, 0.0)
+    ref_m = np.where(mask, want, 0.0)
+    return {"query_blocks": int(same.shape[1]), "sets_equal": float(same.mean()),
+            "gap_separated": float((ref.gap > 1e-4).mean()),
+            "max_abs": float(np.abs(diff).max()),
+            "rel_l2": float(np.sqrt((diff ** 2).sum() / max((ref_m ** 2).sum(), 1e-300)))}
+
+
+def workload_config(wl, world: int, l2_note: str) -> dict:
+    """The `config` object of the JSON line: the same keys and values in both arms."""
+    return {"workload": wl["desc"], "L": wl["L"], "H": wl["H"], "d": 64, "block": wl["block"],
+            "topk": wl["topk"], "forced": wl.get("forced", 0), "qblock": 64, "seed": wl["seed"],
+            **wl.get("geo", {}),
+            "parallelism": "independent layer per GPU" if world > 1 else "single GPU",
+            "l2": l2_note}
+
+
+def l2_note(L: int, H: int) -> str:
+    gb = L * H * 64 * 2 / 1e9
+    if gb > 0.126:
+        return "inputs exceed L2 (each of Q/K/V is %.2f GB > 126 MB); no flush" % gb
+    return "inputs fit in L2 (each of Q/K/V is %.1f MB); no flush" % (gb * 1e3)
+
+
 def run_reference(args, wl):
-    """--impl reference: the CPU oracle on bounded samples; rank 0 only."""
+    """--impl reference: the CPU oracle on bounded samples; rank 0 only. Nothing of the CUDA
+    library is loaded on this path: sizes come from the oracle's own Problem, inputs from the
+    seeded generator (on the GPU when there is one, so that they equal the native arm's)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -383,33 +442,34 @@ def run_reference(args, wl):
     import torch
 
     from oracle import oracle as O
-    from sparse_global_attention_s3r_b200 import api, synth
+    from sparse_global_attention_s3r_b200 import synth
 
-    cfg = api.Config(L=wl["L"], H=wl["H"], block=wl["block"], topk=wl["topk"],
-                     forced=wl.get("forced", 0), **wl.get("geo", {}))
+    pb = O.Problem(wl["L"], wl["H"], 64, wl["block"], wl["topk"], forced=wl.get("forced", 0),
+                   **wl.get("geo", {}))
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    x = synth.make_inputs(cfg.L, cfg.H, cfg.d, cfg.block, wl["seed"], device=dev)
+    x = synth.make_inputs(pb.L, pb.H, pb.d, pb.block, wl["seed"], device=dev)
     bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
     gates = x.gates.cpu().numpy()
     del x
-    n_blocks = max(1, min(4, cfg.nqb))
+    n_blocks = max(1, min(4, pb.nqb))
     for w in range(args.warmup):
-        oracle_sample(cfg, bits, gates, n_blocks, seed=w)
+        oracle_sample(pb, bits, gates, n_blocks, seed=w)
     vals, secs = [], []
     desc = threads = None
     for s in range(args.steps):
-        v, t, desc, threads = oracle_sample(cfg, bits, gates, n_blocks, seed=100 + s)
+        v, t, desc, threads = oracle_sample(pb, bits, gates, n_blocks, seed=100 + s)
         vals.append(v)
         secs.append(t)
     value = statistics.median(vals)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * cfg.L / value, "higher_is_better": True, "scaling": "weak",
+        # the seconds one sampled step really took; the full layer is extrapolated below
+        "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl["desc"], "L": cfg.L, "H": cfg.H, "d": cfg.d,
-                   "block": cfg.block, "topk": cfg.topk, "qblock": 64, "seed": wl["seed"],
-                   **wl.get("geo", {})},
+        "config": workload_config(wl, world, l2_note(pb.L, pb.H)),
+        "extrapolated_full_layer_ms": 1e3 * pb.L / value,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": desc + f"; median of {args.steps} samples of "
                                           f"{statistics.median(secs):.1f} s"},
@@ -474,6 +534,14 @@ def run_native(args, wl):
     barrier()
     ms_max = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
     stage_ms = {n: statistics.mean(e.stage_ms()[n] for e in stage_ev) for n in _lib.STAGES}
+    step_ms = [sum(e.stage_ms().values()) for e in stage_ev]
+    # the GPU's lists and output on the query blocks the CPU-baseline leg will give the oracle
+    do_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    got = None
+    if do_cpu:
+        blocks = sample_blocks(cfg.nqb, args.oracle_blocks, 7)
+        rows = torch.cat([torch.arange(64 * i, min(64 * i + 64, cfg.L)) for i in blocks]).to(dev)
+        got = (sa.idx[:, blocks].cpu().numpy(), sa.out.index_select(0, rows).double().cpu().numpy())
     bwd = (time_backward(args, cfg, q, k, v, gates, sa.idx, dev, barrier, load_peaks())
            if not args.no_backward else None)
 
@@ -532,16 +600,18 @@ def run_native(args, wl):
             dense = {"unavailable": str(e).splitlines()[0][:200]}
         del qh, kh_, vh_
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    cpu = parity = None
+    if do_cpu:
         from oracle import oracle as O
 
         bits = [O.bf16_bits(t_) for t_ in (q, k, v)]
+        res = {}
         val, secs, desc, threads = oracle_sample(cfg, bits, gates.cpu().numpy(),
-                                                 args.oracle_blocks, seed=7)
+                                                 args.oracle_blocks, seed=7, result=res)
         cpu = {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": desc + f"; {secs:.1f} s of CPU work"}
-        del bits
+        parity = parity_stats(*got, res["ref"], cfg.forced)
+        del bits, res
 
     if world > 1:
         dist.barrier()
@@ -565,17 +635,24 @@ def run_native(args, wl):
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = peaks["source"] + (" sustained bf16" if bound == "tensor" else " copy")
     if dom == "cmp":
-        # The compressed branch needs two exponentials per (query, summary) pair. Their unit
-        # (MUFU.EX2, 16 per clock per SM) sets its speed of light, 203 ms at 1000 views, well above
-        # the tensor work's 110-130 ms: the binding roofline is this ALU one; the tensor view
-        # (the algorithmic bf16 FLOPs against the measured GEMM peak) is kept beside it.
+        # The compressed branch needs two exponentials per (query, summary) pair; their units
+        # (MUFU.EX2 at 16 per clock per SM, tests/test_gpu_exp2_rate.py, plus the part evaluated
+        # as a polynomial on the FMA pipe) bound it before its tensor work does. That exp2 rate
+        # is reported beside the tensor roofline, not instead of it.
         ex2_peak = EX2_PER_CLK_SM * SM_COUNT * peaks.get("sm_max_mhz", 1965.0) * 1e6
         ach = work["cmp_exp2"] / dom_s
-        tensor_view = dict(roof)
-        roof = {"bound": "alu", "what": "exp2 on the MUFU pipe", "achieved": ach / 1e12,
-                "peak": ex2_peak / 1e12, "unit": "Texp2/s", "frac": ach / ex2_peak,
-                "peak_source": "16 ex2 per clock per SM x 148 SMs x max SM clock",
-                "tensor_view": tensor_view}
+        roof["exp2_view"] = {"achieved": ach / 1e12, "unit": "Texp2/s",
+                             "mufu_peak": ex2_peak / 1e12, "frac_of_mufu": ach / ex2_peak,
+                             "mufu_peak_source": "16 ex2 per clock per SM (measured by "
+                                                 "tests/test_gpu_exp2_rate.py) x 148 SMs x max "
+                                                 "SM clock"}
+    # both attention branches against the measured sustained bf16 peak (the stated target: 0.5)
+    two_ms = stage_ms["cmp"] + stage_ms["sel_combine"]
+    if two_ms > 0:
+        two = work["flops"] / (two_ms / 1e3) / 1e12
+        roof["two_branches"] = {"stages": ["cmp", "sel_combine"], "ms": two_ms,
+                                "achieved": two, "unit": "TFLOP/s",
+                                "frac": two / peaks["bf16_tflops_sustained"], "target_frac": 0.5}
     roof["traffic"] = measured_traffic(dom, args.workload)
     roof["kernel"] = dom
     stages = {}
@@ -592,14 +669,9 @@ def run_native(args, wl):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": wl["desc"], "L": cfg.L, "H": cfg.H, "d": cfg.d, "block": cfg.block,
-                   "topk": cfg.topk, "forced": cfg.forced, "qblock": 64, "seed": wl["seed"],
-                   **wl.get("geo", {}),
-                   "kernels": "pool + one fused kernel" if args.single_kernel else
-                              "pool + compressed/top-k + selection/combine",
-                   "parallelism": "independent layer per GPU" if world > 1 else "single GPU",
-                   "l2": "inputs exceed L2 (each of Q/K/V is %.2f GB > 126 MB); no flush" %
-                         (q.numel() * 2 / 1e9)},
+        "config": workload_config(wl, world, l2_note(cfg.L, cfg.H)),
+        "kernels": "pool + one fused kernel" if args.single_kernel else
+                   "pool + compressed/top-k + selection/combine",
         "tflops": tflops,
         "frac_bf16_peak": tflops / world / peaks["bf16_tflops"],
         "frac_bf16_peak_sustained": tflops / world / peaks["bf16_tflops_sustained"],
@@ -617,7 +689,21 @@ def run_native(args, wl):
     }
     if bwd is not None:
         line["backward"] = bwd
+    if parity is not None:
+        line["parity"] = parity
     print(json.dumps(line), flush=True)
+    if args.records:  # one record per (config, timed step), appended
+        with open(args.records, "a") as f:
+            for s_, ms_ in enumerate(step_ms):
+                rec = {"workload": args.workload, "config": line["config"], "step": s_,
+                       "ms": ms_, "tokens_per_s": cfg.L / (ms_ / 1e3),
+                       "tflops": work["flops"] / (ms_ / 1e3) / 1e12,
+                       "frac_bf16_sustained": work["flops"] / (ms_ / 1e3) / 1e12
+                       / peaks["bf16_tflops_sustained"],
+                       "stage_ms": {n: e_ for n, e_ in stage_ev[s_].stage_ms().items()},
+                       "stage_rates": stages, "parity": parity,
+                       "host_cores": cpu["cores"] if cpu else None, "clocks": line["clocks"]}
+                f.write(json.dumps(rec) + "\n")
 
 
 # the pi^3-like sweep at N = 200 views (L = 274,800, H = 16): each (b, top-k) setting is a stack of
@@ -678,6 +764,38 @@ def run_sweep(args):
     print(json.dumps(line))
 
 
+def run_sweep_records(args):
+    """--sweep: run each named workload in its own process, appending to --records; a workload
+    whose records are already in the file is skipped, so an interrupted sweep resumes."""
+    if not args.records:
+        raise SystemExit("--sweep needs --records")
+    names = [n.strip() for n in args.sweep.split(",") if n.strip()]
+    unknown = [n for n in names if n not in WORKLOADS]
+    if unknown:
+        raise SystemExit(f"unknown workloads: {unknown}")
+    done = set()
+    if os.path.exists(args.records):
+        with open(args.records) as f:
+            for ln in f:
+                try:
+                    done.add(json.loads(ln)["workload"])
+                except (ValueError, KeyError):
+                    continue
+    passthrough = ["--steps", str(args.steps), "--warmup", str(args.warmup),
+                   "--oracle-blocks", str(args.oracle_blocks)]
+    for flag in ("no_cpu_baseline", "no_backward", "no_dense_context", "single_kernel"):
+        if getattr(args, flag):
+            passthrough.append("--" + flag.replace("_", "-"))
+    for n in names:
+        if n in done:
+            print(f"sweep: {n} already recorded, skipped", flush=True)
+            continue
+        r = subprocess.run([sys.executable, os.path.abspath(__file__), "--workload", n,
+                            "--records", args.records] + passthrough)
+        if r.returncode != 0:
+            raise SystemExit(f"sweep: {n} failed with exit code {r.returncode}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -696,7 +814,14 @@ def main():
                     help="skip timing dense attention (torch SDPA) on a sample of query rows")
     ap.add_argument("--dense-rows", type=int, default=16384,
                     help="query rows of the dense-attention context sample")
+    ap.add_argument("--records", default=None,
+                    help="append one JSON record per (workload, timed step) to this file")
+    ap.add_argument("--sweep", default=None,
+                    help="comma-separated workloads, each run in its own process with --records; "
+                         "workloads already in the records file are skipped (resume)")
     args = ap.parse_args()
+    if args.sweep:
+        return run_sweep_records(args)
     if args.workload == "pi3_sweep":
         if args.impl == "reference":
             raise SystemExit("--impl reference times the oracle on the single-layer workloads")

@@ -34,17 +34,20 @@
  * Conventions:
  *   - Every pointer argument is a DEVICE pointer of the current CUDA device, 16-byte aligned,
  *     to a dense row-major array; the caller owns every buffer. The library never allocates or
- *     frees device memory and never synchronises the stream.
+ *     frees device memory. Only s3r_read_device_status and s3r_last_device_error synchronise the
+ *     stream (they read a word the stream's kernels write); every other call is asynchronous.
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream). The return value
  *     reports host-side validation and launch errors only; a call that returns an error has
  *     launched nothing, except S3R_ERR_CUDA which reports a failed launch.
  *   - Conditions detected on the device (a bounded wait that expired, an out-of-range index when
  *     S3R_FLAG_DEBUG_CHECKS is set) are OR-ed into the 32-bit word params->dev_status when it is
  *     non-NULL, and into the workspace's status word in s3r_sparse_attn_fwd. Read it with
- *     s3r_read_device_status after the stream has finished.
+ *     s3r_read_device_status (or s3r_last_device_error).
  *   - bf16 values are passed as their 16-bit patterns (s3r_bf16).
- *   - No C++ exception crosses this boundary; the functions are thread-safe (no global state
- *     besides a launch counter).
+ *   - No C++ exception crosses this boundary. The functions are thread-safe. The global state is
+ *     a launch counter and, for s3r_sparse_attn_fwd_static only, one device array per GPU with a
+ *     per-device table of its address; calls of that entry point that overlap on the GPU race
+ *     on the array (see its comment). Every other entry point works on caller buffers only.
  */
 #ifndef S3R_H
 #define S3R_H
@@ -74,10 +77,11 @@ typedef enum {
 
 /* params.flags */
 #define S3R_FLAG_DEBUG_CHECKS 0x1u /* validate idx on the device in s3r_sel_attn */
-#define S3R_FLAG_TEST_TIMEOUT 0x2u /* testing only: the compressed-branch and selection kernels
-                                      wait on a barrier that nothing signals, with a 1 ms limit, so
-                                      their timeout paths run: S3R_DEV_TIMEOUT is set and the
-                                      outputs are invalid */
+#define S3R_FLAG_TEST_TIMEOUT 0x2u /* testing only: the tensor-core kernels (compressed branch,
+                                      selection, the single fused kernel, and the backward's dq,
+                                      dKc/dVc and dk/dv kernels) wait on a barrier that nothing
+                                      signals, with a 1 ms limit, so their timeout paths run:
+                                      S3R_DEV_TIMEOUT is set and the outputs are invalid */
 #define S3R_FLAG_SINGLE_KERNEL 0x4u /* s3r_sparse_attn_fwd with topk <= 32: after pooling, one
                                        kernel per (query tile, head) runs the compressed branch,
                                        the top-k and the selection branch with the gated combine,
@@ -90,6 +94,12 @@ typedef enum {
                                        skips recomputing the forward. The workspace then grows
                                        (s3r_workspace_bytes reports it); S3R_FLAG_SINGLE_KERNEL
                                        is ignored (the 3-kernel path runs) */
+
+#define S3R_FLAG_NVTX 0x10u         /* s3r_sparse_attn_fwd and s3r_sparse_attn_bwd push one NVTX
+                                       range per stage ("s3r.pool", "s3r.cmp", ...), so profilers
+                                       (ncu --nvtx, nsys) can attribute kernels to stages; off by
+                                       default (the ranges cost host time only when a tool is
+                                       attached) */
 
 typedef struct {
   int64_t L;      /* tokens = N views * P tokens per view, >= 1 */
@@ -164,6 +174,13 @@ s3r_status s3r_read_device_status(uint32_t* dev_status, s3r_stream stream, uint3
 
 /* Device status word inside a workspace given to s3r_sparse_attn_fwd. */
 uint32_t* s3r_workspace_status_word(void* workspace);
+
+/* The same read as s3r_read_device_status, returning only the status: synchronise `stream`, read
+ * and clear the 32-bit device word at flag_buf (params->dev_status, or a workspace's word), and
+ * map its bits to a status: S3R_ERR_TIMEOUT if a bounded wait expired, S3R_ERR_INVALID_ARG if a
+ * debug check found an index outside [0, nb), S3R_OK if neither. A NULL or misaligned flag_buf is
+ * S3R_ERR_INVALID_ARG; a failed copy S3R_ERR_CUDA. */
+s3r_status s3r_last_device_error(void* flag_buf, s3r_stream stream);
 
 /* Compression branch, pooling ("Compressie-tak": average pooling).
  *   k, v         [L, H, d] bf16 (read)
@@ -267,9 +284,18 @@ s3r_status s3r_sparse_attn_bwd(const s3r_params* params, const s3r_bf16* q, cons
  * S3R_STATIC_WORKSPACE_BYTES inside the library, present on every GPU that loads the library
  * until the process exits. It allocates nothing.
  *   Sizes whose workspace (s3r_workspace_bytes) exceeds S3R_STATIC_WORKSPACE_BYTES are rejected
- *   with S3R_ERR_WORKSPACE before anything is launched; other arguments as s3r_sparse_attn_fwd.
+ *   with S3R_ERR_WORKSPACE before anything is launched; other arguments as s3r_sparse_attn_fwd,
+ *   with three more rules, each checked before any launch:
+ *     - params->dev_status must be a device word of the caller (S3R_ERR_INVALID_ARG if NULL):
+ *       the array's own status word is not visible to the caller, so an expired bounded wait
+ *       is reported only there;
+ *     - S3R_FLAG_SAVE_FOR_BWD is rejected with S3R_ERR_UNSUPPORTED: what it keeps would live in
+ *       the shared array, which s3r_sparse_attn_bwd cannot be given and the next call overwrites;
+ *     - `stream` (if not NULL) must belong to the current device (S3R_ERR_INVALID_ARG).
  *   The first call on a device looks up the array's device address on that device (the current
- *   one); make that first call before any stream capture.
+ *   one) and keeps it for the life of the process; make that first call before any stream
+ *   capture. After a cudaDeviceReset of that device the kept address is stale: do not call this
+ *   entry point on that device again in the same process.
  *   All calls share the one array per device and it keeps the last call's contents (the parts
  *   that must start at zero are cleared by every call). Calls whose executions overlap on the GPU
  *   (different streams, or different host threads) race on it: serialise them. */

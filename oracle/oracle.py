@@ -68,6 +68,8 @@ def lib():
             "s3r_ref_combine": [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, p, p, p, p],
             "s3r_ref_block_tokens": [p, ctypes.c_int64, p],
             "s3r_ref_bwd": [p, p, p, p, p, p, p, p, p, ctypes.c_int64, p, p, p, p, p],
+            "s3r_ref_bwd_keys": [p, p, p, p, p, p, p, p, ctypes.c_int32, p, ctypes.c_int64, p, p,
+                                 p],
         }.items():
             fn = getattr(L, name)
             fn.restype = ctypes.c_int
@@ -290,6 +292,40 @@ def backward(pb: Problem, q_bits, k_bits, v_bits, gates, idx, dout, kc=None, vc=
                            _ptr(g.dgates))
     assert rc == 0, rc
     return g
+
+
+def backward_keys(pb: Problem, q_bits, k_bits, v_bits, gates, idx, dout, head: int, kblocks,
+                  kc=None, vc=None, threads: int = 0):
+    """dk, dv of one head for the tokens of the key blocks `kblocks` (float64), the same
+    gradients as ``backward`` without forming the other blocks': the compressed branch summed over
+    every row, spread over each block's tokens through the pooled mean, plus the selection branch
+    of the query blocks whose lists hold the block. idx is the full [H, nqb, forced + topk], dout
+    the full [L, H, d]. Returns (dk, dv), each [len(kblocks), block, d]: row u of entry a is the
+    u-th token of block kblocks[a] (``Problem.block_tokens`` order); rows past its count are 0."""
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    k_bits = np.ascontiguousarray(k_bits, dtype=np.uint16)
+    v_bits = np.ascontiguousarray(v_bits, dtype=np.uint16)
+    if kc is None:
+        kc = pool(pb, k_bits, threads=threads)
+    if vc is None:
+        vc = pool(pb, v_bits, threads=threads)
+    kc = np.ascontiguousarray(kc, dtype=np.float64)
+    vc = np.ascontiguousarray(vc, dtype=np.float64)
+    gates = np.ascontiguousarray(gates, dtype=np.float32)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    dout = np.ascontiguousarray(dout, dtype=np.float64)
+    kb = np.ascontiguousarray(kblocks, dtype=np.int64)
+    shape = (pb.L, pb.H, pb.d)
+    assert q_bits.shape == shape and dout.shape == shape and gates.shape == (pb.L, pb.H, 2)
+    assert idx.shape == (pb.H, pb.nqb, pb.nsel), idx.shape
+    dk = np.empty((kb.size, pb.block, pb.d))
+    dv = np.empty((kb.size, pb.block, pb.d))
+    rc = lib().s3r_ref_bwd_keys(ctypes.byref(_params(pb, threads=threads)), _ptr(q_bits),
+                                _ptr(k_bits), _ptr(v_bits), _ptr(kc), _ptr(vc), _ptr(gates),
+                                _ptr(idx), int(head), _ptr(kb), kb.size, _ptr(dout), _ptr(dk),
+                                _ptr(dv))
+    assert rc == 0, rc
+    return dk, dv
 
 
 @dataclass

@@ -47,6 +47,8 @@
  *                       off (dense selection; attention over torch-pooled means); key gradients
  *                       summing to zero and value gradients conserving the gated mass; equal
  *                       values giving no query/key gradient.
+ *   s3r_ref_bwd_keys    equal to the rows of s3r_ref_bwd's dk, dv for the listed blocks (1-D,
+ *                       forced blocks, 2-D windows, ragged tail).
  * The backward (the path is trained end to end, arXiv abstract) holds the selection lists fixed,
  * since a top-k has no gradient, and passes the bf16 rounding of the pooled K/V straight through.
  */
@@ -642,6 +644,197 @@ int s3r_ref_bwd(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, c
   bwd_ctx c = {p, q, k, v, kc, vc, gates, idx, &rm, dout, dq, dk, dv, dgates, 0};
   parallel_for(p->H, p->threads, bwd_task, &c); /* heads touch disjoint slices of every array */
   row_map_free(&rm);
+  return c.bad_index ? -3 : 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* backward, key side only: dk, dv of the tokens of a few key blocks of one head               */
+/* ------------------------------------------------------------------------------------------ */
+
+/* The same gradients as s3r_ref_bwd, for one head and the tokens of the listed key blocks only,
+ * so that they can be checked at sizes where the full backward is out of reach. A token t of
+ * block j receives:
+ *   from the compressed branch, through the pooled mean: (scale sum_r dS_rj q_r) / n_j for dk and
+ *     (sum_r P_rj g0_r dout_r) / n_j for dv, summed over every row r of the sequence;
+ *   from the selection branch: scale sum_r dS_rt q_r and sum_r P_rt g1_r dout_r, summed over the
+ *     rows r of the query blocks whose lists hold block j.
+ * Work is split over row chunks (compressed branch, partial sums added in chunk order) and over
+ * the listed blocks (selection branch), which does not change the arithmetic of any term. */
+typedef struct {
+  const s3r_ref_params* p;
+  const uint16_t *q, *k, *v;
+  const double *kc, *vc;
+  const float* gates;
+  const int32_t* idx;
+  const double* dout;
+  int64_t h, nkb, chunk;
+  const int64_t* kblocks;
+  double *dkc_part, *dvc_part; /* [tasks][nkb][d] */
+  double *dk, *dv;             /* [nkb][block][d] */
+  int bad_index;
+} bwdk_ctx;
+
+/* the compressed branch over rows [task*chunk, ...): each row's P over all summaries and O_cmp,
+ * then dS against the listed summaries */
+static void bwdk_cmp_task(void* vctx, int64_t task) {
+  bwdk_ctx* c = (bwdk_ctx*)vctx;
+  const s3r_ref_params* p = c->p;
+  const int64_t nb = s3r_ref_num_blocks(p);
+  const int64_t H = p->H, d = p->d, HD = H * d, h = c->h;
+  double* dkc = c->dkc_part + task * c->nkb * d;
+  double* dvc = c->dvc_part + task * c->nkb * d;
+  double* pr = (double*)malloc(sizeof(double) * (size_t)nb);
+  double* qv = (double*)malloc(sizeof(double) * (size_t)d);
+  double* oc = (double*)malloc(sizeof(double) * (size_t)d);
+  double* doc = (double*)malloc(sizeof(double) * (size_t)d);
+  for (int64_t e = 0; e < c->nkb * d; ++e) dkc[e] = 0.0, dvc[e] = 0.0;
+  const int64_t r1 = (task + 1) * c->chunk < p->L ? (task + 1) * c->chunk : p->L;
+  for (int64_t r = task * c->chunk; r < r1; ++r) {
+    for (int64_t e = 0; e < d; ++e) qv[e] = bf16_value(c->q[r * HD + h * d + e]);
+    double m = -INFINITY;
+    for (int64_t j = 0; j < nb; ++j) {
+      double dot = 0.0;
+      for (int64_t e = 0; e < d; ++e) dot += qv[e] * c->kc[j * HD + h * d + e];
+      pr[j] = p->scale * dot;
+      if (pr[j] > m) m = pr[j];
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < nb; ++j) l += exp(pr[j] - m);
+    for (int64_t e = 0; e < d; ++e) oc[e] = 0.0;
+    for (int64_t j = 0; j < nb; ++j) {
+      pr[j] = exp(pr[j] - m) / l;
+      for (int64_t e = 0; e < d; ++e) oc[e] += pr[j] * c->vc[j * HD + h * d + e];
+    }
+    const double g0 = sigmoid((double)c->gates[(r * H + h) * 2 + 0]);
+    double dc = 0.0;
+    for (int64_t e = 0; e < d; ++e) {
+      doc[e] = g0 * c->dout[r * HD + h * d + e];
+      dc += doc[e] * oc[e];
+    }
+    for (int64_t a = 0; a < c->nkb; ++a) {
+      const int64_t j = c->kblocks[a];
+      double dp = 0.0;
+      for (int64_t e = 0; e < d; ++e) dp += doc[e] * c->vc[j * HD + h * d + e];
+      const double dsj = pr[j] * (dp - dc);
+      for (int64_t e = 0; e < d; ++e) {
+        dkc[a * d + e] += p->scale * dsj * qv[e];
+        dvc[a * d + e] += pr[j] * doc[e];
+      }
+    }
+  }
+  free(pr), free(qv), free(oc), free(doc);
+}
+
+/* the selection branch for listed block number a: every query block whose list holds it */
+static void bwdk_sel_task(void* vctx, int64_t a) {
+  bwdk_ctx* c = (bwdk_ctx*)vctx;
+  const s3r_ref_params* p = c->p;
+  const int64_t nb = s3r_ref_num_blocks(p), nqb = ceil_div(p->L, p->qblock);
+  const int64_t H = p->H, d = p->d, HD = H * d, h = c->h, jt = c->kblocks[a];
+  const int32_t n_list = p->forced + p->topk;
+  char* chosen = (char*)malloc((size_t)nb);
+  int64_t* tokens = (int64_t*)malloc(sizeof(int64_t) * (size_t)n_list * (size_t)p->block);
+  int64_t* mine = (int64_t*)malloc(sizeof(int64_t) * (size_t)p->block);
+  const int64_t n_mine = s3r_ref_block_tokens(p, jt, mine);
+  double* ss = (double*)malloc(sizeof(double) * (size_t)n_list * (size_t)p->block);
+  double* qv = (double*)malloc(sizeof(double) * (size_t)d);
+  double* os = (double*)malloc(sizeof(double) * (size_t)d);
+  double* dos = (double*)malloc(sizeof(double) * (size_t)d);
+  double* dk = c->dk + a * p->block * d;
+  double* dv = c->dv + a * p->block * d;
+  for (int64_t i = 0; i < nqb; ++i) {
+    const int32_t* sel = c->idx + (h * nqb + i) * n_list;
+    int holds = 0;
+    for (int32_t s = 0; s < n_list; ++s) holds |= sel[s] == jt;
+    if (!holds) continue;
+    int64_t nt = 0;
+    for (int64_t j = 0; j < nb; ++j) chosen[j] = 0;
+    for (int32_t s = 0; s < n_list; ++s) {
+      const int64_t j = sel[s];
+      if (j < 0 || j >= nb) {
+        c->bad_index = 1;
+        continue;
+      }
+      if (chosen[j]) continue;
+      chosen[j] = 1;
+      nt += s3r_ref_block_tokens(p, j, tokens + nt);
+    }
+    const int64_t r0 = i * p->qblock, r1 = r0 + p->qblock < p->L ? r0 + p->qblock : p->L;
+    for (int64_t r = r0; r < r1; ++r) {
+      for (int64_t e = 0; e < d; ++e) qv[e] = bf16_value(c->q[r * HD + h * d + e]);
+      double ms = -INFINITY;
+      for (int64_t t = 0; t < nt; ++t) {
+        double dot = 0.0;
+        for (int64_t e = 0; e < d; ++e) dot += qv[e] * bf16_value(c->k[tokens[t] * HD + h * d + e]);
+        ss[t] = p->scale * dot;
+        if (ss[t] > ms) ms = ss[t];
+      }
+      double ls = 0.0;
+      for (int64_t t = 0; t < nt; ++t) ls += exp(ss[t] - ms);
+      for (int64_t e = 0; e < d; ++e) os[e] = 0.0;
+      for (int64_t t = 0; t < nt; ++t) {
+        ss[t] = exp(ss[t] - ms) / ls;
+        for (int64_t e = 0; e < d; ++e) os[e] += ss[t] * bf16_value(c->v[tokens[t] * HD + h * d + e]);
+      }
+      const double g1 = sigmoid((double)c->gates[(r * H + h) * 2 + 1]);
+      double ds = 0.0;
+      for (int64_t e = 0; e < d; ++e) {
+        dos[e] = g1 * c->dout[r * HD + h * d + e];
+        ds += dos[e] * os[e];
+      }
+      for (int64_t t = 0; t < nt; ++t) {
+        int64_t slot = -1;
+        for (int64_t u = 0; u < n_mine; ++u)
+          if (mine[u] == tokens[t]) slot = u;
+        if (slot < 0) continue;
+        double dp = 0.0;
+        for (int64_t e = 0; e < d; ++e) dp += dos[e] * bf16_value(c->v[tokens[t] * HD + h * d + e]);
+        const double dst = ss[t] * (dp - ds);
+        for (int64_t e = 0; e < d; ++e) {
+          dk[slot * d + e] += p->scale * dst * qv[e];
+          dv[slot * d + e] += ss[t] * dos[e];
+        }
+      }
+    }
+  }
+  free(chosen), free(tokens), free(mine), free(ss), free(qv), free(os), free(dos);
+}
+
+int s3r_ref_bwd_keys(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k,
+                     const uint16_t* v, const double* kc, const double* vc, const float* gates,
+                     const int32_t* idx, int32_t h, const int64_t* kblocks, int64_t nkb,
+                     const double* dout, double* dk, double* dv) {
+  if (check_params(p) || !q || !k || !v || !kc || !vc || !gates || !idx || !dout || !dk || !dv ||
+      !kblocks || nkb < 1 || h < 0 || h >= p->H || p->topk < 1 || p->forced < 0)
+    return -1;
+  const int64_t nb = s3r_ref_num_blocks(p), d = p->d;
+  for (int64_t a = 0; a < nkb; ++a)
+    if (kblocks[a] < 0 || kblocks[a] >= nb) return -1;
+  const int64_t chunk = 256, ntask = ceil_div(p->L, chunk);
+  bwdk_ctx c = {p, q, k, v, kc, vc, gates, idx, dout, h, nkb, chunk, kblocks, NULL, NULL, dk, dv,
+                0};
+  c.dkc_part = (double*)malloc(sizeof(double) * (size_t)(ntask * nkb * d));
+  c.dvc_part = (double*)malloc(sizeof(double) * (size_t)(ntask * nkb * d));
+  for (int64_t e = 0; e < nkb * p->block * d; ++e) dk[e] = 0.0, dv[e] = 0.0;
+  parallel_for(ntask, p->threads, bwdk_cmp_task, &c);
+  parallel_for(nkb, p->threads, bwdk_sel_task, &c);
+  /* pooling backward: each summary is the mean of its block's tokens */
+  int64_t* tokens = (int64_t*)malloc(sizeof(int64_t) * (size_t)p->block);
+  for (int64_t a = 0; a < nkb; ++a) {
+    const int64_t n = s3r_ref_block_tokens(p, kblocks[a], tokens);
+    for (int64_t e = 0; e < d; ++e) {
+      double sk = 0.0, sv = 0.0;
+      for (int64_t t = 0; t < ntask; ++t) {
+        sk += c.dkc_part[(t * nkb + a) * d + e];
+        sv += c.dvc_part[(t * nkb + a) * d + e];
+      }
+      for (int64_t u = 0; u < n; ++u) {
+        dk[(a * p->block + u) * d + e] += sk / (double)n;
+        dv[(a * p->block + u) * d + e] += sv / (double)n;
+      }
+    }
+  }
+  free(tokens), free(c.dkc_part), free(c.dvc_part);
   return c.bad_index ? -3 : 0;
 }
 

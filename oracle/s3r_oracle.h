@@ -116,6 +116,18 @@ int s3r_ref_bwd(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k, c
                 const int64_t* qblocks, int64_t nq, const double* dout, double* dq, double* dk,
                 double* dv, double* dgates);
 
+/* dk, dv of one head h for the tokens of nkb listed key blocks kblocks[], each in [0, nb): the
+ * same gradients as s3r_ref_bwd (selection lists idx [H, nqb, F + k] held fixed, pooled rounding
+ * passed straight through), computed from all L rows of q, gates [L, H, 2] and dout [L, H, d]
+ * without forming the other blocks' gradients. dk, dv are [nkb, block, d]: row u of listed block
+ * a is the u-th token of that block (ascending, as s3r_ref_block_tokens lists them); rows past
+ * the block's token count are zero. Returns 0, -1 on bad arguments, -3 if idx held an index
+ * outside [0, nb). */
+int s3r_ref_bwd_keys(const s3r_ref_params* p, const uint16_t* q, const uint16_t* k,
+                     const uint16_t* v, const double* kc, const double* vc, const float* gates,
+                     const int32_t* idx, int32_t h, const int64_t* kblocks, int64_t nkb,
+                     const double* dout, double* dk, double* dv);
+
 /* Gated aggregation over n rows: out = sigmoid(g[...,0]) * o_cmp + sigmoid(g[...,1]) * o_sel. */
 int s3r_ref_combine(int64_t n, int32_t H, int32_t d, const double* o_cmp, const double* o_sel,
                     const float* gates, double* out);

@@ -24,6 +24,7 @@ S3R_FLAG_DEBUG_CHECKS = 0x1
 S3R_FLAG_TEST_TIMEOUT = 0x2
 S3R_FLAG_SINGLE_KERNEL = 0x4
 S3R_FLAG_SAVE_FOR_BWD = 0x8
+S3R_FLAG_NVTX = 0x10
 S3R_MAX_BLOCKS = 49152
 S3R_STATIC_WORKSPACE_BYTES = 32 << 20
 STAGES = ("pool", "cmp", "topk", "sel_combine")  # S3R_STAGE_* order
@@ -39,6 +40,7 @@ EXPORTS = {
     "s3r_num_key_blocks": (ctypes.c_int64, [_P]),
     "s3r_read_device_status": (ctypes.c_int, [_P, _P, _P]),
     "s3r_workspace_status_word": (_P, [_P]),
+    "s3r_last_device_error": (ctypes.c_int, [_P, _P]),
     "s3r_compress_kv": (ctypes.c_int, [_P, _P, _P, _P, _P, _P]),
     "s3r_cmp_attn_and_score": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "s3r_topk_blocks": (ctypes.c_int, [_P, _P, _P, _P]),

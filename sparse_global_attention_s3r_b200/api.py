@@ -36,7 +36,8 @@ class Config:
     P = special + grid_h * grid_w tokens; key blocks are each view's special tokens, then
     win_h x (block / win_h) windows of its patch grid.
     save_for_backward: the forward keeps in its workspace what the backward needs, and a backward
-    call with the same config and workspace skips recomputing the forward."""
+    call with the same config and workspace skips recomputing the forward.
+    nvtx: the whole-path calls push one NVTX range per stage (s3r.pool, s3r.cmp, ...)."""
 
     L: int
     H: int
@@ -53,6 +54,7 @@ class Config:
     special: int = 0
     win_h: int = 0
     save_for_backward: bool = False
+    nvtx: bool = False  # one NVTX range per stage of the whole-path calls, for profilers
 
     @property
     def nsel(self) -> int:
@@ -74,7 +76,8 @@ class Config:
                            (_lib.S3R_FLAG_DEBUG_CHECKS if self.debug_checks else 0)
                            | (_lib.S3R_FLAG_TEST_TIMEOUT if self.test_timeout else 0)
                            | (_lib.S3R_FLAG_SINGLE_KERNEL if self.single_kernel else 0)
-                           | (_lib.S3R_FLAG_SAVE_FOR_BWD if self.save_for_backward else 0),
+                           | (_lib.S3R_FLAG_SAVE_FOR_BWD if self.save_for_backward else 0)
+                           | (_lib.S3R_FLAG_NVTX if self.nvtx else 0),
                            self.forced, self.grid_h, self.grid_w, self.special, self.win_h,
                            None if dev_status is None else dev_status.data_ptr(),
                            None if stage_events is None else ctypes.addressof(stage_events))
@@ -216,9 +219,12 @@ def sparse_attn_fwd(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tens
 
 def sparse_attn_fwd_static(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                            gates: torch.Tensor, out: Optional[torch.Tensor] = None,
-                           idx_out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                           idx_out: Optional[torch.Tensor] = None,
+                           dev_status: Optional[torch.Tensor] = None) -> torch.Tensor:
     """The whole path without a workspace argument: the library's built-in scratch array is used
-    (sizes up to S3R_STATIC_WORKSPACE_BYTES of workspace; see include/s3r.h)."""
+    (sizes up to S3R_STATIC_WORKSPACE_BYTES of workspace; see include/s3r.h). The entry point
+    reports device-side conditions only through a caller's status word: pass dev_status (one
+    int32 on the device, read it with read_device_status), or one is allocated here."""
     for n, t in (("q", q), ("k", k), ("v", v)):
         _need(t, n, _lhd(cfg), torch.bfloat16)
     _need(gates, "gates", (cfg.L, cfg.H, 2), torch.float32)
@@ -227,7 +233,9 @@ def sparse_attn_fwd_static(cfg: Config, q: torch.Tensor, k: torch.Tensor, v: tor
     _need(out, "out", _lhd(cfg), torch.bfloat16)
     if idx_out is not None:
         _need(idx_out, "idx_out", (cfg.H, cfg.nqb, cfg.nsel), torch.int32)
-    p = cfg.params()
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=q.device)
+    p = cfg.params(dev_status)
     _lib.call("s3r_sparse_attn_fwd_static", ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v),
               _ptr(gates), _ptr(out), _ptr(idx_out), _stream())
     return out

@@ -5,6 +5,8 @@
 #include <climits>
 #include <cmath>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.h"
 #include "s3r.h"
 
@@ -12,6 +14,13 @@ namespace s3r {
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+void stage_range_push(const Problem& p, const char* name) {
+  if (p.flags & S3R_FLAG_NVTX) nvtxRangePushA(name);
+}
+void stage_range_pop(const Problem& p) {
+  if (p.flags & S3R_FLAG_NVTX) nvtxRangePop();
+}
 
 size_t topk_smem_bytes(int64_t nb);
 
@@ -216,26 +225,40 @@ int fused_forward(const s3r_params* params, const uint16_t* q, const uint16_t* k
   };
   if (cudaMemsetAsync(status, 0, 4, stream) != cudaSuccess) return S3R_ERR_CUDA;
   if (mark(0) != cudaSuccess) return S3R_ERR_CUDA;
-  if ((st = launched(launch_pool_kv(p, k, v, kc, vc, kh, vh, stream))) != S3R_OK) return st;
-  if (mark(1) != cudaSuccess) return S3R_ERR_CUDA;
+  // one stage: NVTX range, launch, event
+  auto stage = [&](const char* name, int ev_after, auto&& launch) -> s3r_status {
+    stage_range_push(p, name);
+    const s3r_status r = launched(launch());
+    stage_range_pop(p);
+    if (r != S3R_OK) return r;
+    return mark(ev_after) == cudaSuccess ? S3R_OK : S3R_ERR_CUDA;
+  };
+  if ((st = stage("s3r.pool", 1, [&] { return launch_pool_kv(p, k, v, kc, vc, kh, vh, stream); })) !=
+      S3R_OK)
+    return st;
   const bool fused_topk = p.k <= kFusedTopkMax;
   if ((p.flags & S3R_FLAG_SINGLE_KERNEL) && fused_topk && hm && !save) {
-    st = launched(launch_fused_tc(p, q, kc, vc, kh, vh, gate_logits, out, idx_out, stream));
+    st = stage("s3r.fused", 2, [&] {
+      return launch_fused_tc(p, q, kc, vc, kh, vh, gate_logits, out, idx_out, stream);
+    });
     if (st != S3R_OK) return st;
-    for (int i = 2; i <= 4; ++i)
+    for (int i = 3; i <= 4; ++i)
       if (mark(i) != cudaSuccess) return S3R_ERR_CUDA;
     return S3R_OK;
   }
-  if ((st = launched(launch_cmp_attn_tc(p, q, kc, vc, lse_c, o_cmp, fused_topk ? nullptr : scores,
-                                        fused_topk ? idx : nullptr, stream))) != S3R_OK)
+  if ((st = stage("s3r.cmp", 2, [&] {
+         return launch_cmp_attn_tc(p, q, kc, vc, lse_c, o_cmp, fused_topk ? nullptr : scores,
+                                   fused_topk ? idx : nullptr, stream);
+       })) != S3R_OK)
     return st;
-  if (mark(2) != cudaSuccess) return S3R_ERR_CUDA;
-  if (!fused_topk && (st = launched(launch_topk(p, scores, idx, stream))) != S3R_OK) return st;
-  if (mark(3) != cudaSuccess) return S3R_ERR_CUDA;
-  st = launched(launch_sel_attn(p, q, hm ? kh : k, hm ? vh : v, hm, idx, o_sel, o_cmp, gate_logits,
-                                out, stream, lse_s));
-  if (st != S3R_OK) return st;
-  return mark(4) == cudaSuccess ? S3R_OK : S3R_ERR_CUDA;
+  if ((st = stage("s3r.topk", 3, [&] {
+         return fused_topk ? cudaSuccess : launch_topk(p, scores, idx, stream);
+       })) != S3R_OK)
+    return st;
+  return stage("s3r.sel_combine", 4, [&] {
+    return launch_sel_attn(p, q, hm ? kh : k, hm ? vh : v, hm, idx, o_sel, o_cmp, gate_logits, out,
+                           stream, lse_s);
+  });
 }
 
 }  // namespace s3r
@@ -280,6 +303,15 @@ s3r_status s3r_read_device_status(uint32_t* dev_status, s3r_stream stream, uint3
   if (cudaMemsetAsync(dev_status, 0, 4, stream) != cudaSuccess) return S3R_ERR_CUDA;
   *out = v;
   return (v & S3R_DEV_TIMEOUT) ? S3R_ERR_TIMEOUT : S3R_OK;
+}
+
+s3r_status s3r_last_device_error(void* flag_buf, s3r_stream stream) {
+  uint32_t bits = 0;
+  const s3r_status st = s3r_read_device_status(static_cast<uint32_t*>(flag_buf), stream, &bits);
+  if (st == S3R_ERR_INVALID_ARG || st == S3R_ERR_CUDA) return st;
+  if (bits & S3R_DEV_TIMEOUT) return S3R_ERR_TIMEOUT;
+  if (bits & S3R_DEV_BAD_INDEX) return S3R_ERR_INVALID_ARG;
+  return S3R_OK;
 }
 
 s3r_status s3r_compress_kv(const s3r_params* params, const s3r_bf16* k, const s3r_bf16* v,
@@ -371,6 +403,7 @@ s3r_status s3r_sparse_attn_bwd(const s3r_params* params, const s3r_bf16* q, cons
     return S3R_ERR_CUDA;
   // the forward again, keeping what the backward needs (unless the forward call saved it)
   if (!(p.flags & S3R_FLAG_SAVE_FOR_BWD)) {
+    stage_range_push(p, "s3r.bwd.recompute");
     if ((st = launched(launch_pool_kv(p, k, v, b16(w.kc), b16(w.vc), b16(w.kh), b16(w.vh),
                                       stream))) != S3R_OK)
       return st;
@@ -380,6 +413,7 @@ s3r_status s3r_sparse_attn_bwd(const s3r_params* params, const s3r_bf16* q, cons
     if ((st = launched(launch_sel_attn(p, q, b16(w.kh), b16(w.vh), true, idx, f32(w.o_sel),
                                        nullptr, nullptr, nullptr, stream, f32(w.lse_s)))) != S3R_OK)
       return st;
+    stage_range_pop(p);
   }
   if (ev && cudaEventRecord(static_cast<cudaEvent_t>(ev[1]), stream) != cudaSuccess)
     return S3R_ERR_CUDA;

@@ -253,6 +253,7 @@ struct __align__(8) Bars {
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full, s_empty, ds_full, ds_empty, o_full, drain;
+  uint64_t never;  // never signalled: waited on only under S3R_FLAG_TEST_TIMEOUT
 };
 constexpr uint32_t kOffMisc = kOffBars + sizeof(Bars);
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
@@ -268,6 +269,7 @@ struct BwdQArgs {
   float scale, scale_log2;
   uint32_t* status;
   uint64_t limit_ns;
+  uint32_t flags;
 };
 
 __device__ __forceinline__ int64_t list_block(const int32_t* list, int s, int n, int64_t nb,
@@ -319,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(&bars->ds_empty, 1);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->never, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -438,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float sl2 = a.scale_log2;
     const int32_t* list = glist[qb];
     bool ok = true;
+    if (a.flags & S3R_FLAG_TEST_TIMEOUT) ok = mbar_wait(&bars->never, 0, abort, lim);
     for (int t = 0; ok && t < nsteps; ++t) {
       if (!(ok = mbar_wait(&bars->s_full, t & 1, abort, lim))) break;
       tc_fence_after();
@@ -546,6 +550,7 @@ struct __align__(8) Bars {
   uint64_t kv_full;
   uint64_t st_full[kStages], st_empty[kStages];
   uint64_t s_full, p_full, mma_done, o_full, drain;
+  uint64_t never;  // never signalled: waited on only under S3R_FLAG_TEST_TIMEOUT
 };
 constexpr uint32_t kOffMisc = kOffBars + sizeof(Bars);
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
@@ -567,6 +572,7 @@ struct BwdKVArgs {
   float scale, scale_log2;
   uint32_t* status;
   uint64_t limit_ns;
+  uint32_t flags;
 };
 
 template <bool kSel>
@@ -626,6 +632,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(&bars->mma_done, 1);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->never, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -762,6 +769,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const bool diag = !kSel || half == grp;
     const float sl2 = a.scale_log2;
     bool ok = true;
+    if (a.flags & S3R_FLAG_TEST_TIMEOUT) ok = mbar_wait(&bars->never, 0, abort, lim);
     for (int t = 0; ok && t < nsteps; ++t) {
       const int stage = t % kStages;
       if (!(ok = mbar_wait(&bars->s_full, t & 1, abort, lim))) break;
@@ -902,8 +910,9 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& B, cudaStream_t st,
   };
   const int64_t kv_rows = p.nb * p.b;
   if (static_cast<int64_t>(p.H) * kv_rows > INT32_MAX) return cudaErrorInvalidValue;
-  const uint64_t lim = 2000000000ull;
+  const uint64_t lim = (p.flags & S3R_FLAG_TEST_TIMEOUT) ? 1000000ull : 2000000000ull;
   cudaError_t e;
+  stage_range_push(p, "s3r.bwd.prep");
   // D, gate gradients, statistics planes
   {
     const int64_t threads = w.Lp * p.H * 16;
@@ -939,7 +948,9 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& B, cudaStream_t st,
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  stage_range_pop(p);
   if ((e = mark(2)) != cudaSuccess) return e;
+  stage_range_push(p, "s3r.bwd.dq");
   // dq
   {
     CUtensorMap tq, to, tkc, tvc, tkh, tvh;
@@ -954,13 +965,15 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& B, cudaStream_t st,
     const int lb = p.b == 32 ? 5 : p.b == 64 ? 6 : 7;
     BwdQArgs a{B.idx, B.stats, B.dq, p.L, w.Lp, p.nb, p.nqb, kv_rows, p.geo, p.H, p.b, lb,
                p.nsel, static_cast<int>((p.nb + 63) / 64), static_cast<int>(p.nsel * p.b / 32),
-               p.scale, p.scale_log2, p.status, lim};
+               p.scale, p.scale_log2, p.status, lim, p.flags};
     dim3 grid(static_cast<unsigned>((p.L + 127) / 128), p.H);
     bwd_q_kernel<<<grid, kThreads, q_outer::kSmemBytes, st>>>(tq, to, tkc, tvc, tkh, tvh, a);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  stage_range_pop(p);
   if ((e = mark(3)) != cudaSuccess) return e;
+  stage_range_push(p, "s3r.bwd.dkv_cmp");
   // dKc, dVc, then the token dk, dv (with the pooled gradients spread over each block)
   {
     CUtensorMap tkc, tvc, tq, to;
@@ -972,13 +985,15 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& B, cudaStream_t st,
     if ((e = prepare(bwd_kv_kernel<false>, kv_outer::kSmemBytes)) != cudaSuccess) return e;
     BwdKVArgs a{B.stats, nullptr, nullptr, nullptr, nullptr, nullptr, B.dkc, B.dvc, p.L, w.Lp, p.nb,
                 p.nqb, kv_rows, w.per_head, 0, p.geo, p.H, p.b, 1, p.scale, p.scale_log2,
-                p.status, lim};
+                p.status, lim, p.flags};
     dim3 grid(static_cast<unsigned>((p.nb + 127) / 128), p.H);
     bwd_kv_kernel<false><<<grid, kThreads, kv_outer::kSmemBytes, st>>>(tkc, tvc, tq, to, a);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  stage_range_pop(p);
   if ((e = mark(4)) != cudaSuccess) return e;
+  stage_range_push(p, "s3r.bwd.dkv_sel");
   {
     CUtensorMap tkh, tvh, tq, to;
     if (!make_tmap_rows64(&tkh, B.kh, p.H * kv_rows, 64) ||
@@ -989,12 +1004,13 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& B, cudaStream_t st,
     if ((e = prepare(bwd_kv_kernel<true>, kv_outer::kSmemBytes)) != cudaSuccess) return e;
     BwdKVArgs a{B.stats, B.off, B.ent, B.order, B.dkc, B.dvc, B.dk, B.dv, p.L, w.Lp, p.nb,
                 p.nqb, kv_rows, w.per_head, w.G, p.geo, p.H, p.b, w.cpb, p.scale, p.scale_log2,
-                p.status, lim};
+                p.status, lim, p.flags};
     dim3 grid(static_cast<unsigned>((w.G * p.H + 1) / 2), 1);
     bwd_kv_kernel<true><<<grid, kThreads, kv_outer::kSmemBytes, st>>>(tkh, tvh, tq, to, a);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  stage_range_pop(p);
   return mark(5);
 }
 

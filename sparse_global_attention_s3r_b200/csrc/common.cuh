@@ -26,27 +26,30 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
-// 2^x for two values on the FMA pipe (no MUFU): Cody-Waite reduction x = n + f with n the nearest
-// integer (f in [-1/2, 1/2]), a degree-5 minimax polynomial for 2^f fitted for this library
-// (relative error 7.5e-8 in exact arithmetic, 2.3e-7 evaluated in fp32, the accuracy of
-// ex2.approx), and 2^n added to the exponent field. x is clamped below at -126 (2^-126 ~ 1e-38
-// stands in for anything smaller, including -inf).
+// 2^x for two values on the FMA pipe (no MUFU), for x < 128, at the accuracy of MUFU.EX2.
+// Round-to-nearest range reduction x = n + f, f in [-1/2, 1/2] (Cody-Waite with one constant):
+// adding 1.5 * 2^23 + 127 rounds x to an integer and leaves the biased exponent 127 + n in the low
+// bits of the sum. A degree-5 minimax polynomial fitted for this library approximates 2^f
+// (relative error 7.5e-8 in exact arithmetic, 2.1e-7 evaluated with fp32 FMAs). One multiply
+// scales it by 2^n, whose bit pattern is those low bits shifted into the exponent field. x is
+// clamped below at -127, where that pattern is +0: the result is +0 for x below about -126.5,
+// close to where MUFU.EX2 with flush-to-zero returns 0 (x < -126).
 __device__ __forceinline__ float2 exp2_poly5x2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound keeps round(x) in the low bits
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  constexpr float kMagic = 12583039.0f;  // 1.5 * 2^23 + 127
+  x.x = fmaxf(x.x, -127.f);
+  x.y = fmaxf(x.y, -127.f);
+  const float2 t = __fadd2_rn(x, make_float2(kMagic, kMagic));
+  const float2 n = __fadd2_rn(t, make_float2(-kMagic, -kMagic));
   const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-  float2 p = make_float2(1.327647199e-03f, 1.327647199e-03f);
-  p = __ffma2_rn(p, f, make_float2(9.675541334e-03f, 9.675541334e-03f));
+  float2 p = __ffma2_rn(make_float2(1.327647199e-03f, 1.327647199e-03f), f,
+                        make_float2(9.675541334e-03f, 9.675541334e-03f));
   p = __ffma2_rn(p, f, make_float2(5.550713273e-02f, 5.550713273e-02f));
   p = __ffma2_rn(p, f, make_float2(2.402211972e-01f, 2.402211972e-01f));
   p = __ffma2_rn(p, f, make_float2(6.931469671e-01f, 6.931469671e-01f));
   p = __ffma2_rn(p, f, make_float2(1.000000072e+00f, 1.000000072e+00f));
-  // the low mantissa bits of t hold n; shifted by 23 they land on the exponent field
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+  const float2 s = make_float2(__uint_as_float(__float_as_uint(t.x) << 23),
+                               __uint_as_float(__float_as_uint(t.y) << 23));
+  return __fmul2_rn(p, s);
 }
 
 // max(a, b, c) in one instruction (sm_100 three-input max)

@@ -84,6 +84,10 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& b, cudaStream_t st, v
 
 void count_launch();
 
+// NVTX ranges around the stages of the whole-path calls, when S3R_FLAG_NVTX is set.
+void stage_range_push(const Problem& p, const char* name);
+void stage_range_pop(const Problem& p);
+
 // Workspace bytes of the fused path (0 if params are invalid), and the fused path itself on a
 // caller-provided workspace (returns an s3r_status value).
 size_t fused_workspace_bytes(const s3r_params* params);

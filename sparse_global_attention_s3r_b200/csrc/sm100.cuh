@@ -45,17 +45,32 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
   return t;
 }
+// As mbar_test, but a thread whose phase has not completed is suspended in hardware until it
+// does, or for at most about `suspend_ns`, instead of returning at once. A waiting warp then
+// takes no issue slots from the warps that do the work.
+__device__ __forceinline__ bool mbar_test_suspend(uint64_t* bar, uint32_t parity,
+                                                  uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+// Longest suspension of one try_wait in mbar_wait: the abort flag and the time limit are checked
+// between suspensions, so this bounds how late a waiter notices either.
+constexpr uint32_t kSuspendNs = 20000;
 // Wait until the phase of `bar` with parity `parity` has completed. False on timeout / abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_test(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) return false;
-    }
+  for (;;) {
+    if (mbar_test_suspend(bar, parity, kSuspendNs)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 

@@ -48,6 +48,19 @@ extern "C" s3r_status s3r_sparse_attn_fwd_static(const s3r_params* params, const
     return static_cast<s3r_status>(
         s3r::fused_forward(params, q, k, v, gate_logits, out, idx_out, nullptr, 0, stream));
   if (need > S3R_STATIC_WORKSPACE_BYTES) return S3R_ERR_WORKSPACE;
+  // What a saving forward keeps for the backward would live in the shared array, which the
+  // caller cannot hand to s3r_sparse_attn_bwd and the next call overwrites.
+  if (params->flags & S3R_FLAG_SAVE_FOR_BWD) return S3R_ERR_UNSUPPORTED;
+  // The array's own status word is not visible to the caller, so device-side conditions (an
+  // expired bounded wait) must go to a word the caller can read.
+  if (!params->dev_status) return S3R_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return S3R_ERR_CUDA;
+  if (stream) {  // the array's address is the current device's: the stream must run there
+    int stream_dev = -1;
+    if (cudaStreamGetDevice(stream, &stream_dev) != cudaSuccess || stream_dev != dev)
+      return S3R_ERR_INVALID_ARG;
+  }
   void* ws = s3r::static_workspace_on_current_device();
   if (!ws) return S3R_ERR_CUDA;
   return static_cast<s3r_status>(s3r::fused_forward(params, q, k, v, gate_logits, out, idx_out,

@@ -3,6 +3,8 @@
 // Speed3R (gist.science summary, "Methodologie" §1 "Selectie-tak"): the selection branch attends
 // to the top-k blocks chosen by the compression branch's scores. Ties go to the lower block index.
 //
+// Two kernels. For k <= kWarpTopkMax (every default configuration), topk_warp_kernel streams each
+// row once through one warp (see there). Larger k use topk_kernel:
 // One CTA per score row [nb] (one query block of one head). Scores are probabilities summed over
 // rows, so they are non-negative and their fp32 bit patterns order like unsigned integers; the
 // 64-bit key (bits << 32 | ~index) orders by descending score, then ascending index, and is unique.
@@ -234,20 +236,160 @@ __global__ void __launch_bounds__(kThreads)
     out[e] = first + static_cast<int32_t>(~static_cast<uint32_t>(sort_buf[e] & 0xFFFFFFFFull));
 }
 
+// ------------------------------------------------------------------------------------------
+// Streaming path for k <= kWarpTopkMax: one warp per row, kRowsPerCta warps per CTA walking rows
+// with a grid stride, no block-wide barrier. The warp reads its row once with coalesced loads
+// (the next kUnroll per lane in flight while the current ones are examined) and keeps in shared
+// memory a buffer of candidate keys together with theta, the k-th largest key among those it has
+// dropped or kept so far: at least k elements have keys >= theta, so an element whose key is
+// below it cannot be in the top-k. A 32-bit compare of the score bits against the upper half of
+// theta rejects almost every element once theta has risen; the few that pass are appended by
+// ballot. When the buffer would overflow it is sorted (warp-synchronous bitonic sort, descending)
+// and cut to its first k keys, and theta becomes the k-th. At the end of the row the buffer is
+// sorted once more and its first k keys are the row's top-k, in descending order. The buffer
+// holds kCap >= 2k + 32 keys, so a cut frees room for at least k + 32 more.
+// ------------------------------------------------------------------------------------------
+constexpr int kRowsPerCta = 8;
+constexpr int kUnroll = 8;         // loads in flight per lane
+constexpr int kWarpTopkMax = 240;  // 2k + 32 <= 512
+
+// descending bitonic sort of buf[0, n) by one warp; n a power of two, 32 <= n
+__device__ __forceinline__ void warp_bitonic_desc(uint64_t* buf, int n, int lane) {
+  for (int lsize = 1; (1 << lsize) <= n; ++lsize) {
+    const int size = 1 << lsize;
+    for (int lst = lsize - 1; lst >= 0; --lst) {
+      const int stride = 1 << lst;
+      for (int i = lane; i < (n >> 1); i += 32) {  // pair i: e has bit lst clear
+        const int e = ((i >> lst) << (lst + 1)) | (i & (stride - 1)), partner = e + stride;
+        const bool desc = (e & size) == 0;
+        const uint64_t x = buf[e], y = buf[partner];
+        if ((x < y) == desc) {
+          buf[e] = y;
+          buf[partner] = x;
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// sort the warp's cnt candidates and keep the first min(k, cnt); returns the new count and sets
+// theta to the k-th key (0 while fewer than k candidates exist)
+__device__ __forceinline__ int warp_compact(uint64_t* buf, int cnt, int k, uint64_t& theta,
+                                            int lane) {
+  int n2 = 32;
+  while (n2 < cnt) n2 <<= 1;
+  for (int e = cnt + lane; e < n2; e += 32) buf[e] = 0ull;  // below every real key
+  __syncwarp();
+  warp_bitonic_desc(buf, n2, lane);
+  const int kept = cnt < k ? cnt : k;
+  theta = cnt >= k ? buf[k - 1] : 0ull;
+  __syncwarp();
+  return kept;
+}
+
+template <int kCap>
+__global__ void __launch_bounds__(kRowsPerCta * 32)
+    topk_warp_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, int row_len,
+                     int first, int k, int64_t rows) {
+  extern __shared__ uint64_t warp_keys[];  // [kRowsPerCta][kCap]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t* buf = warp_keys + warp * kCap;
+  const int n = row_len - first;  // blocks first .. row_len-1 compete
+  const uint32_t below = (1u << lane) - 1u;
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + warp; row < rows;
+       row += static_cast<int64_t>(gridDim.x) * kRowsPerCta) {
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(scores + row * row_len + first);
+    int32_t* out = idx + row * (first + k);
+    for (int f = lane; f < first; f += 32) out[f] = f;
+    out += first;
+    uint64_t theta = 0ull;
+    int cnt = 0;
+    uint32_t x[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int j = u * 32 + lane;
+      x[u] = j < n ? __ldg(src + j) : 0u;
+    }
+    for (int base = 0; base < n; base += 32 * kUnroll) {
+      uint32_t nx[kUnroll];  // the next batch, in flight while this one is examined
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base + 32 * kUnroll + u * 32 + lane;
+        nx[u] = j < n ? __ldg(src + j) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j = base + u * 32 + lane;
+        // keys with score bits below theta's upper half are below theta
+        bool pass = j < n && x[u] >= static_cast<uint32_t>(theta >> 32);
+        if (!__any_sync(0xffffffffu, pass)) continue;
+        const uint64_t key = (static_cast<uint64_t>(x[u]) << 32) |
+                             static_cast<uint32_t>(~static_cast<uint32_t>(j));
+        pass = pass && key > theta;
+        uint32_t m = __ballot_sync(0xffffffffu, pass);
+        if (cnt + __popc(m) > kCap) {
+          cnt = warp_compact(buf, cnt, k, theta, lane);
+          pass = pass && key > theta;
+          m = __ballot_sync(0xffffffffu, pass);
+        }
+        if (pass) buf[cnt + __popc(m & below)] = key;
+        cnt += __popc(m);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) x[u] = nx[u];
+    }
+    __syncwarp();
+    cnt = warp_compact(buf, cnt, k, theta, lane);
+    for (int e = lane; e < k; e += 32)
+      out[e] = first + static_cast<int32_t>(~static_cast<uint32_t>(buf[e] & 0xFFFFFFFFull));
+    __syncwarp();  // the buffer is reused by the warp's next row
+  }
+}
+
+template <int kCap>
+cudaError_t launch_warp_topk(const Problem& p, const float* scores, int32_t* idx, int64_t rows,
+                             cudaStream_t st) {
+  constexpr int smem = kRowsPerCta * kCap * 8;
+  cudaError_t e = cudaFuncSetAttribute(topk_warp_kernel<kCap>,
+                                       cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148, per_sm = 1;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_warp_kernel<kCap>,
+                                                         kRowsPerCta * 32, smem)) != cudaSuccess)
+    return e;
+  const int64_t need = (rows + kRowsPerCta - 1) / kRowsPerCta;
+  const int64_t fill = static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1);
+  const unsigned grid = static_cast<unsigned>(need < fill ? need : fill);
+  topk_warp_kernel<kCap><<<grid, kRowsPerCta * 32, smem, st>>>(
+      scores, idx, static_cast<int>(p.nb), p.F, p.k, rows);
+  count_launch();
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 static_assert(kWarps * 256 * 4 >= kSortMax * 8, "sort buffer must fit in the histogram space");
+static_assert(2 * kWarpTopkMax + 32 <= 512, "the largest buffer holds 2k + 32 keys");
 
 size_t topk_smem_bytes(int64_t nb) {
   return static_cast<size_t>(kWarps) * 256 * 4 + static_cast<size_t>(nb) * 4;
 }
 
 cudaError_t launch_topk(const Problem& p, const float* scores, int32_t* idx, cudaStream_t st) {
+  const int64_t rows = static_cast<int64_t>(p.H) * p.nqb;
+  if (p.k <= kWarpTopkMax) {
+    if (2 * p.k + 32 <= 128) return launch_warp_topk<128>(p, scores, idx, rows, st);
+    if (2 * p.k + 32 <= 256) return launch_warp_topk<256>(p, scores, idx, rows, st);
+    return launch_warp_topk<512>(p, scores, idx, rows, st);
+  }
   const size_t smem = topk_smem_bytes(p.nb);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int64_t rows = static_cast<int64_t>(p.H) * p.nqb;
   topk_kernel<<<static_cast<unsigned>(rows), kThreads, smem, st>>>(scores, idx,
                                                                    static_cast<int>(p.nb), p.F, p.k);
   count_launch();

@@ -24,7 +24,7 @@ def declared_functions():
 def test_library_exports_every_declared_function():
     lib = _lib.load()
     names = declared_functions()
-    assert len(names) == 16, names
+    assert len(names) == 17, names
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_lib.EXPORTS)
@@ -211,6 +211,23 @@ def test_static_entry_point_rejects_oversized_and_bad_sizes_before_any_launch():
     bad = _params(d=128)
     assert lib.s3r_sparse_attn_fwd_static(ctypes.byref(bad), A16, A16, A16, A16, A16, None,
                                           None) == _lib.S3R_ERR_UNSUPPORTED
+
+
+def test_static_entry_point_needs_a_status_word_and_rejects_save_for_backward():
+    lib = _lib.load()
+    # no status word: the array's own word is invisible to the caller, so a timeout would be lost
+    assert lib.s3r_sparse_attn_fwd_static(ctypes.byref(_params()), A16, A16, A16, A16, A16, None,
+                                          None) == _lib.S3R_ERR_INVALID_ARG
+    # what a saving forward keeps would live in the shared array, out of the backward's reach
+    save = _params(flags=_lib.S3R_FLAG_SAVE_FOR_BWD, dev_status=A16.value)
+    assert lib.s3r_sparse_attn_fwd_static(ctypes.byref(save), A16, A16, A16, A16, A16, None,
+                                          None) == _lib.S3R_ERR_UNSUPPORTED
+
+
+def test_last_device_error_rejects_bad_flag_words():
+    lib = _lib.load()
+    assert lib.s3r_last_device_error(None, None) == _lib.S3R_ERR_INVALID_ARG
+    assert lib.s3r_last_device_error(ctypes.c_void_p((1 << 20) + 2), None) == _lib.S3R_ERR_INVALID_ARG
 
 
 def test_num_key_blocks_of_the_geometries():

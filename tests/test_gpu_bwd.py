@@ -182,3 +182,36 @@ def test_bwd_status_word_stays_clear(dev):
     api.sparse_attn_bwd(cfg, d["q"], d["k"], d["v"], d["gates"], idx,
                         _dout(L, H, 57).to(dev), dev_status=word)
     assert api.read_device_status(word) == 0
+
+
+def test_bwd_bounded_wait_timeout_is_reported_and_the_context_survives(dev):
+    """S3R_FLAG_TEST_TIMEOUT makes the backward's tensor-core kernels (dq, dKc/dVc, dk/dv) wait
+    on a barrier nothing signals, with a 1 ms limit. After a saving forward the backward runs only
+    those kernels, so the status word must carry S3R_DEV_TIMEOUT from them; the next backward on
+    the same workspace must then be correct again."""
+    import dataclasses
+
+    from sparse_global_attention_s3r_b200 import _lib
+
+    L, H, b, k, F, seed = CASES["ragged_b32_odd_k"]
+    x = synth.make_inputs(L, H, 64, b, seed)
+    save = api.Config(L=L, H=H, block=b, topk=k, forced=F, save_for_backward=True)
+    d = {n: getattr(x, n).to(dev) for n in ("q", "k", "v", "gates")}
+    ws = torch.empty(api.bwd_workspace_bytes(save), dtype=torch.uint8, device=dev)
+    idx = torch.empty((H, save.nqb, save.nsel), dtype=torch.int32, device=dev)
+    api.sparse_attn_fwd(save, d["q"], d["k"], d["v"], d["gates"], workspace=ws, idx_out=idx)
+    dout = _dout(L, H, seed).to(dev)
+    word = torch.zeros(1, dtype=torch.int32, device=dev)
+    timed_out = dataclasses.replace(save, test_timeout=True)
+    api.sparse_attn_bwd(timed_out, d["q"], d["k"], d["v"], d["gates"], idx, dout, workspace=ws,
+                        dev_status=word)
+    assert api.read_device_status(word) & _lib.S3R_DEV_TIMEOUT
+    grads = api.sparse_attn_bwd(save, d["q"], d["k"], d["v"], d["gates"], idx, dout,
+                                workspace=ws, dev_status=word)
+    assert api.read_device_status(word) == 0
+    bits = [O.bf16_bits(t) for t in (x.q, x.k, x.v)]
+    ref = O.backward(O.Problem(L, H, 64, b, k, forced=F), *bits, x.gates.numpy(),
+                     idx.cpu().numpy(), dout.cpu().double().numpy())
+    for n, got, want in zip(("dq", "dk", "dv", "dgates"), grads,
+                            (ref.dq, ref.dk, ref.dv, ref.dgates)):
+        _check(n, got, want)

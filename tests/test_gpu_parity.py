@@ -82,6 +82,30 @@ def test_topk_blocks_bit_exact(dev, name):
         np.testing.assert_array_equal(got, want)
 
 
+@pytest.mark.parametrize("k,forced", [(1, 0), (33, 0), (40, 5), (256, 0), (257, 3)])
+def test_topk_adversarial_orders_bit_exact(dev, k, forced):
+    """Score rows built against the streaming top-k: ascending scores (every element beats the
+    running k-th key, so the candidate buffer overflows and is cut again and again), descending,
+    all equal (the lowest indices win), a few distinct values repeated, and random. k = 257 takes
+    the block-wide radix-select kernel. Bit-exact against the oracle's top-k on the same fp32
+    values."""
+    g = torch.Generator().manual_seed(100 + k)
+    nb = 3001
+    cfg = api.Config(L=nb * 32, H=1, block=32, topk=k, forced=forced)
+    rows = torch.stack([
+        torch.linspace(0.0, 1.0, nb),
+        torch.linspace(1.0, 0.0, nb),
+        torch.full((nb,), 0.25),
+        torch.randint(0, 4, (nb,), generator=g).float() / 4,
+        torch.rand(nb, generator=g),
+    ])
+    full = torch.zeros((1, cfg.nqb, nb))
+    full[0, :rows.shape[0]] = rows
+    got = api.topk_blocks(cfg, full.to(dev))[0, :rows.shape[0]].cpu().numpy()
+    want, _ = O.topk(rows.double().numpy(), k, forced)
+    np.testing.assert_array_equal(got, want)
+
+
 def test_topk_large_k_unsorted_and_max_blocks(dev):
     g = torch.Generator().manual_seed(9)
     # k > 2048: the set is exact, emitted in ascending index order

@@ -85,6 +85,14 @@ MUTANTS = {
         "const int64_t r = rm->first[i], o = rm->offset[i] + rr;"),
     "bwd_cmp_key_grad_misses_scale": (
         "dkc[j * d + e] += p->scale * dsj * qv[e];", "dkc[j * d + e] += dsj * qv[e];"),
+    "bwd_keys_pool_spread_without_divisor": (
+        "dk[(a * p->block + u) * d + e] += sk / (double)n;",
+        "dk[(a * p->block + u) * d + e] += sk;"),
+    "bwd_keys_sel_drops_softmax_centering": (
+        "const double dst = ss[t] * (dp - ds);", "const double dst = ss[t] * dp;"),
+    "bwd_keys_cmp_value_grad_ignores_gate": (
+        "dvc[a * d + e] += pr[j] * doc[e];",
+        "dvc[a * d + e] += pr[j] * c->dout[r * HD + h * d + e];"),
     "bwd_sel_dq_from_values": (
         "dqr[e] += p->scale * dsa * bf16_value(c->k[t * HD + h * d + e]);",
         "dqr[e] += p->scale * dsa * bf16_value(c->v[t * HD + h * d + e]);"),

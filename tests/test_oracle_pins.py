@@ -925,3 +925,31 @@ def test_bwd_random_configurations_equal_autograd():
                                    [gr.dq, gr.dk, gr.dv, gr.dgates], leaves):
             np.testing.assert_allclose(mine, ref.grad.numpy(), rtol=0, atol=1e-11,
                                        err_msg=f"trial {trial}: {name} {pb}")
+
+
+def test_bwd_keys_equal_autograd_rows_of_the_listed_blocks():
+    """s3r_ref_bwd_keys: dk and dv of one head for the tokens of a few key blocks (the first, the
+    ragged last, one in the middle) equal torch autograd of the torch restatement of the forward
+    on those tokens, on 1-D blocks, with forced blocks, and on 2-D windows with special tokens;
+    the rows past a block's token count are zero."""
+    for pb, seed in [(O.Problem(200, 2, 16, 32, 3), 401),
+                     (O.Problem(190, 2, 16, 16, 2, forced=2), 402),
+                     (O.Problem(2 * (3 + 6 * 10), 2, 16, 16, 3, forced=1, grid_h=6, grid_w=10,
+                                special=3, win_h=2), 403)]:
+        q, kk, v, g, dout = _bwd_inputs(pb, seed)
+        kc = O.pool(pb, kk, exact=True)
+        vc = O.pool(pb, v, exact=True)
+        fwd = O.sparse_attn(pb, q, kk, v, g, pooled=(kc, vc))
+        leaves = _leaves(q, kk, v, g)
+        out = _torch_path(pb, *leaves, fwd.idx)
+        (out * torch.from_numpy(dout)).sum().backward()
+        blocks = [0, pb.nb - 1, pb.nb // 2]
+        for h in range(pb.H):
+            dk, dv = O.backward_keys(pb, q, kk, v, g, fwd.idx, dout, h, blocks, kc=kc, vc=vc)
+            for a, j in enumerate(blocks):
+                t = pb.block_tokens(j)
+                np.testing.assert_allclose(dk[a, :t.size], leaves[1].grad.numpy()[t, h], rtol=0,
+                                           atol=1e-11, err_msg=f"{pb} head {h} block {j}")
+                np.testing.assert_allclose(dv[a, :t.size], leaves[2].grad.numpy()[t, h], rtol=0,
+                                           atol=1e-11, err_msg=f"{pb} head {h} block {j}")
+                assert not dk[a, t.size:].any() and not dv[a, t.size:].any()
