@@ -118,15 +118,17 @@ EX2_PER_CLK_SM = 16
 SM_COUNT = 148
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the kernel that bounds
-# the step, from one ncu capture of the default workload (python bench.py --steps 2 --warmup 3
-# --no-cpu-baseline), with the SHA-256 of the sources that kernel was built from: once any of them
-# changes, the figure no longer describes the kernel and the roofline reports null.
+# the step at 1000 views: one ncu capture of that kernel on the 100-view layer (python bench.py
+# --workload n100 --steps 1 --warmup 3 --no-backward --no-cpu-baseline --no-dense-context; 290.8
+# MB read + 514.0 MB written), scaled by the ratio of rows (10.0: its traffic, Q read and O_cmp
+# written, is proportional to L). With the SHA-256 of the sources that kernel was built from: once
+# any of them changes, the figure no longer describes the kernel and the roofline reports null.
 TRAFFIC = {
-    "cmp": {"workload": "n1000", "bytes": 3004162304 + 5629871104,
+    "cmp": {"workload": "n1000", "bytes": (290766080 + 514033920) * 10,
              "sources": ["sparse_global_attention_s3r_b200/csrc/cmp_attn_tc.cu",
                          "sparse_global_attention_s3r_b200/csrc/common.cuh",
                          "sparse_global_attention_s3r_b200/csrc/sm100.cuh"],
-             "sha256": "e9f86e53355f80f5358f0ad84a73e3af03ddfb748dd0fffdbb9ed91733994b67"},
+             "sha256": "671e42957c5721277805d187ef85fba85fd85c18963b466fa8e0b7c350dcdf95"},
 }
 
 

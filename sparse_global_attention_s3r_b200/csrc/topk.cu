@@ -250,7 +250,13 @@ __global__ void __launch_bounds__(kThreads)
 // holds kCap >= 2k + 32 keys, so a cut frees room for at least k + 32 more.
 // ------------------------------------------------------------------------------------------
 constexpr int kRowsPerCta = 8;
-constexpr int kUnroll = 8;         // loads in flight per lane
+#ifndef S3R_TOPK_UNROLL
+#define S3R_TOPK_UNROLL 8
+#endif
+#ifndef S3R_TOPK_MIN_CTAS
+#define S3R_TOPK_MIN_CTAS 4
+#endif
+constexpr int kUnroll = S3R_TOPK_UNROLL;  // loads per lane in flight beside the current ones
 constexpr int kWarpTopkMax = 240;  // 2k + 32 <= 512
 
 // descending bitonic sort of buf[0, n) by one warp; n a power of two, 32 <= n
@@ -289,7 +295,7 @@ __device__ __forceinline__ int warp_compact(uint64_t* buf, int cnt, int k, uint6
 }
 
 template <int kCap>
-__global__ void __launch_bounds__(kRowsPerCta * 32)
+__global__ void __launch_bounds__(kRowsPerCta * 32, S3R_TOPK_MIN_CTAS)
     topk_warp_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, int row_len,
                      int first, int k, int64_t rows) {
   extern __shared__ uint64_t warp_keys[];  // [kRowsPerCta][kCap]
