@@ -26,7 +26,7 @@ Other workloads:
 
 - n100, vggt32, tiny;
 - n1000_k40, n100_k40: top-k = 40, which writes the score matrix and runs the stand-alone top-k
-  kernel;
+  kernel; n1000_k40_h1 is one head of n1000_k40;
 - n1000_windows: 2-D key windows;
 - vggt32_ref, vggt32_ref_windows: the reference view kept;
 - pi3_sweep: 24 layers per (b, top-k) setting at 200 views.
@@ -68,6 +68,11 @@ WORKLOADS = {
     "n1000_k40": dict(desc="1000-view sequence, top-k=40 (score matrix + stand-alone top-k): "
                            "L=1,374,000, H=16, d=64, b=64, 1 layer",
                       L=1374000, H=16, block=64, topk=40, seed=3),
+    # one head of that layer: the same 21,470-block score rows, 1/16 of them (1.84 GB), a size
+    # at which the stand-alone top-k can be profiled launch by launch
+    "n1000_k40_h1": dict(desc="1000-view sequence, one head, top-k=40 (score matrix + "
+                              "stand-alone top-k): L=1,374,000, H=1, d=64, b=64, 1 layer",
+                         L=1374000, H=1, block=64, topk=40, seed=3),
     "n100": dict(desc="100-view layer: L=137,400, H=16, d=64, b=64, top-k=32",
                  L=137400, H=16, block=64, topk=32, seed=2),
     "n100_k40": dict(desc="100-view layer, top-k=40 (score matrix + stand-alone top-k): "

@@ -238,40 +238,52 @@ __global__ void __launch_bounds__(kThreads)
 
 // ------------------------------------------------------------------------------------------
 // Streaming path for k <= kWarpTopkMax: one warp per row, kRowsPerCta warps per CTA walking rows
-// with a grid stride, no block-wide barrier. The warp reads its row once with coalesced loads
-// (the next kUnroll per lane in flight while the current ones are examined) and keeps in shared
-// memory a buffer of candidate keys together with theta, the k-th largest key among those it has
-// dropped or kept so far: at least k elements have keys >= theta, so an element whose key is
-// below it cannot be in the top-k. A 32-bit compare of the score bits against the upper half of
-// theta rejects almost every element once theta has risen; the few that pass are appended by
-// ballot. When the buffer would overflow it is sorted (warp-synchronous bitonic sort, descending)
-// and cut to its first k keys, and theta becomes the k-th. At the end of the row the buffer is
-// sorted once more and its first k keys are the row's top-k, in descending order. The buffer
-// holds kCap >= 2k + 32 keys, so a cut frees room for at least k + 32 more.
+// with a grid stride, no block-wide barrier. The warp reads its row once with 16-byte loads
+// (kVec per lane of the next batch in flight while the current batch is examined) and keeps, in
+// its slice of shared memory:
+//   top[0, K2)   the K2 (power of two >= k) largest keys seen so far, sorted descending, zero-filled
+//                while fewer than K2 keys have been seen (zero is below every real key)
+//   cand[0, C)   keys appended since top was last brought up to date, unsorted
+// theta = top[k-1] is the k-th largest key among those seen (or zero): at least k elements reach
+// it, so an element whose key is below it cannot be in the top-k. A 32-bit compare of the score
+// bits against the upper half of theta rejects almost every element once theta has risen; the few
+// that pass are appended to cand by ballot. When cand would overflow, it is sorted descending and
+// merged into top: the element-wise maximum of top[i] and cand[K2-1-i] holds the K2 largest keys
+// of both as a bitonic sequence, which K2's half-cleaner stages sort (a warp-synchronous bitonic
+// network; every compare-exchange is unrolled at compile time). At the end of the row the last
+// candidates are merged the same way and top[0, k) is the row's top-k, in descending order.
 // ------------------------------------------------------------------------------------------
 constexpr int kRowsPerCta = 8;
-#ifndef S3R_TOPK_UNROLL
-#define S3R_TOPK_UNROLL 8
+#ifndef S3R_TOPK_VEC
+#define S3R_TOPK_VEC 2
 #endif
 #ifndef S3R_TOPK_MIN_CTAS
 #define S3R_TOPK_MIN_CTAS 4
 #endif
-constexpr int kUnroll = S3R_TOPK_UNROLL;  // loads per lane in flight beside the current ones
-constexpr int kWarpTopkMax = 240;  // 2k + 32 <= 512
+constexpr int kVec = S3R_TOPK_VEC;  // 16-byte loads per lane in flight beside the current ones
+constexpr int kWarpTopkMax = 256;   // K2 <= 256
 
-// descending bitonic sort of buf[0, n) by one warp; n a power of two, 32 <= n
-__device__ __forceinline__ void warp_bitonic_desc(uint64_t* buf, int n, int lane) {
-  for (int lsize = 1; (1 << lsize) <= n; ++lsize) {
-    const int size = 1 << lsize;
-    for (int lst = lsize - 1; lst >= 0; --lst) {
-      const int stride = 1 << lst;
-      for (int i = lane; i < (n >> 1); i += 32) {  // pair i: e has bit lst clear
-        const int e = ((i >> lst) << (lst + 1)) | (i & (stride - 1)), partner = e + stride;
-        const bool desc = (e & size) == 0;
-        const uint64_t x = buf[e], y = buf[partner];
-        if ((x < y) == desc) {
-          buf[e] = y;
-          buf[partner] = x;
+__device__ __forceinline__ void cmp_exchange_desc(uint64_t* b, int e, int partner, bool desc) {
+  const uint64_t x = b[e], y = b[partner];
+  const uint64_t hi = x > y ? x : y, lo = x > y ? y : x;
+  b[e] = desc ? hi : lo;
+  b[partner] = desc ? lo : hi;
+}
+
+// descending bitonic sort of b[0, N) by one warp (N a power of two, 32 <= N)
+template <int N>
+__device__ __forceinline__ void warp_sort_desc(uint64_t* b, int lane) {
+  constexpr int kPairs = N / 2 > 32 ? N / 64 : 1;  // compare-exchanges per lane and stage
+#pragma unroll
+  for (int size = 2; size <= N; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int q = 0; q < kPairs; ++q) {
+        const int i = q * 32 + lane;  // pair i: element e has the stride bit clear
+        if (N / 2 >= 32 || i < N / 2) {
+          const int e = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));
+          cmp_exchange_desc(b, e, e + stride, (e & size) == 0);
         }
       }
       __syncwarp();
@@ -279,28 +291,68 @@ __device__ __forceinline__ void warp_bitonic_desc(uint64_t* buf, int n, int lane
   }
 }
 
-// sort the warp's cnt candidates and keep the first min(k, cnt); returns the new count and sets
-// theta to the k-th key (0 while fewer than k candidates exist)
-__device__ __forceinline__ int warp_compact(uint64_t* buf, int cnt, int k, uint64_t& theta,
-                                            int lane) {
-  int n2 = 32;
-  while (n2 < cnt) n2 <<= 1;
-  for (int e = cnt + lane; e < n2; e += 32) buf[e] = 0ull;  // below every real key
-  __syncwarp();
-  warp_bitonic_desc(buf, n2, lane);
-  const int kept = cnt < k ? cnt : k;
-  theta = cnt >= k ? buf[k - 1] : 0ull;
-  __syncwarp();
-  return kept;
+// sort the bitonic sequence b[0, N) descending: the half-cleaner stages of a bitonic network
+template <int N>
+__device__ __forceinline__ void warp_bitonic_clean_desc(uint64_t* b, int lane) {
+  constexpr int kPairs = N / 2 > 32 ? N / 64 : 1;
+#pragma unroll
+  for (int stride = N >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+    for (int q = 0; q < kPairs; ++q) {
+      const int i = q * 32 + lane;
+      if (N / 2 >= 32 || i < N / 2) {
+        const int e = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));
+        cmp_exchange_desc(b, e, e + stride, true);
+      }
+    }
+    __syncwarp();
+  }
 }
 
-template <int kCap>
+// merge cand[0, cnt) into top (see above); returns the new theta
+template <int K2, int C>
+__device__ __forceinline__ uint64_t warp_merge(uint64_t* top, uint64_t* cand, int cnt, int k,
+                                               int) {
+  // the lane index is re-read here so that the compiler does not keep the unrolled networks'
+  // addresses live in registers across the whole scan
+  int lane;
+  asm volatile("mov.u32 %0, %%laneid;\n" : "=r"(lane));
+  for (int e = cnt + lane; e < C; e += 32) cand[e] = 0ull;
+  __syncwarp();
+  warp_sort_desc<C>(cand, lane);
+  constexpr int kLo = K2 > C ? K2 - C : 0;  // below kLo, cand[K2-1-i] does not exist
+#pragma unroll
+  for (int i = kLo + lane; i < K2; i += 32) {
+    const uint64_t x = top[i], y = cand[K2 - 1 - i];
+    top[i] = x > y ? x : y;
+  }
+  __syncwarp();
+  warp_bitonic_clean_desc<K2>(top, lane);
+  return top[k - 1];
+}
+
+// The merge is inlined at each of its call sites, except for the largest list: there its
+// unrolled networks are long enough that one shared copy, reached by a call, runs faster.
+template <int K2, int C>
+__device__ __noinline__ uint64_t warp_merge_call(uint64_t* top, uint64_t* cand, int cnt, int k) {
+  return warp_merge<K2, C>(top, cand, cnt, k, 0);
+}
+template <int K2, int C>
+__device__ __forceinline__ uint64_t merge(uint64_t* top, uint64_t* cand, int cnt, int k, int lane) {
+  if constexpr (K2 >= 256)
+    return warp_merge_call<K2, C>(top, cand, cnt, k);
+  else
+    return warp_merge<K2, C>(top, cand, cnt, k, lane);
+}
+
+template <int K2, int C>
 __global__ void __launch_bounds__(kRowsPerCta * 32, S3R_TOPK_MIN_CTAS)
     topk_warp_kernel(const float* __restrict__ scores, int32_t* __restrict__ idx, int row_len,
                      int first, int k, int64_t rows) {
-  extern __shared__ uint64_t warp_keys[];  // [kRowsPerCta][kCap]
+  extern __shared__ uint64_t warp_keys[];  // [kRowsPerCta][K2 + C]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint64_t* buf = warp_keys + warp * kCap;
+  uint64_t* top = warp_keys + warp * (K2 + C);
+  uint64_t* cand = top + K2;
   const int n = row_len - first;  // blocks first .. row_len-1 compete
   const uint32_t below = (1u << lane) - 1u;
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerCta + warp; row < rows;
@@ -309,68 +361,123 @@ __global__ void __launch_bounds__(kRowsPerCta * 32, S3R_TOPK_MIN_CTAS)
     int32_t* out = idx + row * (first + k);
     for (int f = lane; f < first; f += 32) out[f] = f;
     out += first;
+#pragma unroll
+    for (int i = lane; i < K2; i += 32) top[i] = 0ull;
+    __syncwarp();
     uint64_t theta = 0ull;
     int cnt = 0;
-    uint32_t x[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int j = u * 32 + lane;
-      x[u] = j < n ? __ldg(src + j) : 0u;
-    }
-    for (int base = 0; base < n; base += 32 * kUnroll) {
-      uint32_t nx[kUnroll];  // the next batch, in flight while this one is examined
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int j = base + 32 * kUnroll + u * 32 + lane;
-        nx[u] = j < n ? __ldg(src + j) : 0u;
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int j = base + u * 32 + lane;
-        // keys with score bits below theta's upper half are below theta
-        bool pass = j < n && x[u] >= static_cast<uint32_t>(theta >> 32);
-        if (!__any_sync(0xffffffffu, pass)) continue;
-        const uint64_t key = (static_cast<uint64_t>(x[u]) << 32) |
-                             static_cast<uint32_t>(~static_cast<uint32_t>(j));
+    // offer one element per lane (block index j, valid or not) to cand
+    auto offer = [&](uint32_t x, int j, bool pass) {
+      const uint64_t key =
+          (static_cast<uint64_t>(x) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(j));
+      pass = pass && key > theta;
+      uint32_t m = __ballot_sync(0xffffffffu, pass);
+      if (cnt + __popc(m) > C) {
+        theta = merge<K2, C>(top, cand, cnt, k, lane);
+        cnt = 0;
         pass = pass && key > theta;
-        uint32_t m = __ballot_sync(0xffffffffu, pass);
-        if (cnt + __popc(m) > kCap) {
-          cnt = warp_compact(buf, cnt, k, theta, lane);
-          pass = pass && key > theta;
-          m = __ballot_sync(0xffffffffu, pass);
-        }
-        if (pass) buf[cnt + __popc(m & below)] = key;
-        cnt += __popc(m);
+        m = __ballot_sync(0xffffffffu, pass);
       }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) x[u] = nx[u];
+      if (pass) cand[cnt + __popc(m & below)] = key;
+      cnt += __popc(m);
+    };
+    // offer the four elements of one 16-byte load per lane (blocks j0 .. j0+3): four exact tests,
+    // a prefix count of the passing keys from three ballots (a lane passes at most four), and
+    // predicated appends. If they would overflow cand, they go in one element at a time instead,
+    // merging as needed.
+    auto offer4 = [&](const uint4 c, const int j0, const bool v) {
+      const uint32_t lo = ~static_cast<uint32_t>(j0);  // ~(j0 + e) = lo - e
+      const uint64_t k0 = static_cast<uint64_t>(c.x) << 32 | lo;
+      const uint64_t k1 = static_cast<uint64_t>(c.y) << 32 | (lo - 1u);
+      const uint64_t k2 = static_cast<uint64_t>(c.z) << 32 | (lo - 2u);
+      const uint64_t k3 = static_cast<uint64_t>(c.w) << 32 | (lo - 3u);
+      const bool p0 = v && k0 > theta, p1 = v && k1 > theta, p2 = v && k2 > theta,
+                 p3 = v && k3 > theta;
+      const int pc = p0 + p1 + p2 + p3;
+      const uint32_t b0 = __ballot_sync(0xffffffffu, pc & 1);
+      const uint32_t b1 = __ballot_sync(0xffffffffu, pc & 2);
+      const uint32_t b2 = __ballot_sync(0xffffffffu, pc & 4);
+      const int total = __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2);
+      if (cnt + total > C) {
+        uint4 r = c;
+        uint32_t pm = p0 | p1 << 1 | p2 << 2 | p3 << 3;
+#pragma unroll 1
+        for (int e = 0; e < 4; ++e) {  // one copy of the code for the four elements
+          offer(r.x, j0 + e, pm & 1u);
+          r = make_uint4(r.y, r.z, r.w, 0u);
+          pm >>= 1;
+        }
+        return;
+      }
+      int pos = cnt + __popc(b0 & below) + 2 * __popc(b1 & below) + 4 * __popc(b2 & below);
+      if (p0) cand[pos++] = k0;
+      if (p1) cand[pos++] = k1;
+      if (p2) cand[pos++] = k2;
+      if (p3) cand[pos] = k3;
+      cnt += total;
+    };
+    // elements before the first 16-byte boundary of the row, and after the last one
+    int head = static_cast<int>(((16u - (reinterpret_cast<uintptr_t>(src) & 15u)) & 15u) >> 2);
+    if (head > n) head = n;
+    const int nvec = (n - head) >> 2, tail0 = head + 4 * nvec;
+    {
+      const bool v = lane < head;
+      const uint32_t x = v ? __ldg(src + lane) : 0u;
+      if (__any_sync(0xffffffffu, v)) offer(x, lane, v);
     }
-    __syncwarp();
-    cnt = warp_compact(buf, cnt, k, theta, lane);
+    const uint4* vsrc = reinterpret_cast<const uint4*>(src + head);
+    uint4 x[kVec];
+#pragma unroll
+    for (int u = 0; u < kVec; ++u) {
+      const int vi = u * 32 + lane;
+      x[u] = vi < nvec ? __ldg(vsrc + vi) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int vb = 0; vb < nvec; vb += 32 * kVec) {
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const uint4 c = x[u];
+        {  // the same slot of the next batch goes in flight before this one is examined
+          const int vi = vb + 32 * kVec + u * 32 + lane;
+          x[u] = vi < nvec ? __ldg(vsrc + vi) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        const int vi = vb + u * 32 + lane;
+        const bool v = vi < nvec;
+        // keys with score bits below theta's upper half are below theta
+        const uint32_t th = static_cast<uint32_t>(theta >> 32);
+        const uint32_t mx = max(max(c.x, c.y), max(c.z, c.w));
+        if (__any_sync(0xffffffffu, v && mx >= th)) offer4(c, head + 4 * vi, v);
+      }
+    }
+    {
+      const bool v = tail0 + lane < n;
+      const uint32_t xt = v ? __ldg(src + tail0 + lane) : 0u;
+      if (__any_sync(0xffffffffu, v)) offer(xt, tail0 + lane, v);
+    }
+    merge<K2, C>(top, cand, cnt, k, lane);
     for (int e = lane; e < k; e += 32)
-      out[e] = first + static_cast<int32_t>(~static_cast<uint32_t>(buf[e] & 0xFFFFFFFFull));
-    __syncwarp();  // the buffer is reused by the warp's next row
+      out[e] = first + static_cast<int32_t>(~static_cast<uint32_t>(top[e] & 0xFFFFFFFFull));
+    __syncwarp();  // the buffers are reused by the warp's next row
   }
 }
 
-template <int kCap>
+template <int K2, int C>
 cudaError_t launch_warp_topk(const Problem& p, const float* scores, int32_t* idx, int64_t rows,
                              cudaStream_t st) {
-  constexpr int smem = kRowsPerCta * kCap * 8;
-  cudaError_t e = cudaFuncSetAttribute(topk_warp_kernel<kCap>,
+  constexpr int smem = kRowsPerCta * (K2 + C) * 8;
+  cudaError_t e = cudaFuncSetAttribute(topk_warp_kernel<K2, C>,
                                        cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148, per_sm = 1;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_warp_kernel<kCap>,
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_warp_kernel<K2, C>,
                                                          kRowsPerCta * 32, smem)) != cudaSuccess)
     return e;
   const int64_t need = (rows + kRowsPerCta - 1) / kRowsPerCta;
   const int64_t fill = static_cast<int64_t>(sms) * (per_sm > 0 ? per_sm : 1);
   const unsigned grid = static_cast<unsigned>(need < fill ? need : fill);
-  topk_warp_kernel<kCap><<<grid, kRowsPerCta * 32, smem, st>>>(
+  topk_warp_kernel<K2, C><<<grid, kRowsPerCta * 32, smem, st>>>(
       scores, idx, static_cast<int>(p.nb), p.F, p.k, rows);
   count_launch();
   return cudaGetLastError();
@@ -379,7 +486,6 @@ cudaError_t launch_warp_topk(const Problem& p, const float* scores, int32_t* idx
 }  // namespace
 
 static_assert(kWarps * 256 * 4 >= kSortMax * 8, "sort buffer must fit in the histogram space");
-static_assert(2 * kWarpTopkMax + 32 <= 512, "the largest buffer holds 2k + 32 keys");
 
 size_t topk_smem_bytes(int64_t nb) {
   return static_cast<size_t>(kWarps) * 256 * 4 + static_cast<size_t>(nb) * 4;
@@ -388,9 +494,10 @@ size_t topk_smem_bytes(int64_t nb) {
 cudaError_t launch_topk(const Problem& p, const float* scores, int32_t* idx, cudaStream_t st) {
   const int64_t rows = static_cast<int64_t>(p.H) * p.nqb;
   if (p.k <= kWarpTopkMax) {
-    if (2 * p.k + 32 <= 128) return launch_warp_topk<128>(p, scores, idx, rows, st);
-    if (2 * p.k + 32 <= 256) return launch_warp_topk<256>(p, scores, idx, rows, st);
-    return launch_warp_topk<512>(p, scores, idx, rows, st);
+    if (p.k <= 32) return launch_warp_topk<32, 64>(p, scores, idx, rows, st);
+    if (p.k <= 64) return launch_warp_topk<64, 64>(p, scores, idx, rows, st);
+    if (p.k <= 128) return launch_warp_topk<128, 64>(p, scores, idx, rows, st);
+    return launch_warp_topk<256, 128>(p, scores, idx, rows, st);
   }
   const size_t smem = topk_smem_bytes(p.nb);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

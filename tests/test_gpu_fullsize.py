@@ -21,6 +21,8 @@ FULL = {  # name: (L, H, b, k, seed, sampled query blocks[, 2-D geometry, forced
     "vggt32": (43968, 16, 64, 16, 1, 64),
     "n100": (137400, 16, 64, 32, 2, 48),
     "n1000": (1374000, 16, 64, 32, 3, 64),
+    # top-k = 40: the score matrix is written and the stand-alone top-k selects
+    "n1000_k40": (1374000, 16, 64, 40, 6, 32),
     "pi3_b32": (274800, 16, 32, 32, 4000, 24),
     "pi3_b64": (274800, 16, 64, 16, 4001, 24),
     "pi3_b128": (274800, 16, 128, 8, 4002, 24),
