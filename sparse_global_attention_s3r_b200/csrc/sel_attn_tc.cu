@@ -7,19 +7,24 @@
 //
 // One CTA = two 64-row query blocks of one head (a 128-row tile, one TMEM lane per row). The k
 // selected blocks of a query block form a list of k*b tokens, walked in steps of 64 tokens. Each
-// step gathers, with 2-D TMA boxes straight from K/V [L, H, 64], the next 64 tokens of each of the
-// two query blocks into one 128-token K tile and V tile (rows past L read as zeros). Then
+// step gathers, with 2-D TMA boxes straight from K/V [L, H, 64] (or their head-major copies), the
+// next 64 tokens of each of the two query blocks into one 128-token K tile and V tile (rows past L
+// read as zeros). K and V tiles have rings and barriers of their own: a K tile is released as soon
+// as its Q K^T has completed, and the K gathers run kKLead steps ahead of the V gathers, so the
+// next steps' keys are in flight while P V still holds the V ring. Then
 //   S = Q K^T       tcgen05.mma, M=128 x N=128: rows of query block 0 only use columns 0-63 (its
 //                   tokens), rows of block 1 columns 64-127
 //   O += P V        tcgen05.mma with bf16 P as the TMEM operand; the P columns of the other
 //                   block's tokens are zero (written once), so the product stays block-diagonal
 // The MMA work is twice what a 64-row tile would need, in exchange for the 128-lane layouts.
-// Softmax: one warp per TMEM lane quadrant (32 rows of one query block), 4 rows x 16 columns per
-// thread with the 16x256b load shape; the reference max of a row is fixed at the first step and
+// Softmax: two warps per TMEM lane quadrant, each holding 16 rows of one query block, 2 rows x 16
+// columns per thread with the 16x256b load shape (a row lies in one warp, so its maximum and sum
+// need only the quad's shuffles); the reference max of a row is fixed at the first step and
 // moves (with O and the row sum rescaled in TMEM once the previous product has completed) only if
 // a logit exceeds it by 32 in base-2 units, so the bf16 P stays below 2^32.
-// Roles (224 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-5 softmax
-// (warp w holds lane quadrant w%4), warp 6 idle. TMEM: S (128 cols) | O (64) | P (64 = 128 keys).
+// Roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-9 softmax
+// (warp w holds rows 16*((w-2)/4) .. +15 of lane quadrant w%4). TMEM: S (128 cols) | O (64) |
+// P (64 = 128 keys).
 // Every wait is bounded in time and watches a CTA abort flag (S3R_DEV_TIMEOUT on expiry).
 #include <climits>
 
@@ -36,9 +41,18 @@ using namespace sm100;
 
 constexpr int kBM = 128;                 // rows: two 64-row query blocks
 constexpr int kStep = 64;                // tokens per query block per step
-constexpr int kStages = 2;               // K/V tile ring depth
-constexpr int kThreads = 224;            // 7 warps
-constexpr int kSoftmaxThreads = 128;
+#ifndef S3R_SEL_K_STAGES
+#define S3R_SEL_K_STAGES 3
+#endif
+#ifndef S3R_SEL_K_LEAD
+#define S3R_SEL_K_LEAD 2
+#endif
+constexpr int kStagesK = S3R_SEL_K_STAGES;  // K tile ring depth
+constexpr int kStagesV = 2;                 // V tile ring depth
+constexpr int kKLead = S3R_SEL_K_LEAD;      // steps by which the K gathers run ahead of V's
+static_assert(kKLead >= 0 && kKLead < kStagesK + 2, "a lead the rings cannot hold deadlocks");
+constexpr int kThreads = 320;            // 10 warps
+constexpr int kSoftmaxThreads = 256;
 constexpr uint32_t kQBytes = kBM * 128;  // 16 KB
 constexpr uint32_t kTileBytes = 2 * kStep * 128;  // 128 tokens x 128 B = 16 KB (K or V)
 constexpr uint32_t kColS = 0, kColO = 128, kColP = 192, kTmemCols = 256;
@@ -49,7 +63,8 @@ constexpr int kIdxCache = 256;    // selection lists up to this length are stage
 
 struct __align__(8) Bars {
   uint64_t q_full;
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t k_full[kStagesK], k_empty[kStagesK];  // K tile of a step: freed once Q K^T completed
+  uint64_t v_full[kStagesV], v_empty[kStagesV];  // V tile: freed once P V completed
   uint64_t s_full, s_empty;
   uint64_t p_full, p_empty;
   uint64_t o_full, drain;
@@ -57,8 +72,9 @@ struct __align__(8) Bars {
 };
 
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKV = kQBytes;  // stage s: K tile at +2s*16K, V tile at +16K
-constexpr uint32_t kOffIdx = kOffKV + kStages * 2 * kTileBytes;  // [2][kIdxCache] int32
+constexpr uint32_t kOffK = kQBytes;                          // K tile of stage s at +s*16K
+constexpr uint32_t kOffV = kOffK + kStagesK * kTileBytes;    // V tile of stage s at +s*16K
+constexpr uint32_t kOffIdx = kOffV + kStagesV * kTileBytes;  // [2][kIdxCache] int32
 constexpr uint32_t kOffBars = kOffIdx + 2 * kIdxCache * 4;
 constexpr uint32_t kOffMisc = kOffBars + sizeof(Bars);
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
@@ -103,9 +119,8 @@ __device__ __forceinline__ int64_t sel_block(const int32_t* list, int s, int k, 
   return ok ? j : 0;
 }
 
-// 128 registers: two CTAs of 7 warps per SM (at most 4 warps x 4096 registers per SM
-// sub-partition, whose register file holds 16K)
-__global__ void __maxnreg__(128)
+// two CTAs of 10 warps per SM: at most 96 registers a thread
+__global__ void __launch_bounds__(kThreads, 2)
     sel_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const SelArgs a) {
@@ -137,9 +152,13 @@ __global__ void __maxnreg__(128)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+    for (int s = 0; s < kStagesK; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kStagesV; ++s) {
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_empty, kSoftmaxThreads / 32);
@@ -166,18 +185,12 @@ __global__ void __maxnreg__(128)
     // ------------------------------------------------------------------ TMA producer (gather)
     if (lane == 0) {
       bool ok = true;
-      int issued = 0;
+      int issued_k = 0, issued_v = 0;
       mbar_arrive_expect_tx(&bars->q_full, kQBytes);
       tma_load_2d(sbase + kOffQ, &tmQ, h * 64, static_cast<int32_t>(q0), &bars->q_full);
       const int box = a.box;
-      for (int t = 0; t < ns; ++t) {
-        const int stage = t % kStages;
-        if (!mbar_wait(&bars->kv_empty[stage], ((t / kStages) & 1) ^ 1, abort, lim)) {
-          ok = false;
-          break;
-        }
-        const uint32_t sk = sbase + kOffKV + stage * 2 * kTileBytes;
-        mbar_arrive_expect_tx(&bars->kv_full[stage], 2 * kTileBytes);
+      // the step's boxes of K (v = 0) or V (v = 1) into the stage's tile
+      auto gather = [&](int t, int v, uint32_t dst, uint64_t* bar) {
         for (int qb = 0; qb < 2; ++qb) {
           const int32_t* list = list_of[qb];
           for (int part = 0; part < kStep / box; ++part) {
@@ -196,18 +209,43 @@ __global__ void __maxnreg__(128)
             }
             const uint32_t row_off = (qb * kStep + part * box) * 128;
             const int32_t x = h * a.kv_xh, y = static_cast<int32_t>(h * a.kv_yh + row);
-            tma_load_2d(sk + row_off, &tmK, x, y, &bars->kv_full[stage]);
-            tma_load_2d(sk + kTileBytes + row_off, &tmV, x, y, &bars->kv_full[stage]);
+            tma_load_2d(dst + row_off, v ? &tmV : &tmK, x, y, bar);
           }
         }
-        issued = t + 1;
+      };
+      // K of step u, then V of step u - kKLead: the K tiles run ahead, since Q K^T needs them a
+      // whole softmax earlier than P V needs the V tiles
+      for (int u = 0; u < ns + kKLead; ++u) {
+        if (u < ns) {
+          const int sk = u % kStagesK;
+          if (!mbar_wait(&bars->k_empty[sk], ((u / kStagesK) & 1) ^ 1, abort, lim)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->k_full[sk], kTileBytes);
+          gather(u, 0, sbase + kOffK + sk * kTileBytes, &bars->k_full[sk]);
+          issued_k = u + 1;
+        }
+        const int t = u - kKLead;
+        if (t >= 0 && t < ns) {
+          const int sv = t % kStagesV;
+          if (!mbar_wait(&bars->v_empty[sv], ((t / kStagesV) & 1) ^ 1, abort, lim)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->v_full[sv], kTileBytes);
+          gather(t, 1, sbase + kOffV + sv * kTileBytes, &bars->v_full[sv]);
+          issued_v = t + 1;
+        }
       }
       if (!ok) {
         raise_abort(abort, a.status);
         int dummy = 0;
         mbar_wait(&bars->q_full, 0, &dummy, lim);
-        for (int t = issued - 1; t >= 0 && t >= issued - kStages; --t)
-          mbar_wait(&bars->kv_full[t % kStages], (t / kStages) & 1, &dummy, lim);
+        for (int t = issued_k - 1; t >= 0 && t >= issued_k - kStagesK; --t)
+          mbar_wait(&bars->k_full[t % kStagesK], (t / kStagesK) & 1, &dummy, lim);
+        for (int t = issued_v - 1; t >= 0 && t >= issued_v - kStagesV; --t)
+          mbar_wait(&bars->v_full[t % kStagesV], (t / kStagesV) & 1, &dummy, lim);
       }
     }
   } else if (warp == 1) {
@@ -217,27 +255,29 @@ __global__ void __maxnreg__(128)
       tc_fence_after();
       const uint64_t dq = desc_sw128(sbase + kOffQ);
       auto qk = [&](int t) -> bool {
-        const int stage = t % kStages;
-        if (!mbar_wait(&bars->kv_full[stage], (t / kStages) & 1, abort, lim)) return false;
+        const int stage = t % kStagesK;
+        if (!mbar_wait(&bars->k_full[stage], (t / kStagesK) & 1, abort, lim)) return false;
         if (!mbar_wait(&bars->s_empty, (t & 1) ^ 1, abort, lim)) return false;
         tc_fence_after();
-        const uint64_t dk = desc_sw128(sbase + kOffKV + stage * 2 * kTileBytes);
+        const uint64_t dk = desc_sw128(sbase + kOffK + stage * kTileBytes);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_ss(tbase + kColS, dq + 2 * ks, dk + 2 * ks, kIdescQK, ks > 0);
         tc_commit(&bars->s_full);
+        tc_commit(&bars->k_empty[stage]);
         return true;
       };
       auto pv = [&](int t) -> bool {
-        const int stage = t % kStages;
+        const int stage = t % kStagesV;
         if (!mbar_wait(&bars->p_full, t & 1, abort, lim)) return false;
+        if (!mbar_wait(&bars->v_full[stage], (t / kStagesV) & 1, abort, lim)) return false;
         tc_fence_after();
-        const uint64_t dv = desc_sw128(sbase + kOffKV + stage * 2 * kTileBytes + kTileBytes);
+        const uint64_t dv = desc_sw128(sbase + kOffV + stage * kTileBytes);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)  // 128 keys in steps of 16: 16 rows x 128 B = 2048 B
           mma_ts(tbase + kColO, tbase + kColP + ks * 8, dv + 128 * ks, kIdescPV,
                  (t > 0 || ks > 0) ? 1u : 0u);
-        tc_commit(&bars->kv_empty[stage]);
+        tc_commit(&bars->v_empty[stage]);
         tc_commit(&bars->p_empty);
         return true;
       };
@@ -255,48 +295,45 @@ __global__ void __maxnreg__(128)
         mbar_wait(&bars->drain, 0, &dummy, lim);
       }
     }
-  } else if (warp <= 5) {
+  } else {
     // ------------------------------------------------------------------ softmax warps
-    const int g = warp & 3;       // TMEM lane quadrant: rows 32g .. 32g+31
-    const int qb = g >> 1;        // which of the two query blocks these rows belong to
+    // warp w holds rows 16*sub .. 16*sub+15 of TMEM lane quadrant w%4 (sub = (w-2)/4), so that
+    // each row lies in one warp: 2 rows x 16 columns per thread with the 16x256b load shape
+    const int g = warp & 3;                   // TMEM lane quadrant: rows 32g .. 32g+31
+    const int sub = (warp - 2) >> 2;          // which 16 of them
+    const int qb = g >> 1;                    // which of the two query blocks these rows belong to
     const int tq = lane & 3;
-    const uint32_t tl0 = tbase + (static_cast<uint32_t>(g * 32) << 16);
-    const uint32_t tl16 = tbase + (static_cast<uint32_t>(g * 32 + 16) << 16);
+    const uint32_t tl = tbase + (static_cast<uint32_t>(g * 32 + sub * 16) << 16);
     const float sl2 = a.scale_log2;
     const int32_t* list = list_of[qb];
     bool ok = true;
 
     {  // the other query block's P columns of these rows stay zero for the whole kernel
-      const uint32_t z[32] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u,
-                              0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-      tmem_st32(tl0 + kColP + (1 - qb) * 32, z);
-      tmem_wait_st_regs(z);
+      const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      tmem_st16x256_x4(tl + kColP + (1 - qb) * 32, z);
+      tmem_wait_st_keep16(z);
     }
 
-    // value v[i][c]: row tr + 8i of the quadrant, column c of this thread within the step's 64
-    // columns of the query block: 32*(c/8) + 8*((c%8)/2) + 2*tq + c%2
+    // value v[i][c]: row tr + 8i of the warp's 16 rows, column c of this thread within the
+    // step's 64 columns of the query block: 32*(c/8) + 8*((c%8)/2) + 2*tq + c%2
     auto col_of = [&](int c) { return 32 * (c >> 3) + 8 * ((c & 7) >> 1) + 2 * tq + (c & 1); };
-    float mr[4], l[4];
+    float mr[2], l[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) mr[i] = -INFINITY, l[i] = 0.f;
+    for (int i = 0; i < 2; ++i) mr[i] = -INFINITY, l[i] = 0.f;
     if (a.flags & S3R_FLAG_TEST_TIMEOUT) ok = mbar_wait(&bars->never, 0, abort, lim);
 
     for (int t = 0; ok && t < ns; ++t) {
       if (!(ok = mbar_wait(&bars->s_full, t & 1, abort, lim))) break;
       tc_fence_after();
-      uint32_t r[4][16];
-      tmem_ld16x256_x4(tl0 + kColS + qb * 64, r[0]);
-      tmem_ld16x256_x4(tl16 + kColS + qb * 64, r[1]);
-      tmem_ld16x256_x4(tl0 + kColS + qb * 64 + 32, r[2]);
-      tmem_ld16x256_x4(tl16 + kColS + qb * 64 + 32, r[3]);
+      uint32_t r[2][16];
+      tmem_ld16x256_x4(tl + kColS + qb * 64, r[0]);
+      tmem_ld16x256_x4(tl + kColS + qb * 64 + 32, r[1]);
       tmem_wait_ld_n<16>(r[0]);
       tmem_wait_ld_n<16>(r[1]);
-      tmem_wait_ld_n<16>(r[2]);
-      tmem_wait_ld_n<16>(r[3]);
       tc_fence_before();
       __syncwarp();  // one arrival per warp: its lanes' TMEM loads have all completed
       if (lane == 0) mbar_arrive(&bars->s_empty);
-      float v[4][16];
+      float v[2][16];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
@@ -304,10 +341,8 @@ __global__ void __maxnreg__(128)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int c = hh * 8 + 2 * rep + e;
-            v[0][c] = __uint_as_float(r[2 * hh][4 * rep + e]);
-            v[1][c] = __uint_as_float(r[2 * hh][4 * rep + 2 + e]);
-            v[2][c] = __uint_as_float(r[2 * hh + 1][4 * rep + e]);
-            v[3][c] = __uint_as_float(r[2 * hh + 1][4 * rep + 2 + e]);
+            v[0][c] = __uint_as_float(r[hh][4 * rep + e]);
+            v[1][c] = __uint_as_float(r[hh][4 * rep + 2 + e]);
           }
       // columns whose slot holds no token: past the list, an out-of-range index, past L, or
       // outside a view's patch grid. A 64-slot step spans at most two selected blocks (b >= 32).
@@ -336,14 +371,14 @@ __global__ void __maxnreg__(128)
           }
 #pragma unroll
           for (int c = 0; c < 16; ++c)
-            if (!((bits >> col_of(c)) & 1ull)) v[0][c] = v[1][c] = v[2][c] = v[3][c] = -INFINITY;
+            if (!((bits >> col_of(c)) & 1ull)) v[0][c] = v[1][c] = -INFINITY;
         }
       }
       // row maxima of this step (the quad's 4 threads hold the same rows)
-      float tmax[4];
+      float tmax[2];
       bool move = false;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 2; ++i) {
         float m = fmax3(fmax3(v[i][0], v[i][1], v[i][2]), fmax3(v[i][3], v[i][4], v[i][5]),
                         fmax3(v[i][6], v[i][7], v[i][8]));
         m = fmax3(m, fmax3(v[i][9], v[i][10], v[i][11]), fmax3(v[i][12], v[i][13], v[i][14]));
@@ -356,31 +391,29 @@ __global__ void __maxnreg__(128)
       // P(t) may overwrite the P buffer (and O may be rescaled) once P*V of step t-1 completed
       if (!(ok = mbar_wait(&bars->p_empty, (t & 1) ^ 1, abort, lim))) break;
       if (__any_sync(0xffffffffu, move)) {  // rare after the first step: move references
-        float f[4];
+        float f[2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2; ++i) {
           const float mn = tmax[i] * sl2 > mr[i] * sl2 + kMoveRef ? tmax[i] : mr[i];
           f[i] = mr[i] == -INFINITY ? 0.f : exp2_approx((mr[i] - mn) * sl2);
           l[i] *= f[i];
           mr[i] = mn;
         }
-        if (t > 0) {  // O rows of this warp (lane = row) times the factor of their row
-          const int src = 4 * (lane & 7);  // a thread of the quad that holds row `lane`
-          const float f0 = __shfl_sync(0xffffffffu, f[0], src);
-          const float f1 = __shfl_sync(0xffffffffu, f[1], src);
-          const float f2 = __shfl_sync(0xffffffffu, f[2], src);
-          const float f3 = __shfl_sync(0xffffffffu, f[3], src);
-          const int which = lane >> 3;
-          const float fr = which == 0 ? f0 : which == 1 ? f1 : which == 2 ? f2 : f3;
+        if (t > 0) {  // the warp's O rows times the factor of their row, in the same layout
           tc_fence_after();
 #pragma unroll 1
-          for (int q4 = 0; q4 < 4; ++q4) {
+          for (int hh = 0; hh < 2; ++hh) {
             uint32_t o[16];
-            tmem_ld32x16(tl0 + kColO + 16 * q4, o);
+            tmem_ld16x256_x4(tl + kColO + 32 * hh, o);
             tmem_wait_ld_n<16>(o);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * fr);
-            tmem_st32x16(tl0 + kColO + 16 * q4, o);
+            for (int rep = 0; rep < 4; ++rep)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                o[4 * rep + e] = __float_as_uint(__uint_as_float(o[4 * rep + e]) * f[0]);
+                o[4 * rep + 2 + e] = __float_as_uint(__uint_as_float(o[4 * rep + 2 + e]) * f[1]);
+              }
+            tmem_st16x256_x4(tl + kColO + 32 * hh, o);
             tmem_wait_st_keep16(o);
           }
         }
@@ -389,18 +422,18 @@ __global__ void __maxnreg__(128)
       // the columns at a time. 16x128b store layout: repetition rep covers TMEM columns
       // 4rep..4rep+3 (keys 8rep.. of the half), lane tr -> register 2rep, lane tr+8 -> 2rep+1;
       // value columns (hh*8 + 2rep, +1) are exactly keys 32hh + 8rep + 2tq + {0,1}.
-      float off[4];
+      float off[2];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) off[i] = mr[i] == -INFINITY ? 0.f : -mr[i] * sl2;
+      for (int i = 0; i < 2; ++i) off[i] = mr[i] == -INFINITY ? 0.f : -mr[i] * sl2;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        uint32_t a0[8], a1[8];
+        uint32_t a0[8];
 #pragma unroll
         for (int rep = 0; rep < 4; ++rep) {
           const int c = hh * 8 + 2 * rep;
-          float e[4][2];
+          float e[2][2];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < 2; ++i) {
             const float2 x = __ffma2_rn(make_float2(v[i][c], v[i][c + 1]), make_float2(sl2, sl2),
                                         make_float2(off[i], off[i]));
             e[i][0] = exp2_approx(x.x);
@@ -409,57 +442,52 @@ __global__ void __maxnreg__(128)
           }
           a0[2 * rep] = pack_bf16(e[0][0], e[0][1]);
           a0[2 * rep + 1] = pack_bf16(e[1][0], e[1][1]);
-          a1[2 * rep] = pack_bf16(e[2][0], e[2][1]);
-          a1[2 * rep + 1] = pack_bf16(e[3][0], e[3][1]);
         }
         // keys 64*qb + 32*hh .. : TMEM columns 32*qb + 16*hh of the P region
-        tmem_st16x128_x4(tl0 + kColP + qb * 32 + hh * 16, a0);
-        tmem_st16x128_x4(tl16 + kColP + qb * 32 + hh * 16, a1);
+        tmem_st16x128_x4(tl + kColP + qb * 32 + hh * 16, a0);
         tmem_wait_st_keep8(a0);
-        tmem_wait_st_keep8(a1);
       }
       tc_fence_before();
       __syncwarp();  // one arrival per warp: its lanes' TMEM stores have all completed
       if (lane == 0) mbar_arrive(&bars->p_full);
     }
 
-    // finish: O / l per row (lane = row for the 32x32b loads), then write O_sel or the combine
+    // finish: O / l per row, then write O_sel or the combine. The 32x32b load gives lane = row
+    // of the quadrant; this warp writes the rows it owns (lanes 16*sub .. 16*sub+15).
     if (ok && (ok = mbar_wait(&bars->o_full, 0, abort, lim))) {
-      float lsum[4];
+      float lsum[2];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 2; ++i) {
         float s = l[i];
         s += __shfl_xor_sync(0xffffffffu, s, 1);
         s += __shfl_xor_sync(0xffffffffu, s, 2);
         lsum[i] = s;
       }
+      // row `lane` of the quadrant is held by lane 4*(lane%8) of warp sub = lane/16, as i = (lane/8)%2
       const int src = 4 * (lane & 7);
+      const bool hi = (lane >> 3) & 1;
       const float s0 = __shfl_sync(0xffffffffu, lsum[0], src);
       const float s1 = __shfl_sync(0xffffffffu, lsum[1], src);
-      const float s2 = __shfl_sync(0xffffffffu, lsum[2], src);
-      const float s3 = __shfl_sync(0xffffffffu, lsum[3], src);
-      const int which = lane >> 3;
-      const float rs = which == 0 ? s0 : which == 1 ? s1 : which == 2 ? s2 : s3;
+      const float rs = hi ? s1 : s0;
       const float inv = rs > 0.f ? 1.f / rs : 0.f;
+      const bool mine = (lane >> 4) == sub;
+      const int64_t row = q0 + g * 32 + lane;
       if (a.lse) {  // lse = (reference max * scale * log2 e + log2 of the row sum) * ln 2
         const float m0 = __shfl_sync(0xffffffffu, mr[0], src);
         const float m1 = __shfl_sync(0xffffffffu, mr[1], src);
-        const float m2 = __shfl_sync(0xffffffffu, mr[2], src);
-        const float m3 = __shfl_sync(0xffffffffu, mr[3], src);
-        const float mrow = which == 0 ? m0 : which == 1 ? m1 : which == 2 ? m2 : m3;
-        const int64_t lrow = q0 + g * 32 + lane;
-        if (lrow < a.L)
-          a.lse[static_cast<int64_t>(h) * a.L + lrow] =
+        const float mrow = hi ? m1 : m0;
+        if (mine && row < a.L)
+          a.lse[static_cast<int64_t>(h) * a.L + row] =
               rs > 0.f ? (mrow * sl2 + log2f(rs)) * kLn2 : -INFINITY;
       }
       tc_fence_after();
+      const uint32_t tq0 = tbase + (static_cast<uint32_t>(g * 32) << 16);
       uint32_t o[2][32];
-      tmem_ld32(tl0 + kColO, o[0]);
-      tmem_ld32(tl0 + kColO + 32, o[1]);
+      tmem_ld32(tq0 + kColO, o[0]);
+      tmem_ld32(tq0 + kColO + 32, o[1]);
       tmem_wait_ld_regs(o[0]);
       tmem_wait_ld_regs(o[1]);
-      const int64_t row = q0 + g * 32 + lane;
-      if (row < a.L) {
+      if (mine && row < a.L) {
         const int64_t at = (row * a.H + h) * 64;
         if (a.o_sel) {
           float4* dst = reinterpret_cast<float4*>(a.o_sel + at);
