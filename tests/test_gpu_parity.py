@@ -82,13 +82,16 @@ def test_topk_blocks_bit_exact(dev, name):
         np.testing.assert_array_equal(got, want)
 
 
-@pytest.mark.parametrize("k,forced", [(1, 0), (33, 0), (40, 5), (256, 0), (257, 3)])
+@pytest.mark.parametrize("k,forced", [(1, 0), (32, 0), (33, 0), (40, 5), (64, 0), (65, 2),
+                                     (128, 0), (129, 0), (256, 0), (257, 3)])
 def test_topk_adversarial_orders_bit_exact(dev, k, forced):
     """Score rows built against the streaming top-k: ascending scores (every element beats the
-    running k-th key, so the candidate buffer overflows and is cut again and again), descending,
-    all equal (the lowest indices win), a few distinct values repeated, and random. k = 257 takes
-    the block-wide radix-select kernel. Bit-exact against the oracle's top-k on the same fp32
-    values."""
+    running k-th key, so the candidate buffer overflows and is merged again and again),
+    descending, all equal (the lowest indices win), a few distinct values repeated, and random.
+    The k values take each size of the warp kernel's sorted list (32, 64, 128, 256) at and past
+    its bounds; k = 257 takes the block-wide radix-select kernel. Rows of 3001 scores start at
+    every 4-byte offset of a 16-byte line, so the unaligned head and tail are exercised.
+    Bit-exact against the oracle's top-k on the same fp32 values."""
     g = torch.Generator().manual_seed(100 + k)
     nb = 3001
     cfg = api.Config(L=nb * 32, H=1, block=32, topk=k, forced=forced)
