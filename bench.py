@@ -124,16 +124,16 @@ SM_COUNT = 148
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the kernel that bounds
 # the step at 1000 views: one ncu capture of that kernel on the 100-view layer (python bench.py
-# --workload n100 --steps 1 --warmup 3 --no-backward --no-cpu-baseline --no-dense-context; 290.8
-# MB read + 514.0 MB written), scaled by the ratio of rows (10.0: its traffic, Q read and O_cmp
+# --workload n100 --steps 1 --warmup 3 --no-backward --no-cpu-baseline --no-dense-context; 290.5
+# MB read + 513.2 MB written), scaled by the ratio of rows (10.0: its traffic, Q read and O_cmp
 # written, is proportional to L). With the SHA-256 of the sources that kernel was built from: once
 # any of them changes, the figure no longer describes the kernel and the roofline reports null.
 TRAFFIC = {
-    "cmp": {"workload": "n1000", "bytes": (290766080 + 514033920) * 10,
+    "cmp": {"workload": "n1000", "bytes": (290472704 + 513215744) * 10,
              "sources": ["sparse_global_attention_s3r_b200/csrc/cmp_attn_tc.cu",
                          "sparse_global_attention_s3r_b200/csrc/common.cuh",
                          "sparse_global_attention_s3r_b200/csrc/sm100.cuh"],
-             "sha256": "671e42957c5721277805d187ef85fba85fd85c18963b466fa8e0b7c350dcdf95"},
+             "sha256": "8828d658b7681ded38a8e6083a06784d26930157f351ac1ec61579703cd77c02"},
 }
 
 
