@@ -311,8 +311,7 @@ __device__ __forceinline__ void warp_bitonic_clean_desc(uint64_t* b, int lane) {
 
 // merge cand[0, cnt) into top (see above); returns the new theta
 template <int K2, int C>
-__device__ __forceinline__ uint64_t warp_merge(uint64_t* top, uint64_t* cand, int cnt, int k,
-                                               int) {
+__device__ __forceinline__ uint64_t warp_merge(uint64_t* top, uint64_t* cand, int cnt, int k) {
   // the lane index is re-read here so that the compiler does not keep the unrolled networks'
   // addresses live in registers across the whole scan
   int lane;
@@ -335,14 +334,14 @@ __device__ __forceinline__ uint64_t warp_merge(uint64_t* top, uint64_t* cand, in
 // unrolled networks are long enough that one shared copy, reached by a call, runs faster.
 template <int K2, int C>
 __device__ __noinline__ uint64_t warp_merge_call(uint64_t* top, uint64_t* cand, int cnt, int k) {
-  return warp_merge<K2, C>(top, cand, cnt, k, 0);
+  return warp_merge<K2, C>(top, cand, cnt, k);
 }
 template <int K2, int C>
-__device__ __forceinline__ uint64_t merge(uint64_t* top, uint64_t* cand, int cnt, int k, int lane) {
+__device__ __forceinline__ uint64_t merge(uint64_t* top, uint64_t* cand, int cnt, int k) {
   if constexpr (K2 >= 256)
     return warp_merge_call<K2, C>(top, cand, cnt, k);
   else
-    return warp_merge<K2, C>(top, cand, cnt, k, lane);
+    return warp_merge<K2, C>(top, cand, cnt, k);
 }
 
 template <int K2, int C>
@@ -373,7 +372,7 @@ __global__ void __launch_bounds__(kRowsPerCta * 32, S3R_TOPK_MIN_CTAS)
       pass = pass && key > theta;
       uint32_t m = __ballot_sync(0xffffffffu, pass);
       if (cnt + __popc(m) > C) {
-        theta = merge<K2, C>(top, cand, cnt, k, lane);
+        theta = merge<K2, C>(top, cand, cnt, k);
         cnt = 0;
         pass = pass && key > theta;
         m = __ballot_sync(0xffffffffu, pass);
@@ -453,7 +452,7 @@ __global__ void __launch_bounds__(kRowsPerCta * 32, S3R_TOPK_MIN_CTAS)
       const uint32_t xt = v ? __ldg(src + tail0 + lane) : 0u;
       if (__any_sync(0xffffffffu, v)) offer(xt, tail0 + lane, v);
     }
-    merge<K2, C>(top, cand, cnt, k, lane);
+    merge<K2, C>(top, cand, cnt, k);
     for (int e = lane; e < k; e += 32)
       out[e] = first + static_cast<int32_t>(~static_cast<uint32_t>(top[e] & 0xFFFFFFFFull));
     __syncwarp();  // the buffers are reused by the warp's next row
