@@ -132,11 +132,12 @@ Workspace layout(const Problem& p) {
 
 // Workspace of the backward call, every region 256-byte aligned:
 //   status | Kc | Vc | Kh | Vh (as the forward) | O_cmp, O_sel [L,H,d] f32 | lse_c, lse_s [H,L]
-//   | statistics [6][H][Lp] f32 | dKc, dVc [nb,H,d] f32 | cnt, cursor [H,nb] | off [H,nb+1]
+//   | statistics [6][H][Lp] f32 | dKc, dVc [nb,H,d] f32 | dKc, dVc partial sums of the pieces of
+//   the summaries' walk over the queries [2][C][nb,H,d] f32 (C > 1 only) | cnt, cursor [H,nb] | off [H,nb+1]
 //   | ent [H,nqb*nsel] | order [H*G] | hist, hcur [nqb+1] | hoff [nqb+2] i32
 struct BwdWorkspace {
-  size_t status, kc, vc, kh, vh, o_cmp, o_sel, lse_c, lse_s, stats, dkc, dvc, cnt, cursor, off,
-      ent, order, hist, hcur, hoff, total;
+  size_t status, kc, vc, kh, vh, o_cmp, o_sel, lse_c, lse_s, stats, dkc, dvc, dkv_part, cnt,
+      cursor, off, ent, order, hist, hcur, hoff, total;
 };
 
 BwdWorkspace bwd_ws_layout(const Problem& p) {
@@ -169,6 +170,7 @@ BwdWorkspace bwd_ws_layout(const Problem& p) {
   w.stats = take(6 * H * bl.Lp * 4);
   w.dkc = take(static_cast<size_t>(p.nb) * HD * 4);
   w.dvc = take(static_cast<size_t>(p.nb) * HD * 4);
+  w.dkv_part = bl.kv_chunks > 1 ? take(2 * static_cast<size_t>(bl.kv_chunks) * p.nb * HD * 4) : 0;
   w.cnt = take(H * p.nb * 4);
   w.cursor = take(H * p.nb * 4);
   w.off = take(H * (p.nb + 1) * 4);
@@ -419,8 +421,9 @@ s3r_status s3r_sparse_attn_bwd(const s3r_params* params, const s3r_bf16* q, cons
     return S3R_ERR_CUDA;
   BwdBuffers b{q, dout, b16(w.kc), b16(w.vc), b16(w.kh), b16(w.vh), gate_logits, f32(w.o_cmp),
                f32(w.o_sel), f32(w.lse_c), f32(w.lse_s), idx, f32(w.stats), f32(w.dkc),
-               f32(w.dvc), i32(w.cnt), i32(w.cursor), i32(w.off), i32(w.ent), i32(w.order),
-               i32(w.hist), i32(w.hcur), i32(w.hoff), dq, dk, dv, dgates};
+               f32(w.dvc), bwd_layout(p).kv_chunks > 1 ? f32(w.dkv_part) : nullptr, i32(w.cnt),
+               i32(w.cursor), i32(w.off), i32(w.ent), i32(w.order), i32(w.hist), i32(w.hcur),
+               i32(w.hoff), dq, dk, dv, dgates};
   return launched(launch_bwd(p, b, stream, ev));
 }
 

@@ -567,6 +567,8 @@ struct BwdKVArgs {
   float* out_k;         // !kSel: dKc [nb, H, 64]; kSel: dk [L, H, 64]
   float* out_v;
   int64_t L, Lp, nb, nqb, kv_rows, per_head, G;  // kSel: G groups per head
+  int64_t chunk_steps;  // !kSel: 64-query steps of one piece of the walk (blockIdx.z = piece)
+  int64_t part_stride;  // !kSel: elements between the pieces' outputs (0: one piece)
   BlockGeo geo;
   int H, b, cpb;        // cpb: 64-slot groups per key block
   float scale, scale_log2;
@@ -617,9 +619,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     nsteps = 2 * (glen[0] > glen[1] ? glen[0] : glen[1]);
-  } else {
-    nsteps = static_cast<int>((a.L + 63) / 64);
+  } else {  // piece blockIdx.z of the walk over the queries
+    const int64_t all = (a.L + 63) / 64, t0 = static_cast<int64_t>(blockIdx.z) * a.chunk_steps;
+    nsteps = static_cast<int>(all - t0 < a.chunk_steps ? all - t0 : a.chunk_steps);
   }
+  const int64_t qt0 = kSel ? 0 : static_cast<int64_t>(blockIdx.z) * a.chunk_steps;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -692,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             bulk_load(sd + 256, s0 + kDS * plane, 128, full);
           }
         } else {  // 64 consecutive queries
-          const int64_t row0 = static_cast<int64_t>(t) * 64;
+          const int64_t row0 = (qt0 + t) * 64;
           tma_load_2d(sq, &tmQ, h * 64, static_cast<int32_t>(row0), full);
           tma_load_2d(sq + kQTile, &tmO, h * 64, static_cast<int32_t>(row0), full);
           const float* s0 = a.stats + static_cast<int64_t>(h) * a.Lp + row0;
@@ -862,7 +866,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       } else {
         const int64_t j = static_cast<int64_t>(blockIdx.x) * 128 + row;
         if (j < a.nb) {
-          const int64_t dst = (j * a.H + h) * 64 + 32 * half;
+          const int64_t dst =
+              static_cast<int64_t>(blockIdx.z) * a.part_stride + (j * a.H + h) * 64 + 32 * half;
           float4* k4 = reinterpret_cast<float4*>(a.out_k + dst);
           float4* v4 = reinterpret_cast<float4*>(a.out_v + dst);
 #pragma unroll
@@ -883,6 +888,22 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 1) tmem_dealloc(tbase, kTmemCols);
 }
 
+// dKc, dVc = the sum of the pieces' partial sums, added in piece order (part: [2][chunks][n/4])
+__global__ void dkv_reduce_kernel(const float4* __restrict__ part, float4* __restrict__ dkc,
+                                  float4* __restrict__ dvc, int64_t n4, int chunks) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < 2 * n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t which = i >= n4 ? 1 : 0, j = i - which * n4;
+    const float4* src = part + which * chunks * n4 + j;
+    float4 s = src[0];
+    for (int c = 1; c < chunks; ++c) {
+      const float4 x = src[c * n4];
+      s = make_float4(s.x + x.x, s.y + x.y, s.z + x.z, s.w + x.w);
+    }
+    (which ? dvc : dkc)[j] = s;
+  }
+}
+
 template <typename K>
 cudaError_t prepare(K kernel, uint32_t smem) {
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -899,6 +920,25 @@ BwdLayout bwd_layout(const Problem& p) {
   w.per_head = p.nqb * p.nsel;
   w.cpb = p.b > 64 ? p.b / 64 : 1;
   w.G = p.nb * w.cpb;
+  // The dKc/dVc kernel runs one CTA per 128 summaries and head, each walking every query. When
+  // those CTAs fill the last wave of a B200 (148 SMs x 2 resident CTAs) poorly, the walk is split
+  // into c pieces of at least 32 steps: the smallest c up to 16 whose waves are at least 95 %
+  // full, else the one that fills them best. The pieces' partial sums are added in order.
+  const int64_t tiles = (p.nb + 127) / 128 * p.H, steps = (p.L + 63) / 64;
+  constexpr int64_t kResident = 2 * 148;
+  int best = 1;
+  int64_t best_num = 0, best_den = 1;  // fill of the best c so far, as a fraction
+  for (int c = 1; c <= 16 && (c == 1 || (steps + c - 1) / c >= 32); ++c) {
+    const int64_t ctas = c * tiles, waves = (ctas + kResident - 1) / kResident;
+    const int64_t num = ctas, den = waves * kResident;  // fill = ctas / (waves * resident)
+    if (100 * num >= 95 * den) {
+      best = c;
+      break;
+    }
+    if (num * best_den > best_num * den) best = c, best_num = num, best_den = den;
+  }
+  w.kv_chunk_steps = (steps + best - 1) / best;
+  w.kv_chunks = static_cast<int>((steps + w.kv_chunk_steps - 1) / w.kv_chunk_steps);
   return w;
 }
 
@@ -983,13 +1023,28 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& B, cudaStream_t st,
         !make_tmap_head_rows(&to, B.dout, p.L, p.H, 64))
       return cudaErrorInvalidValue;
     if ((e = prepare(bwd_kv_kernel<false>, kv_outer::kSmemBytes)) != cudaSuccess) return e;
-    BwdKVArgs a{B.stats, nullptr, nullptr, nullptr, nullptr, nullptr, B.dkc, B.dvc, p.L, w.Lp, p.nb,
-                p.nqb, kv_rows, w.per_head, 0, p.geo, p.H, p.b, 1, p.scale, p.scale_log2,
-                p.status, lim, p.flags};
-    dim3 grid(static_cast<unsigned>((p.nb + 127) / 128), p.H);
+    // with several pieces, each writes its partial sums to the scratch, added in order below
+    const int64_t n = p.nb * p.H * 64;
+    const bool pieces = w.kv_chunks > 1;
+    if (pieces && !B.dkv_part) return cudaErrorInvalidValue;
+    float* out_k = pieces ? B.dkv_part : B.dkc;
+    float* out_v = pieces ? B.dkv_part + w.kv_chunks * n : B.dvc;
+    BwdKVArgs a{B.stats, nullptr, nullptr, nullptr, nullptr, nullptr, out_k, out_v, p.L, w.Lp,
+                p.nb, p.nqb, kv_rows, w.per_head, 0, w.kv_chunk_steps, pieces ? n : 0, p.geo, p.H,
+                p.b, 1, p.scale, p.scale_log2, p.status, lim, p.flags};
+    dim3 grid(static_cast<unsigned>((p.nb + 127) / 128), p.H, w.kv_chunks);
     bwd_kv_kernel<false><<<grid, kThreads, kv_outer::kSmemBytes, st>>>(tkc, tvc, tq, to, a);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (pieces) {
+      const int64_t n4 = n / 4;
+      const int64_t blocks = (2 * n4 + 255) / 256;
+      dkv_reduce_kernel<<<static_cast<unsigned>(blocks < 8192 ? blocks : 8192), 256, 0, st>>>(
+          reinterpret_cast<const float4*>(B.dkv_part), reinterpret_cast<float4*>(B.dkc),
+          reinterpret_cast<float4*>(B.dvc), n4, w.kv_chunks);
+      count_launch();
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
   }
   stage_range_pop(p);
   if ((e = mark(4)) != cudaSuccess) return e;
@@ -1003,8 +1058,8 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& B, cudaStream_t st,
       return cudaErrorInvalidValue;
     if ((e = prepare(bwd_kv_kernel<true>, kv_outer::kSmemBytes)) != cudaSuccess) return e;
     BwdKVArgs a{B.stats, B.off, B.ent, B.order, B.dkc, B.dvc, B.dk, B.dv, p.L, w.Lp, p.nb,
-                p.nqb, kv_rows, w.per_head, w.G, p.geo, p.H, p.b, w.cpb, p.scale, p.scale_log2,
-                p.status, lim, p.flags};
+                p.nqb, kv_rows, w.per_head, w.G, 0, 0, p.geo, p.H, p.b, w.cpb, p.scale,
+                p.scale_log2, p.status, lim, p.flags};
     dim3 grid(static_cast<unsigned>((w.G * p.H + 1) / 2), 1);
     bwd_kv_kernel<true><<<grid, kThreads, kv_outer::kSmemBytes, st>>>(tkh, tvh, tq, to, a);
     count_launch();

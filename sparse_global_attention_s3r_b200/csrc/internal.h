@@ -62,6 +62,8 @@ struct BwdLayout {
   int64_t per_head;  // entries of one head's selection lists: nqb * nsel
   int cpb;           // 64-slot groups per key block (token-side kernel)
   int64_t G;         // groups per head: nb * cpb
+  int kv_chunks;     // pieces the dKc/dVc kernel's walk over the queries is split into
+  int64_t kv_chunk_steps;  // 64-query steps of one piece
 };
 BwdLayout bwd_layout(const Problem& p);
 struct BwdBuffers {
@@ -70,6 +72,7 @@ struct BwdBuffers {
   const int32_t* idx;     // [H, nqb, nsel]
   float* stats;           // [6][H][Lp] scratch
   float *dkc, *dvc;       // [nb, H, 64] scratch
+  float* dkv_part;        // [2][kv_chunks][nb, H, 64] scratch, null when kv_chunks == 1
   int32_t *cnt, *cursor;  // [H, nb] scratch
   int32_t* off;           // [H, nb + 1] scratch
   int32_t* ent;           // [H, per_head] scratch

@@ -125,6 +125,34 @@ def test_workspace_checks():
         assert lib.s3r_sparse_attn_bwd(p, *[A16] * 10, ws, n, None) == _lib.S3R_ERR_WORKSPACE
 
 
+def kv_chunks(L, H, b):
+    """Pieces of the dKc/dVc kernel's walk over the queries: the smallest c <= 16 (pieces of at
+    least 32 64-query steps) whose CTAs fill the waves of 148 SMs x 2 resident CTAs to 95 %, else
+    the best-filling c; then as many pieces as ceil(steps / ceil(steps / c))."""
+    nb = -(-L // b)
+    tiles, steps, res = -(-nb // 128) * H, -(-L // 64), 2 * 148
+    best, best_fill = 1, 0.0
+    for c in range(1, 17):
+        if c > 1 and -(-steps // c) < 32:
+            break
+        ctas = c * tiles
+        fill = ctas / (-(-ctas // res) * res)
+        if 100 * ctas >= 95 * (-(-ctas // res) * res):
+            best = c
+            break
+        if fill > best_fill:
+            best, best_fill = c, fill
+    per = -(-steps // best)
+    return -(-steps // per)
+
+
+def test_kv_chunks_at_the_workload_sizes():
+    # 1000 views: 2688 CTAs fill 9.08 waves, 18.16 in two pieces; 100 views: 272 CTAs
+    assert kv_chunks(1374000, 16, 64) == 2
+    assert kv_chunks(137400, 16, 64) == 13
+    assert kv_chunks(1, 2, 32) == 1
+
+
 @pytest.mark.parametrize("L,H,b,k,F", [(1024, 2, 64, 4, 0), (1374000, 16, 64, 32, 0),
                                        (43968, 16, 64, 16, 22), (1, 1, 128, 1, 0)])
 def test_bwd_workspace_size_matches_layout(L, H, b, k, F):
@@ -136,6 +164,9 @@ def test_bwd_workspace_size_matches_layout(L, H, b, k, F):
             + 2 * r256(nb * H * d * 4) + 2 * r256(H * nb * 4) + r256(H * (nb + 1) * 4)
             + r256(H * nqb * (F + k) * 4) + r256(H * nb * max(1, b // 64) * 4)
             + 2 * r256((nqb + 1) * 4) + r256((nqb + 2) * 4))
+    c = kv_chunks(L, H, b)
+    if c > 1:  # the pieces' partial dKc, dVc
+        want += r256(2 * c * nb * H * d * 4)
     assert api.bwd_workspace_bytes(cfg) == want
 
 
@@ -154,6 +185,9 @@ def test_save_for_backward_workspaces(L, H, b, k):
     scratch = (r256(6 * H * Lp * 4) + 2 * r256(nb * H * 64 * 4) + 2 * r256(H * nb * 4)
                + r256(H * (nb + 1) * 4) + r256(H * nqb * k * 4) + r256(H * nb * max(1, b // 64) * 4)
                + 2 * r256((nqb + 1) * 4) + r256((nqb + 2) * 4))
+    c = kv_chunks(L, H, b)
+    if c > 1:
+        scratch += r256(2 * c * nb * H * 64 * 4)
     assert api.bwd_workspace_bytes(save) == fwd_s + scratch
     lib = _lib.load()
     p = ctypes.byref(save.params())
