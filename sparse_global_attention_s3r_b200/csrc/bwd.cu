@@ -28,7 +28,9 @@
 //                      S^T = K Q^T, dP'^T = V dout^T, then (g P)^T and dS^T are written in place
 //                      over S^T and dP'^T as bf16 and dV += (gP)^T dout, dK += dS^T Q.
 //                      <false>: the 128 rows are block summaries, every query is a column
-//                      (writes dKc, dVc); <true>: rows are two 64-slot groups of key blocks
+//                      (writes dKc, dVc); the walk over the queries may be split into pieces
+//                      (grid z) whose partial sums dkv_reduce_kernel adds in piece order;
+//                      <true>: rows are two 64-slot groups of key blocks
 //                      (neighbours in the longest-first order, of any heads), each walking the
 //                      query blocks that selected its block, 32 rows of one per step
 //                      (block-diagonal); writes dk, dv per token and adds the pooled gradients

@@ -3,8 +3,8 @@
 // Speed3R (gist.science summary, "Methodologie" §1 "Selectie-tak"): the selection branch attends
 // to the top-k blocks chosen by the compression branch's scores. Ties go to the lower block index.
 //
-// Two kernels. For k <= kWarpTopkMax (every default configuration), topk_warp_kernel streams each
-// row once through one warp (see there). Larger k use topk_kernel:
+// Two kernels. For k <= kWarpTopkMax (256), topk_warp_kernel streams each row once through one
+// warp (see there). Larger k use topk_kernel:
 // One CTA per score row [nb] (one query block of one head). Scores are probabilities summed over
 // rows, so they are non-negative and their fp32 bit patterns order like unsigned integers; the
 // 64-bit key (bits << 32 | ~index) orders by descending score, then ascending index, and is unique.
