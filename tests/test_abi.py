@@ -151,6 +151,7 @@ def test_kv_chunks_at_the_workload_sizes():
     assert kv_chunks(1374000, 16, 64) == 2
     assert kv_chunks(137400, 16, 64) == 13
     assert kv_chunks(1, 2, 32) == 1
+    assert kv_chunks(40000, 1, 64) == 16  # the backward parity case of the most pieces
 
 
 @pytest.mark.parametrize("L,H,b,k,F", [(1024, 2, 64, 4, 0), (1374000, 16, 64, 32, 0),

@@ -36,6 +36,9 @@ CASES = {  # name: (L, H, b, k, forced, seed)
     "tail_of_one_row": (65, 1, 32, 3, 0, 48),
     "forced_b32": (2000, 2, 32, 5, 6, 49),        # reference-frame blocks in every list
     "vggt_4_views": (4 * 1374, 2, 64, 16, 22, 50),
+    # 8 summary tiles of one head: the dKc/dVc kernel splits its walk over the queries into the
+    # most pieces it takes, 16, added back in order
+    "sixteen_pieces": (40000, 1, 64, 8, 0, 58),
 }
 
 WINDOWS = {  # name: (views, special, grid_h, grid_w, b, win_h, H, k, forced_views, seed)
