@@ -76,7 +76,8 @@ typedef enum {
 #define S3R_DEV_BAD_INDEX 0x2u /* (debug checks) an idx entry was outside [0, nb) */
 
 /* params.flags */
-#define S3R_FLAG_DEBUG_CHECKS 0x1u /* validate idx on the device in s3r_sel_attn */
+#define S3R_FLAG_DEBUG_CHECKS 0x1u /* validate idx on the device in s3r_sel_attn and
+                                     s3r_sparse_attn_bwd */
 #define S3R_FLAG_TEST_TIMEOUT 0x2u /* testing only: the tensor-core kernels (compressed branch,
                                       selection, the single fused kernel, and the backward's dq,
                                       dKc/dVc and dk/dv kernels) wait on a barrier that nothing
@@ -256,7 +257,8 @@ s3r_status s3r_sparse_attn_fwd(const s3r_params* params, const s3r_bf16* q, cons
  * the workspace, then runs the backward kernels; nothing is kept between calls.
  *   q, k, v     [L, H, d] bf16; gate_logits [L, H, 2] fp32; dout [L, H, d] bf16 (read)
  *   idx         [H, nqb, forced + topk] int32 (read): entries distinct within a list; entries
- *               outside [0, nb) contribute nothing
+ *               outside [0, nb) contribute nothing (with S3R_FLAG_DEBUG_CHECKS they also raise
+ *               S3R_DEV_BAD_INDEX)
  *   dq, dk, dv  [L, H, d] fp32 (written); dgates [L, H, 2] fp32 (written)
  *   workspace   device buffer of at least s3r_bwd_workspace_bytes(params) bytes, 256-byte aligned.
  * Returns S3R_ERR_UNSUPPORTED when H * nb * block exceeds 2^31 - 1 (row coordinates of the

@@ -153,13 +153,20 @@ __global__ void bwd_prep_kernel(const uint16_t* __restrict__ dout, const float* 
 // ------------------------------------------------------------------------------------------
 // the inverse of the selection lists (per head, CSR over key blocks)
 // ------------------------------------------------------------------------------------------
+// Every list entry passes through here once: an entry outside [0, nb) is skipped (its block
+// gets no gradient from that query block) and, with S3R_FLAG_DEBUG_CHECKS, raises
+// S3R_DEV_BAD_INDEX in the status word.
 __global__ void csr_count_kernel(const int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
-                                 int64_t per_head, int64_t total, int64_t nb) {
+                                 int64_t per_head, int64_t total, int64_t nb, uint32_t flags,
+                                 uint32_t* status) {
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t h = e / per_head;
     const int32_t j = idx[e];
-    if (j >= 0 && j < nb) atomicAdd(cnt + h * nb + j, 1);
+    if (j >= 0 && j < nb)
+      atomicAdd(cnt + h * nb + j, 1);
+    else if ((flags & S3R_FLAG_DEBUG_CHECKS) && status)
+      set_status(status, S3R_DEV_BAD_INDEX);
   }
 }
 
@@ -969,7 +976,8 @@ cudaError_t launch_bwd(const Problem& p, const BwdBuffers& B, cudaStream_t st,
     const int64_t total = p.H * w.per_head;
     const unsigned blocks = static_cast<unsigned>((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
     if ((e = cudaMemsetAsync(B.cnt, 0, sizeof(int32_t) * p.H * p.nb, st)) != cudaSuccess) return e;
-    csr_count_kernel<<<blocks, 256, 0, st>>>(B.idx, B.cnt, w.per_head, total, p.nb);
+    csr_count_kernel<<<blocks, 256, 0, st>>>(B.idx, B.cnt, w.per_head, total, p.nb, p.flags,
+                                             p.status);
     count_launch();
     csr_scan_kernel<<<p.H, 1024, 0, st>>>(B.cnt, B.off, B.cursor, p.nb);
     count_launch();

@@ -174,6 +174,32 @@ def test_bwd_from_saved_forward(dev, name):
         torch.testing.assert_close(got, other, rtol=1e-5, atol=1e-6)
 
 
+def test_bwd_debug_checks_flag_bad_indices(dev):
+    """A list entry outside [0, nb) is skipped by the backward and, with debug checks, raises
+    S3R_DEV_BAD_INDEX in the caller's status word; without them the word stays clear."""
+    import dataclasses
+
+    from sparse_global_attention_s3r_b200 import _lib
+
+    L, H, b, k, F, seed = CASES["ragged_b64"]
+    x = synth.make_inputs(L, H, 64, b, seed)
+    cfg = api.Config(L=L, H=H, block=b, topk=k)
+    d = {n: getattr(x, n).to(dev) for n in ("q", "k", "v", "gates")}
+    idx = torch.empty((H, cfg.nqb, cfg.nsel), dtype=torch.int32, device=dev)
+    api.sparse_attn_fwd(cfg, d["q"], d["k"], d["v"], d["gates"], idx_out=idx)
+    idx[0, 3, 1] = cfg.nb + 7
+    dout = _dout(L, H, seed).to(dev)
+    word = torch.zeros(1, dtype=torch.int32, device=dev)
+    api.sparse_attn_bwd(cfg, d["q"], d["k"], d["v"], d["gates"], idx, dout, dev_status=word)
+    assert api.read_device_status(word) == 0
+    checked = dataclasses.replace(cfg, debug_checks=True)
+    grads = api.sparse_attn_bwd(checked, d["q"], d["k"], d["v"], d["gates"], idx, dout,
+                                dev_status=word)
+    assert api.read_device_status(word) & _lib.S3R_DEV_BAD_INDEX
+    for g in grads:
+        assert torch.isfinite(g).all()
+
+
 def test_bwd_status_word_stays_clear(dev):
     L, H, b, k = 1000, 2, 64, 4
     x = synth.make_inputs(L, H, 64, b, 57)
